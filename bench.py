@@ -1,0 +1,351 @@
+#!/usr/bin/env python
+"""Benchmark of the causal sequence convolution on B200.
+
+One step = one call of the fused causal convolution (load, pad, FFT, spectral
+product, inverse FFT, truncate, store) over one batch of the named workload
+(default: the Caracal-Small-shaped fp32 MHF convolution, B=8, L=1024, D=768).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+For N > 1 launch under torchrun: every rank convolves its own batch (its own
+seed) on its own GPU with no collective on the data path (weak scaling);
+timing is the max over ranks.  Prints one JSON line on rank 0.
+
+Timing: inputs larger than L2 -- the step rotates through enough copies of
+(v, g, r) that each step touches buffers last used more than 126 MB of traffic
+ago; CUDA events on the launching stream bracket the K timed steps, with a
+barrier and a device synchronize on both sides.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "causal FFT-conv GB/s and (B*D*L)/s at 1 B200; % of HBM roofline"
+L2_BYTES = 126 * 2 ** 20
+KERNEL_SOURCES = ["fftconv_fused.cuh", "fft_reg.cuh", "ntt.cuh", "api.cu"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="small_f32", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        p = os.path.join(ROOT, "spectral_sequence_mixing_b200", "csrc", f)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """dram bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d.get(workload, {})
+        if e.get("kernel") == kernel and e.get("source_hash") == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self._stop = threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                mask = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join()
+
+    def report(self):
+        if self._nv is None:
+            return None
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
+
+
+def cpu_oracle_rate(w: workloads.Workload, v, g, budget_s: float):
+    """Time the oracle on whole rows of the workload: channel slices [B, L, k]
+    with k doubling until about budget_s of CPU work.  Returns (units/s,
+    threads, description, seconds)."""
+    import oracle
+    fv = workloads.bf16_to_f32(v) if w.dtype == "bf16" else v
+    fg = workloads.bf16_to_f32(g) if w.dtype == "bf16" else g
+    k, spent, units, secs = 1, 0.0, 0, 0.0
+    while True:
+        k = min(k, w.D)
+        sv = np.ascontiguousarray(fv[:, :, :k])
+        sg = np.ascontiguousarray(fg[:, :, :k])
+        t0 = time.perf_counter()
+        if w.dtype == "i32":
+            oracle.causal_conv_int(sv, sg)
+        else:
+            oracle.causal_conv(sv, sg)
+        dt = time.perf_counter() - t0
+        units, secs = w.B * w.L * k, dt
+        spent += dt
+        if spent >= budget_s / 3 or k == w.D or dt * 2 > budget_s - spent:
+            break
+        k *= 2
+    desc = f"oracle on channels [0,{k}) of {w.name}: {w.B}x{w.L}x{k} = {units} outputs (whole rows)"
+    return units / secs, oracle.num_threads(), desc, secs
+
+
+def run_reference(args, rank, world):
+    """The oracle (plain CPU direct sum) timed on the host cores as the
+    reference arm, on the same workload and metric."""
+    if rank != 0:
+        return
+    w = workloads.WORKLOADS[args.workload]
+    v, g = workloads.generate(w)
+    per_step = max(0.05, 120.0 / max(1, args.steps + args.warmup))
+    import oracle
+    fv = workloads.bf16_to_f32(v) if w.dtype == "bf16" else v
+    fg = workloads.bf16_to_f32(g) if w.dtype == "bf16" else g
+    # calibrate the channel count k per step against the per-step budget
+    k = 1
+    while True:
+        t0 = time.perf_counter()
+        sv, sg = np.ascontiguousarray(fv[:, :, :k]), np.ascontiguousarray(fg[:, :, :k])
+        (oracle.causal_conv_int if w.dtype == "i32" else oracle.causal_conv)(sv, sg)
+        dt = time.perf_counter() - t0
+        if dt * 2 > per_step or k >= w.D:
+            break
+        k = min(w.D, k * 2)
+    sv, sg = np.ascontiguousarray(fv[:, :, :k]), np.ascontiguousarray(fg[:, :, :k])
+    fn = oracle.causal_conv_int if w.dtype == "i32" else oracle.causal_conv
+    for _ in range(args.warmup):
+        fn(sv, sg)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        fn(sv, sg)
+    el = time.perf_counter() - t0
+    units = w.B * w.L * k * args.steps
+    gbs = units * 3 * w.elem_bytes / el / 1e9
+    sample = f"oracle on channels [0,{k}) of {w.name} per step ({w.B}x{w.L}x{k} outputs, whole rows)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": {"f32": "f64", "bf16": "f64", "i32": "int64"}[w.dtype], "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "L": w.L, "D": w.D, "io_dtype": w.dtype},
+        "outputs_per_s": units / el,
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    w = workloads.WORKLOADS[args.workload]
+    v_np, g_np = workloads.generate(w, seed=w.seed + 1000 * rank)
+    tdt = {"f32": torch.float32, "bf16": torch.bfloat16, "i32": torch.int32}[w.dtype]
+
+    def to_t(x):
+        if w.dtype == "bf16":
+            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16)
+        return torch.from_numpy(x)
+
+    hv, hg = to_t(v_np), to_t(g_np)
+    v0, g0 = hv.to(dev), hg.to(dev)
+    set_bytes = 3 * w.units * w.elem_bytes
+    n_sets = max(2, math.ceil(2.2 * L2_BYTES / set_bytes))
+    sets = [(v0, g0, torch.empty_like(v0))] + [(v0.clone(), g0.clone(), torch.empty_like(v0)) for _ in
+                                                range(n_sets - 1)]
+    stream = torch.cuda.current_stream(dev)
+    fn = ssm.causal_conv
+
+    for i in range(args.warmup):
+        a, b, c = sets[i % n_sets]
+        fn(a, b, out=c, stream=stream)
+    torch.cuda.synchronize(dev)
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for i in range(args.steps):
+            a, b, c = sets[i % n_sets]
+            fn(a, b, out=c, stream=stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    ms = start.elapsed_time(end)
+    if pg is not None:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    units_total = w.units * world * args.steps
+    gbs = units_total * 3 * w.elem_bytes / (ms * 1e-3) / 1e9
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    phv, phg = hv.pin_memory(), hg.pin_memory()
+    phr = torch.empty_like(phv).pin_memory()
+    dv, dg, dr = sets[0]
+    for _ in range(2):
+        ssm.causal_conv_from_host(phv, phg, phr, dv, dg, dr, stream=stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        ssm.causal_conv_from_host(phv, phg, phr, dv, dg, dr, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ems = e0.elapsed_time(e1)
+    if pg is not None:
+        t = torch.tensor([ems], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ems = float(t.item())
+    e2e_gbs = w.units * world * e2e_steps * 3 * w.elem_bytes / (ems * 1e-3) / 1e9
+
+    peak, peak_src = measured_peaks()
+    kernel = {"f32": "fftconv_fused_kernel", "bf16": "fftconv_fused_kernel", "i32": "ntt_conv_kernel"}[w.dtype]
+    per_launch_bytes = 3 * w.units * w.elem_bytes
+    achieved = per_launch_bytes / (ms_per_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": {"f32": "f32", "bf16": "f32", "i32": "u32"}[w.dtype], "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "L": w.L, "D": w.D, "io_dtype": w.dtype,
+                   "transform_len": 2 ** math.ceil(math.log2(2 * w.L)),
+                   "l2": f"inputs larger than L2: {n_sets} rotating (v,g,r) sets of {set_bytes / 2 ** 20:.0f} MiB",
+                   "parallelism": f"dp{world} (independent batches, no collective)"},
+        "outputs_per_s": units_total / (ms * 1e-3),
+        "hbm_frac": gbs / world / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
+                     "kernel": kernel, "algorithmic_bytes_per_launch": per_launch_bytes,
+                     "traffic": recorded_traffic(w.name, kernel)},
+        "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": 2 * w.units * w.elem_bytes,
+                "d2h_bytes_per_step": w.units * w.elem_bytes, "steps": e2e_steps,
+                "path": "causal_conv_from_host (pinned host buffers)"},
+        "gpu_launches": args.steps,
+        "clocks": clk.report(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ups, cores, desc, secs = cpu_oracle_rate(w, v_np, g_np, budget_s=15.0)
+        line["cpu_baseline"] = {"value": ups * 3 * w.elem_bytes / 1e9, "unit": "GB/s", "cores": cores,
+                                "kind": "oracle", "sample": desc, "seconds": secs}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_env()
+    if world != args.gpus and "RANK" in os.environ:
+        print(f"warning: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,152 @@
+/*
+ * causalconv.h -- C ABI of the B200 (sm_100a) causal sequence convolution.
+ *
+ * Operation (Caracal: Causal Architecture via Spectral Mixing, "Key design 1:
+ * Multi-Head Fourier module" and "Key design 2: frequency-domain causal
+ * mask"): for every batch b and channel d of channel-last tensors,
+ *
+ *     r[b, t, d] = sum_{j=0..t} v[b, j, d] * g[b, t-j, d],     0 <= t < L,
+ *
+ * computed the way the pages describe: each (b, d) row is zero-padded to
+ * N >= 2L, Fourier-transformed, multiplied pointwise, inverse-transformed and
+ * truncated to its first L entries.  x_v (value stream) and x_g (gate stream)
+ * of the Multi-Head Fourier module are v and g here.
+ *
+ * Layout: v, g and r are contiguous row-major [B, L, D] arrays ("channel
+ * last"): element (b, t, d) is at index (b*L + t)*D + d.
+ *
+ * Ownership and execution: every pointer named *_dev or taken by the three
+ * conv entry points is a DEVICE pointer on the calling thread's current CUDA
+ * device, owned by the caller.  Work is enqueued on `stream` (a cudaStream_t;
+ * NULL = the legacy default stream) and the call returns without
+ * synchronising.  The library never allocates device memory on these calls;
+ * its small twiddle/constant tables are static device arrays filled once per
+ * device on the first call (that first call synchronises `stream` once).
+ *
+ * Errors: every argument check runs on the host before any launch; a failed
+ * check returns a non-zero cc_status and enqueues nothing.  CC_ERR_CUDA means
+ * a CUDA API call or the launch itself failed (cudaGetLastError after launch).
+ * Errors raised later by the asynchronous kernel surface at the caller's next
+ * synchronisation, as with any CUDA kernel.
+ */
+#ifndef CAUSALCONV_H
+#define CAUSALCONV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CC_API __attribute__((visibility("default")))
+#else
+#define CC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CC_OK = 0,
+    CC_ERR_INVALID_ARG = 1, /* null pointer, B/L/D < 1, size overflow, bad dtype */
+    CC_ERR_UNSUPPORTED = 2, /* L beyond the supported range for this dtype      */
+    CC_ERR_ALIAS = 3,       /* r overlaps v or g                                */
+    CC_ERR_WORKSPACE = 4,   /* workspace smaller than causal_conv_workspace_bytes */
+    CC_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed      */
+    CC_ERR_NOT_DEVICE = 6   /* a pointer is not device memory of the current device */
+} cc_status;
+
+typedef enum {
+    CC_DTYPE_F32 = 0,  /* float32 in, float32 out, float32 arithmetic        */
+    CC_DTYPE_BF16 = 1, /* bfloat16 in/out (uint16 bit patterns), float32 arithmetic */
+    CC_DTYPE_I32 = 2   /* int32 in/out, exact arithmetic mod p = 2013265921   */
+} cc_dtype;
+
+/*
+ * causal_fftconv_f32 -- float32 causal convolution via a fused
+ * pad -> FFT -> multiply -> inverse FFT -> truncate kernel.
+ *
+ *   v, g  [B, L, D] float32 inputs (device).   r  [B, L, D] float32 output
+ *   (device), must not overlap v or g.  B, L, D >= 1.
+ *   workspace / workspace_bytes: device scratch of at least
+ *   causal_conv_workspace_bytes(CC_DTYPE_F32, B, L, D) bytes (0 for every
+ *   supported L today; pass NULL, 0).
+ *
+ * Accuracy: |r - r_exact| <= 1e-5 * sum_j |v_j g_{t-j}| per element on the
+ * tested workloads; outputs with t < 32 are summed directly (no transform),
+ * because the rounding error of a float transform is spread evenly over a row
+ * and exceeds that per-element bound where the exact sum is tiny
+ * ("Catastrophic Token Leakage in Convolutional Sequence Modeling", TL;DR).
+ * Supported: 1 <= L <= 65536.
+ */
+CC_API int causal_fftconv_f32(const float *v, const float *g, float *r,
+                       int64_t B, int64_t L, int64_t D,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * causal_fftconv_bf16 -- as causal_fftconv_f32 with bfloat16 inputs and
+ * output (raw 16-bit patterns), float32 transform arithmetic and
+ * round-to-nearest-even on the output.  Supported: 1 <= L <= 65536.
+ */
+CC_API int causal_fftconv_bf16(const uint16_t *v, const uint16_t *g, uint16_t *r,
+                        int64_t B, int64_t L, int64_t D,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * causal_ntt_conv_i32 -- exact integer causal convolution through a
+ * number-theoretic transform mod p = 2013265921 = 15 * 2^27 + 1 (primitive
+ * root 31), the leakage-free primitive proposed in "Catastrophic Token Leakage
+ * in Convolutional Sequence Modeling and How to Mitigate It" (abstract).
+ *
+ *   v, g  [B, L, D] int32 (device); negative values are taken mod p.
+ *   r     [B, L, D] int32 (device): the centered residue of the true sum,
+ *         i.e. the unique value in [-(p-1)/2, (p-1)/2] congruent to it mod p.
+ *         It equals the true sum whenever |sum| <= (p-1)/2, e.g. whenever
+ *         L * max|v| * max|g| <= 1006632960 (documented precondition; not
+ *         checked, since checking would read the inputs).
+ * The result is bit-exact and deterministic.  Supported: 1 <= L <= 8192.
+ */
+CC_API int causal_ntt_conv_i32(const int32_t *v, const int32_t *g, int32_t *r,
+                        int64_t B, int64_t L, int64_t D,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * causal_conv_from_host -- the same convolution for HOST buffers: enqueues on
+ * `stream` the copy of v_host and g_host into the caller's device buffers
+ * v_dev and g_dev, the convolution into r_dev, and the copy of r_dev back
+ * into r_host, then returns (asynchronous; pass pinned host memory for
+ * overlap, and synchronise `stream` before reading r_host).
+ *   dtype: a cc_dtype.  All six buffers hold B*L*D elements of that type.
+ * Errors as for the device entry points; nothing is enqueued on failure.
+ */
+CC_API int causal_conv_from_host(int dtype, const void *v_host, const void *g_host, void *r_host,
+                          void *v_dev, void *g_dev, void *r_dev,
+                          int64_t B, int64_t L, int64_t D,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/* Device workspace bytes the conv entry points need for this problem (0 when
+ * no scratch is needed).  Returns (size_t)-1 for an invalid dtype/shape. */
+CC_API size_t causal_conv_workspace_bytes(int dtype, int64_t B, int64_t L, int64_t D);
+
+/* Largest supported L for a dtype (0 for an unknown dtype). */
+CC_API int64_t causal_conv_max_len(int dtype);
+
+/* Static text for a cc_status value. */
+CC_API const char *causal_conv_strerror(int status);
+
+/*
+ * causal_ntt_params -- host-only query of the transform constants the NTT
+ * path uses for transform length N (a power of two, 2 <= N <= 2^27):
+ *   out[0] = p, out[1] = omega_N = 31^((p-1)/N) mod p (an element of order
+ *   exactly N), out[2] = omega_N^-1 mod p, out[3] = N^-1 mod p,
+ *   out[4] = p^-1 mod 2^32 (Montgomery reduction with R = 2^32),
+ *   out[5] = 2^64 mod p (R^2 mod p).
+ * Returns CC_OK, or CC_ERR_INVALID_ARG for a bad N or NULL out.  Launches
+ * nothing and touches no device.
+ */
+CC_API int causal_ntt_params(int64_t N, uint32_t out[6]);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CAUSALCONV_H */

@@ -1,0 +1,136 @@
+"""B200 (sm_100a) causal sequence convolution.
+
+    r[b, t, d] = sum_{j<=t} v[b, j, d] * g[b, t-j, d]
+
+computed as in Caracal: Causal Architecture via Spectral Mixing (Multi-Head
+Fourier module: zero-pad to 2L, FFT, pointwise product, inverse FFT,
+truncate to L), plus the exact number-theoretic variant of "Catastrophic
+Token Leakage in Convolutional Sequence Modeling and How to Mitigate It".
+
+This module is argument marshalling only: every step of the computation runs
+in the CUDA kernels of ``libcausalconv.so`` behind the C ABI declared in
+``include/causalconv.h``.  PyTorch supplies device memory and the stream.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import (CC_DTYPE_BF16, CC_DTYPE_F32, CC_DTYPE_I32, CausalConvError, load, strerror)
+
+__all__ = [
+    "causal_fftconv_f32", "causal_fftconv_bf16", "causal_ntt_conv_i32", "causal_conv",
+    "causal_conv_from_host", "workspace_bytes", "max_len", "ntt_params", "strerror",
+    "CausalConvError", "CC_DTYPE_F32", "CC_DTYPE_BF16", "CC_DTYPE_I32",
+]
+
+_DT = {torch.float32: CC_DTYPE_F32, torch.bfloat16: CC_DTYPE_BF16, torch.int32: CC_DTYPE_I32}
+_FN = {CC_DTYPE_F32: "causal_fftconv_f32", CC_DTYPE_BF16: "causal_fftconv_bf16", CC_DTYPE_I32: "causal_ntt_conv_i32"}
+
+
+def _check(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != 3:
+        raise ValueError(f"{name} must be [B, L, D], got shape {tuple(t.shape)}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} shape {tuple(t.shape)} != {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous ([B, L, D] row-major)")
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _run(dtype_code: int, v: torch.Tensor, g: torch.Tensor, out, workspace, stream):
+    dtype = v.dtype
+    _check(v, "v", dtype)
+    _check(g, "g", dtype, v.shape)
+    if not v.is_cuda or not g.is_cuda or v.device != g.device:
+        raise ValueError("v and g must be CUDA tensors on the same device")
+    B, L, D = v.shape
+    if out is None:
+        out = torch.empty_like(v)
+    _check(out, "out", dtype, v.shape)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    with torch.cuda.device(v.device):
+        st = getattr(load(), _FN[dtype_code])(v.data_ptr(), g.data_ptr(), out.data_ptr(), B, L, D, ws_ptr, ws_bytes,
+                                              _stream_ptr(stream))
+    if st != 0:
+        raise CausalConvError(st, _FN[dtype_code])
+    return out
+
+
+def causal_fftconv_f32(v: torch.Tensor, g: torch.Tensor, out: torch.Tensor | None = None, workspace=None,
+                       stream=None) -> torch.Tensor:
+    """float32 [B, L, D] -> float32 [B, L, D] causal convolution (fused FFT kernel)."""
+    return _run(CC_DTYPE_F32, v, g, out, workspace, stream)
+
+
+def causal_fftconv_bf16(v: torch.Tensor, g: torch.Tensor, out: torch.Tensor | None = None, workspace=None,
+                        stream=None) -> torch.Tensor:
+    """bfloat16 [B, L, D] in/out, float32 transform arithmetic."""
+    return _run(CC_DTYPE_BF16, v, g, out, workspace, stream)
+
+
+def causal_ntt_conv_i32(v: torch.Tensor, g: torch.Tensor, out: torch.Tensor | None = None, workspace=None,
+                        stream=None) -> torch.Tensor:
+    """int32 [B, L, D] exact causal convolution (NTT mod 2013265921, centered residue)."""
+    return _run(CC_DTYPE_I32, v, g, out, workspace, stream)
+
+
+def causal_conv(v: torch.Tensor, g: torch.Tensor, out=None, workspace=None, stream=None) -> torch.Tensor:
+    """Dispatch on dtype: float32 / bfloat16 -> FFT path, int32 -> NTT path."""
+    if v.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {v.dtype}")
+    return _run(_DT[v.dtype], v, g, out, workspace, stream)
+
+
+def causal_conv_from_host(v_host: torch.Tensor, g_host: torch.Tensor, r_host: torch.Tensor, v_dev: torch.Tensor,
+                          g_dev: torch.Tensor, r_dev: torch.Tensor, workspace=None, stream=None) -> None:
+    """Host buffers in and out (pinned for overlap); the library enqueues the
+    H2D copies, the convolution and the D2H copy on ``stream``.  Caller
+    synchronises before reading ``r_host``."""
+    dtype = v_host.dtype
+    if dtype not in _DT:
+        raise TypeError(f"unsupported dtype {dtype}")
+    for name, t in (("v_host", v_host), ("g_host", g_host), ("r_host", r_host), ("v_dev", v_dev), ("g_dev", g_dev),
+                    ("r_dev", r_dev)):
+        _check(t, name, dtype, v_host.shape)
+    if v_host.is_cuda or g_host.is_cuda or r_host.is_cuda:
+        raise ValueError("*_host tensors must live in host memory")
+    B, L, D = v_host.shape
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    with torch.cuda.device(v_dev.device):
+        st = load().causal_conv_from_host(_DT[dtype], v_host.data_ptr(), g_host.data_ptr(), r_host.data_ptr(),
+                                          v_dev.data_ptr(), g_dev.data_ptr(), r_dev.data_ptr(), B, L, D, ws_ptr,
+                                          ws_bytes, _stream_ptr(stream))
+    if st != 0:
+        raise CausalConvError(st, "causal_conv_from_host")
+
+
+def workspace_bytes(dtype: torch.dtype, B: int, L: int, D: int) -> int:
+    return int(load().causal_conv_workspace_bytes(_DT[dtype], B, L, D))
+
+
+def max_len(dtype: torch.dtype) -> int:
+    return int(load().causal_conv_max_len(_DT[dtype]))
+
+
+def ntt_params(N: int) -> dict:
+    out = (ctypes.c_uint32 * 6)()
+    st = load().causal_ntt_params(N, out)
+    if st != 0:
+        raise CausalConvError(st, "causal_ntt_params")
+    return dict(zip(("p", "omega", "omega_inv", "n_inv", "p_inv_mod_2_32", "r2_mod_p"), list(out)))

@@ -1,0 +1,196 @@
+"""Parity of the sm_100a kernels (through the C ABI) with the CPU oracle.
+
+Float paths: |r_gpu - r_ref| <= 1e-5 * sum_j |v_j g_{t-j}| per element (fp32
+I/O) or 2e-2 of that (bf16 I/O), on the seeded workloads.  Integer path:
+bit-exact.  The oracle computes the plain definition
+r_t = sum_{j<=t} v_j g_{t-j} (Caracal, key designs 1 and 2).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from conftest import cuda_available
+from gpu_helpers import BF16_TOL, F32_TOL, as_f32, float_violations, run_gpu, to_dev, from_dev
+
+pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not cuda_available(), reason="needs a CUDA GPU")]
+
+P = 2013265921
+
+
+def _rand_float(shape, seed, scale_g=1.0):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return (rng.standard_normal(shape).astype(np.float32),
+            (scale_g * rng.standard_normal(shape)).astype(np.float32))
+
+
+# shapes spanning several tiles with ragged tails in L (vs N/2) and D (vs the channel tile)
+FLOAT_SHAPES = [(1, 1, 1), (1, 2, 3), (1, 3, 2), (2, 31, 5), (1, 32, 4), (1, 33, 7), (3, 200, 19), (1, 256, 8),
+                (2, 257, 9), (2, 513, 5), (2, 1000, 37), (1, 1024, 12)]
+
+
+@pytest.mark.parametrize("shape", FLOAT_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_f32_parity_full_oracle(shape):
+    v, g = _rand_float(shape, seed=sum(shape))
+    r = run_gpu(v, g, "f32")
+    r_ref, den = oracle.causal_conv(v, g)
+    n_bad, worst = float_violations(r, r_ref, den, F32_TOL)
+    assert n_bad == 0, f"{n_bad} elements beyond the fp32 bound, worst ratio {worst:.3g}"
+
+
+@pytest.mark.parametrize("shape", FLOAT_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_bf16_parity_full_oracle(shape):
+    v, g = _rand_float(shape, seed=7 + sum(shape), scale_g=0.125)
+    vb, gb = workloads.bf16_round(v), workloads.bf16_round(g)
+    r = run_gpu(vb, gb, "bf16")
+    r_ref, den = oracle.causal_conv(as_f32(vb, "bf16"), as_f32(gb, "bf16"))
+    n_bad, worst = float_violations(as_f32(r, "bf16"), r_ref, den, BF16_TOL)
+    assert n_bad == 0, f"{n_bad} elements beyond the bf16 bound, worst ratio {worst:.3g}"
+
+
+INT_SHAPES = [(1, 1, 1), (1, 2, 3), (2, 33, 5), (2, 1000, 37), (1, 4097, 3), (1, 8192, 2)]
+
+
+@pytest.mark.parametrize("shape", INT_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_ntt_bit_exact(shape):
+    rng = np.random.Generator(np.random.PCG64(sum(shape)))
+    v = rng.integers(-128, 128, shape).astype(np.int32)
+    g = rng.integers(-128, 128, shape).astype(np.int32)
+    r = run_gpu(v, g, "i32")
+    assert np.array_equal(r.astype(np.int64), oracle.causal_conv_int(v, g))
+
+
+@pytest.mark.parametrize("case", ["all_min", "all_max", "min_max", "alternating"])
+def test_ntt_extremes(case):
+    B, L, D = 1, 8192, 3
+    if case == "all_min":
+        v = np.full((B, L, D), -128, np.int32); g = v.copy()
+    elif case == "all_max":
+        v = np.full((B, L, D), 127, np.int32); g = v.copy()
+    elif case == "min_max":
+        v = np.full((B, L, D), -128, np.int32); g = np.full((B, L, D), 127, np.int32)
+    else:
+        s = np.where(np.arange(L) % 2 == 0, 127, -128).astype(np.int32).reshape(1, L, 1)
+        v = np.broadcast_to(s, (B, L, D)).copy(); g = -v
+    r = run_gpu(v, g, "i32").astype(np.int64)
+    ref = oracle.causal_conv_int(v, g)
+    assert np.array_equal(r, ref)
+    if case == "all_min":
+        assert r[0, -1, 0] == 2 ** 27
+
+
+def test_ntt_wraps_to_centered_residue():
+    """Sums beyond (p-1)/2 come back as the centered residue mod p."""
+    rng = np.random.Generator(np.random.PCG64(11))
+    B, L, D = 1, 512, 4
+    v = rng.integers(-2 ** 31, 2 ** 31, (B, L, D), dtype=np.int64).astype(np.int32)
+    g = rng.integers(-2 ** 31, 2 ** 31, (B, L, D), dtype=np.int64).astype(np.int32)
+    r = run_gpu(v, g, "i32").astype(np.int64)
+    # exact sums mod p: residues < 2^31, each product < 2^62, reduced before summing
+    vm = v.astype(np.int64) % P
+    gm = g.astype(np.int64) % P
+    ref = np.zeros((B, L, D), np.int64)
+    for t in range(L):
+        ref[:, t, :] = ((vm[:, : t + 1, :] * gm[:, t::-1, :]) % P).sum(axis=1) % P
+    ref = oracle.centered_mod(ref, P)
+    assert np.array_equal(r, ref)
+
+
+CONFIGS_FULL = ["tiny_f32", "small_f32"]
+
+
+@pytest.mark.parametrize("name", CONFIGS_FULL)
+def test_config_full_oracle(name):
+    w = workloads.WORKLOADS[name]
+    v, g = workloads.generate(w)
+    r = run_gpu(v, g, w.dtype)
+    r_ref, den = oracle.causal_conv(as_f32(v, w.dtype), as_f32(g, w.dtype))
+    tol = F32_TOL if w.dtype == "f32" else BF16_TOL
+    n_bad, worst = float_violations(as_f32(r, w.dtype) if w.dtype == "bf16" else r, r_ref, den, tol)
+    assert n_bad == 0, f"{name}: {n_bad} violations, worst ratio {worst:.3g}"
+
+
+def test_config_ntt_full_bit_exact():
+    w = workloads.WORKLOADS["ntt_i32"]
+    v, g = workloads.generate(w)
+    r = run_gpu(v, g, "i32").astype(np.int64)
+    pts = workloads.sample_points(w.B, w.L, w.D, 4096, seed=1004)
+    # sampled check first (fast, informative), then every element
+    ref_pts = oracle.causal_conv_int_points(v, g, pts)
+    assert np.array_equal(r[pts[:, 0], pts[:, 1], pts[:, 2]], ref_pts)
+    assert np.array_equal(r, oracle.causal_conv_int(v, g))
+
+
+def _leak(dtype, v, g, t_c, scale, seed):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    r0 = run_gpu(v, g, dtype)
+    v2, g2 = v.copy(), g.copy()
+    if dtype == "i32":
+        v2[:, t_c + 1:, :] = rng.integers(-128, 128, v2[:, t_c + 1:, :].shape)
+        g2[:, t_c + 1:, :] = rng.integers(-128, 128, g2[:, t_c + 1:, :].shape)
+    else:
+        v2[:, t_c + 1:, :] = scale * rng.standard_normal(v2[:, t_c + 1:, :].shape)
+        g2[:, t_c + 1:, :] = scale * rng.standard_normal(g2[:, t_c + 1:, :].shape)
+    r1 = run_gpu(v2, g2, dtype)
+    return float(np.abs(r1[:, : t_c + 1, :].astype(np.float64) - r0[:, : t_c + 1, :]).max())
+
+
+def test_leakage_ntt_is_exactly_zero():
+    rng = np.random.Generator(np.random.PCG64(5))
+    v = rng.integers(-128, 128, (2, 8192, 8)).astype(np.int32)
+    g = rng.integers(-128, 128, (2, 8192, 8)).astype(np.int32)
+    for t_c in (31, 4096, 8190):
+        assert _leak("i32", v, g, t_c, 1, seed=t_c) == 0.0
+
+
+def test_leakage_f32_measured():
+    """Float transforms leak future tokens through rounding (the TL;DR of
+    "Catastrophic Token Leakage in Convolutional Sequence Modeling"): the
+    prefix moves when only the future changes.  The directly summed head
+    (t < 32) is exactly causal."""
+    v, g = _rand_float((1, 1024, 16), seed=3)
+    assert _leak("f32", v, g, 31, 1e4, seed=1) == 0.0
+    leak_mid = _leak("f32", v, g, 512, 1e4, seed=2)
+    assert np.isfinite(leak_mid) and leak_mid > 0.0
+
+
+def test_from_host_matches_device_path():
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    for dtype, (v, g) in (("f32", _rand_float((2, 1000, 12), 1)),
+                          ("i32", tuple(np.random.Generator(np.random.PCG64(2)).integers(-128, 128, (2, 700, 8))
+                                        .astype(np.int32) for _ in range(2)))):
+        tv, tg = to_dev(v, dtype), to_dev(g, dtype)
+        ref = from_dev(ssm.causal_conv(tv, tg), dtype)
+        hv = torch.from_numpy(v).pin_memory()
+        hg = torch.from_numpy(g).pin_memory()
+        hr = torch.empty_like(hv).pin_memory()
+        dv, dg, dr = torch.empty_like(tv), torch.empty_like(tg), torch.empty_like(tv)
+        ssm.causal_conv_from_host(hv, hg, hr, dv, dg, dr)
+        torch.cuda.synchronize()
+        assert np.array_equal(hr.numpy(), ref)
+
+
+def test_side_stream_and_determinism():
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    v, g = _rand_float((2, 1024, 64), 9)
+    tv, tg = to_dev(v, "f32"), to_dev(g, "f32")
+    ref = ssm.causal_fftconv_f32(tv, tg)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        out = ssm.causal_fftconv_f32(tv, tg, stream=s)
+    s.synchronize()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+
+
+def test_rejects_host_pointer_on_device_entry():
+    import torch
+    from spectral_sequence_mixing_b200 import _lib
+    lib = _lib.load()
+    h = torch.zeros(1, 16, 4)
+    d = torch.zeros(1, 16, 4, device="cuda")
+    d2 = torch.zeros(1, 16, 4, device="cuda")
+    assert lib.causal_fftconv_f32(h.data_ptr(), d.data_ptr(), d2.data_ptr(), 1, 16, 4, None, 0, None) == 6
+    assert lib.causal_fftconv_f32(d.data_ptr(), d2.data_ptr(), h.data_ptr(), 1, 16, 4, None, 0, None) == 6
