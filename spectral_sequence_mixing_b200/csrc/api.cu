@@ -8,21 +8,31 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <vector>
 
 #include "causalconv.h"
 #include "fftconv_fused.cuh"
+#include "bigconv.cuh"
 #include "ntt.cuh"
 
 namespace ccv {
 
 // ------------------------------------------------------------------ tables
-using CfgS = FusedCfg<16, 8>;  // N = 512,  L <= 256
-using CfgM = FusedCfg<32, 4>;  // N = 2048, L <= 1024
+// Transform geometry per size class (the twiddle tables depend only on N1, N2).
+template <typename IO> using CfgS = FusedCfg<16, 8, IO>;  // N = 512,  L <= 256
+template <typename IO> using CfgM = FusedCfg<32, 4, IO>;  // N = 2048, L <= 1024
 
-__device__ float2 g_tw_s[CfgS::TW_SIZE];
-__device__ float2 g_tw_m[CfgM::TW_SIZE];
+__device__ float2 g_tw_s[CfgS<float>::TW_SIZE];
+__device__ float2 g_tw_m[CfgM<float>::TW_SIZE];
+
+// Long rows: one row per CTA (N = 8192) or per 8-CTA cluster (N = 131072).
+template <typename IO> using BigL = BigCfg<32, 16, 16, 1, 1, 256, IO>;   // N = 8192,   L <= 4096
+template <typename IO> using BigX = BigCfg<8, 32, 32, 16, 8, 512, IO>;   // N = 131072, L <= 65536
+constexpr int kMinbBigL = 2, kMinbBigX = 1;
+__device__ float2 g_tw_bl[BigL<float>::TW_SIZE];
+__device__ float2 g_tw_bx[BigX<float>::TW_SIZE];
 
 static double kTwoPi = 6.283185307179586476925286766559;
 
@@ -36,19 +46,47 @@ static float2 omega(int64_t e, int64_t n) {
 
 template <class Cfg>
 static std::vector<float2> fused_twiddles() {
-    constexpr int N = Cfg::N, N1 = Cfg::N1, N2 = Cfg::N2, M2 = Cfg::M2, M = N / 2;
+    // theta = omega_2N; see the table layout in FusedCfg
+    constexpr int N = Cfg::N, N1 = Cfg::N1, N2 = Cfg::N2, M2 = Cfg::M2;
+    const int64_t N2x = 2 * (int64_t)N;
     std::vector<float2> t(Cfg::TW_SIZE);
     for (int k1 = 0; k1 < N1; ++k1)
-        for (int n2 = 0; n2 < N2; ++n2) t[k1 * N2 + n2] = omega((int64_t)n2 * k1, N);
+        for (int n2 = 0; n2 < N2; ++n2) t[k1 * N2 + n2] = omega((int64_t)n2 * (2 * k1 + 1), N2x);
     for (int k2 = 0; k2 < M2; ++k2)
-        for (int k1 = 0; k1 < N1; ++k1) t[Cfg::TW_P + k2 * N1 + k1] = omega(-(int64_t)(k1 + N1 * k2), N);
+        for (int k1 = 0; k1 < N1; ++k1)
+            t[Cfg::TW_P + k2 * N1 + k1] = omega(-(2 * (int64_t)(k1 + N1 * k2) + 1), N2x);
     for (int m2 = 0; m2 < M2; ++m2)
-        for (int k1 = 0; k1 < N1; ++k1) t[Cfg::TW_Q + m2 * N1 + k1] = omega(-(int64_t)k1 * m2, M);
+        for (int k1 = 0; k1 < N1; ++k1) t[Cfg::TW_Q + m2 * N1 + k1] = omega(-2 * (int64_t)m2 * (2 * k1 + 1), N2x);
     return t;
+}
+
+template <class Cfg>
+static std::vector<float2> big_twiddles() {
+    constexpr int S = Cfg::S, SL = Cfg::SL, R0 = Cfg::R0, RA = Cfg::RA, RB = Cfg::RB, RC = Cfg::RC;
+    std::vector<float2> t(Cfg::TW_SIZE);
+    for (int k0 = 0; k0 < R0; ++k0)
+        for (int n = 0; n < SL; ++n) t[Cfg::TW0 + k0 * SL + n] = omega((int64_t)n * (2 * k0 + 1), 2 * (int64_t)S);
+    for (int k = 0; k < RA; ++k)
+        for (int lo = 0; lo < RB * RC; ++lo) t[Cfg::TWA + k * (RB * RC) + lo] = omega((int64_t)lo * k, SL);
+    for (int k = 0; k < RB; ++k)
+        for (int lo = 0; lo < RC; ++lo) t[Cfg::TWB + k * RC + lo] = omega((int64_t)lo * k, RB * RC);
+    return t;
+}
+
+template <class Cfg, typename IO, int MINB>
+static cudaError_t set_big_attr() {
+    return cudaFuncSetAttribute(bigconv_kernel<Cfg::R0, Cfg::RA, Cfg::RB, Cfg::RC, Cfg::CL, Cfg::T, MINB, IO>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_BYTES);
 }
 
 static std::mutex g_init_mu;
 static bool g_init_done[128];
+
+constexpr int kMinbS = 4;
+constexpr int kMinbM = 2;
+
+// Per device: SM count and, per kernel instantiation, resident CTAs per SM.
+static int g_num_sms[128];
 
 template <class Cfg, typename IO, int MINB>
 static cudaError_t set_smem_attr() {
@@ -56,30 +94,40 @@ static cudaError_t set_smem_attr() {
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_BYTES);
 }
 
-constexpr int kMinbS = 3;
-constexpr int kMinbM = 3;
-
 static cudaError_t ensure_init(int dev) {
     if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lk(g_init_mu);
     if (g_init_done[dev]) return cudaSuccess;
     cudaError_t e;
-    float2 w64[64];
-    for (int k = 0; k < 64; ++k) w64[k] = omega(k, 64);
-    if ((e = cudaMemcpyToSymbol(c_w64, w64, sizeof(w64))) != cudaSuccess) return e;
+    float2 w128[128];
+    for (int k = 0; k < 128; ++k) w128[k] = omega(k, 128);
+    if ((e = cudaMemcpyToSymbol(c_w128, w128, sizeof(w128))) != cudaSuccess) return e;
     {
-        auto t = fused_twiddles<CfgS>();
+        auto t = fused_twiddles<CfgS<float>>();
         if ((e = cudaMemcpyToSymbol(g_tw_s, t.data(), t.size() * sizeof(float2))) != cudaSuccess) return e;
     }
     {
-        auto t = fused_twiddles<CfgM>();
+        auto t = fused_twiddles<CfgM<float>>();
         if ((e = cudaMemcpyToSymbol(g_tw_m, t.data(), t.size() * sizeof(float2))) != cudaSuccess) return e;
     }
+    {
+        auto t = big_twiddles<BigL<float>>();
+        if ((e = cudaMemcpyToSymbol(g_tw_bl, t.data(), t.size() * sizeof(float2))) != cudaSuccess) return e;
+    }
+    {
+        auto t = big_twiddles<BigX<float>>();
+        if ((e = cudaMemcpyToSymbol(g_tw_bx, t.data(), t.size() * sizeof(float2))) != cudaSuccess) return e;
+    }
+    if ((e = set_big_attr<BigL<float>, float, kMinbBigL>()) != cudaSuccess) return e;
+    if ((e = set_big_attr<BigL<__nv_bfloat16>, __nv_bfloat16, kMinbBigL>()) != cudaSuccess) return e;
+    if ((e = set_big_attr<BigX<float>, float, kMinbBigX>()) != cudaSuccess) return e;
+    if ((e = set_big_attr<BigX<__nv_bfloat16>, __nv_bfloat16, kMinbBigX>()) != cudaSuccess) return e;
     if ((e = ntt_init_device()) != cudaSuccess) return e;
-    if ((e = set_smem_attr<CfgS, float, kMinbS>()) != cudaSuccess) return e;
-    if ((e = set_smem_attr<CfgS, __nv_bfloat16, kMinbS>()) != cudaSuccess) return e;
-    if ((e = set_smem_attr<CfgM, float, kMinbM>()) != cudaSuccess) return e;
-    if ((e = set_smem_attr<CfgM, __nv_bfloat16, kMinbM>()) != cudaSuccess) return e;
+    if ((e = set_smem_attr<CfgS<float>, float, kMinbS>()) != cudaSuccess) return e;
+    if ((e = set_smem_attr<CfgS<__nv_bfloat16>, __nv_bfloat16, kMinbS>()) != cudaSuccess) return e;
+    if ((e = set_smem_attr<CfgM<float>, float, kMinbM>()) != cudaSuccess) return e;
+    if ((e = set_smem_attr<CfgM<__nv_bfloat16>, __nv_bfloat16, kMinbM>()) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     g_init_done[dev] = true;
     return cudaSuccess;
 }
@@ -97,7 +145,7 @@ static size_t dtype_size(int dtype) {
 static int64_t max_len(int dtype) {
     switch (dtype) {
         case CC_DTYPE_F32:
-        case CC_DTYPE_BF16: return 1024;
+        case CC_DTYPE_BF16: return BigX<float>::LMAX;
         case CC_DTYPE_I32: return kNttMaxL;
         default: return 0;
     }
@@ -155,25 +203,70 @@ static int check_common(int dtype, const void *v, const void *g, const void *r, 
 // ------------------------------------------------------------------ launch
 template <class Cfg, int MINB, typename IO>
 static int launch_fused(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, const float2 *tw,
-                        cudaStream_t s) {
+                        cudaStream_t s, int dev) {
     const int64_t groups = (D + Cfg::ROWS - 1) / Cfg::ROWS;
-    const int64_t blocks = B * groups;
-    if (blocks > INT32_MAX) return CC_ERR_UNSUPPORTED;
-    fftconv_fused_kernel<Cfg::N2, Cfg::ROWS, MINB, IO>
-        <<<(unsigned)blocks, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(v, g, r, (int)L, (int)D, (int)groups, tw);
+    const int64_t tiles = B * groups;
+    if (tiles > INT32_MAX) return CC_ERR_UNSUPPORTED;
+    auto kern = fftconv_fused_kernel<Cfg::N2, Cfg::ROWS, MINB, IO>;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cfg::THREADS, Cfg::SMEM_BYTES) != cudaSuccess ||
+        per_sm < 1) {
+        cudaGetLastError();
+        return CC_ERR_CUDA;
+    }
+    const int64_t grid = std::min<int64_t>(tiles, (int64_t)per_sm * g_num_sms[dev]);
+    // whole-chunk async copies need full, aligned channel groups
+    const bool vec = (D % Cfg::ROWS) == 0 && ((uintptr_t)v % Cfg::CHUNK) == 0 && ((uintptr_t)g % Cfg::CHUNK) == 0;
+    kern<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(v, g, r, (int)L, (int)D, (int)groups, (int)tiles,
+                                                              vec ? 1 : 0, tw);
     return cudaGetLastError() == cudaSuccess ? CC_OK : CC_ERR_CUDA;
 }
 
-template <typename IO>
-static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, cudaStream_t s) {
-    void *tw = nullptr;
-    if (L <= CfgS::N / 2) {
-        if (cudaGetSymbolAddress(&tw, g_tw_s) != cudaSuccess) return CC_ERR_CUDA;
-        return launch_fused<CfgS, kMinbS>(v, g, r, B, L, D, (const float2 *)tw, s);
+template <class Cfg, int MINB, typename IO>
+static int launch_big(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, const float2 *tw,
+                      cudaStream_t s) {
+    const int64_t rows = B * D;
+    if (rows * Cfg::CL > INT32_MAX) return CC_ERR_UNSUPPORTED;
+    auto kern = bigconv_kernel<Cfg::R0, Cfg::RA, Cfg::RB, Cfg::RC, Cfg::CL, Cfg::T, MINB, IO>;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rows * Cfg::CL));
+    cfg.blockDim = dim3(Cfg::T);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = Cfg::CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, v, g, r, (int)L, (int)D, tw);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return CC_ERR_CUDA;
     }
-    if (L <= CfgM::N / 2) {
+    return CC_OK;
+}
+
+template <typename IO>
+static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, cudaStream_t s,
+                            int dev) {
+    void *tw = nullptr;
+    if (L <= CfgS<IO>::LMAX) {
+        if (cudaGetSymbolAddress(&tw, g_tw_s) != cudaSuccess) return CC_ERR_CUDA;
+        return launch_fused<CfgS<IO>, kMinbS>(v, g, r, B, L, D, (const float2 *)tw, s, dev);
+    }
+    if (L <= CfgM<IO>::LMAX) {
         if (cudaGetSymbolAddress(&tw, g_tw_m) != cudaSuccess) return CC_ERR_CUDA;
-        return launch_fused<CfgM, kMinbM>(v, g, r, B, L, D, (const float2 *)tw, s);
+        return launch_fused<CfgM<IO>, kMinbM>(v, g, r, B, L, D, (const float2 *)tw, s, dev);
+    }
+    if (L <= BigL<IO>::LMAX) {
+        if (cudaGetSymbolAddress(&tw, g_tw_bl) != cudaSuccess) return CC_ERR_CUDA;
+        return launch_big<BigL<IO>, kMinbBigL>(v, g, r, B, L, D, (const float2 *)tw, s);
+    }
+    if (L <= BigX<IO>::LMAX) {
+        if (cudaGetSymbolAddress(&tw, g_tw_bx) != cudaSuccess) return CC_ERR_CUDA;
+        return launch_big<BigX<IO>, kMinbBigX>(v, g, r, B, L, D, (const float2 *)tw, s);
     }
     return CC_ERR_UNSUPPORTED;
 }
@@ -213,7 +306,7 @@ int causal_fftconv_f32(const float *v, const float *g, float *r, int64_t B, int6
     int st = check_common(CC_DTYPE_F32, v, g, r, B, L, D, workspace_bytes, &dev);
     if (st != CC_OK) return st;
     if (ensure_init(dev) != cudaSuccess) return CC_ERR_CUDA;
-    return fftconv_dispatch<float>(v, g, r, B, L, D, (cudaStream_t)stream);
+    return fftconv_dispatch<float>(v, g, r, B, L, D, (cudaStream_t)stream, dev);
 }
 
 int causal_fftconv_bf16(const uint16_t *v, const uint16_t *g, uint16_t *r, int64_t B, int64_t L, int64_t D,
@@ -224,7 +317,7 @@ int causal_fftconv_bf16(const uint16_t *v, const uint16_t *g, uint16_t *r, int64
     if (st != CC_OK) return st;
     if (ensure_init(dev) != cudaSuccess) return CC_ERR_CUDA;
     return fftconv_dispatch<__nv_bfloat16>((const __nv_bfloat16 *)v, (const __nv_bfloat16 *)g, (__nv_bfloat16 *)r, B,
-                                           L, D, (cudaStream_t)stream);
+                                           L, D, (cudaStream_t)stream, dev);
 }
 
 int causal_ntt_conv_i32(const int32_t *v, const int32_t *g, int32_t *r, int64_t B, int64_t L, int64_t D,

@@ -96,6 +96,54 @@ def test_ntt_wraps_to_centered_residue():
     assert np.array_equal(r, ref)
 
 
+# rows longer than one fused tile: one row per CTA (L <= 4096) or per 8-CTA cluster (L <= 65536)
+BIG_SHAPES = [(1, 1025, 3), (2, 2000, 5), (1, 4096, 4)]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", BIG_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_big_rows_full_oracle(shape, dtype):
+    v, g = _rand_float(shape, seed=100 + sum(shape), scale_g=0.125 if dtype == "bf16" else 1.0)
+    if dtype == "bf16":
+        v, g = workloads.bf16_round(v), workloads.bf16_round(g)
+    r = run_gpu(v, g, dtype)
+    r_ref, den = oracle.causal_conv(as_f32(v, dtype), as_f32(g, dtype))
+    n_bad, worst = float_violations(as_f32(r, dtype) if dtype == "bf16" else r, r_ref, den,
+                                    F32_TOL if dtype == "f32" else BF16_TOL)
+    assert n_bad == 0, f"{n_bad} violations, worst ratio {worst:.3g}"
+
+
+CLUSTER_SHAPES = [(1, 4097, 3), (2, 20000, 2), (1, 65536, 2)]
+
+
+@pytest.mark.parametrize("shape", CLUSTER_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_cluster_rows_sampled_oracle(shape):
+    B, L, D = shape
+    rng = np.random.Generator(np.random.PCG64(sum(shape)))
+    v = rng.standard_normal(shape).astype(np.float32)
+    g = (rng.standard_normal(shape) * (1.0 + np.arange(L).reshape(1, L, 1)) ** -0.75).astype(np.float32)
+    r = run_gpu(v, g, "f32")
+    pts = workloads.sample_points(B, L, D, 1024, seed=7)
+    r_ref, den = oracle.causal_conv_points(v, g, pts)
+    n_bad, worst = float_violations(r[pts[:, 0], pts[:, 1], pts[:, 2]], r_ref, den, F32_TOL)
+    assert n_bad == 0, f"{n_bad} violations, worst ratio {worst:.3g}"
+
+
+@pytest.mark.parametrize("name", ["large_bf16", "long_f32"])
+def test_config_sampled_oracle(name):
+    """Full-size workloads in the launch configuration the benchmark times,
+    checked on a stratified sample of outputs."""
+    w = workloads.WORKLOADS[name]
+    v, g = workloads.generate(w)
+    r = run_gpu(v, g, w.dtype)
+    pts = workloads.sample_points(w.B, w.L, w.D, 4096, seed=1000 + list(workloads.WORKLOADS).index(name))
+    r_ref, den = oracle.causal_conv_points(as_f32(v, w.dtype), as_f32(g, w.dtype), pts)
+    got = as_f32(r, w.dtype)[pts[:, 0], pts[:, 1], pts[:, 2]] if w.dtype == "bf16" else r[pts[:, 0], pts[:, 1], pts[:, 2]]
+    tol = F32_TOL if w.dtype == "f32" else BF16_TOL
+    n_bad, worst = float_violations(got, r_ref, den, tol)
+    assert n_bad == 0, f"{name}: {n_bad} violations, worst ratio {worst:.3g}"
+
+
 CONFIGS_FULL = ["tiny_f32", "small_f32"]
 
 
