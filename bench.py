@@ -37,7 +37,7 @@ import workloads  # noqa: E402
 
 METRIC = "causal FFT-conv GB/s and (B*D*L)/s at 1 B200; % of HBM roofline"
 L2_BYTES = 126 * 2 ** 20
-KERNEL_SOURCES = ["fftconv_fused.cuh", "fft_reg.cuh", "ntt.cuh", "api.cu"]
+KERNEL_SOURCES = ["fftconv_fused.cuh", "fft_reg.cuh", "bigconv.cuh", "ntt.cuh", "api.cu"]
 
 
 def parse_args():
@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--workload", default="small_f32", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--shape", default=None,
+                    help="B,L,D override of the workload's sizes (same recipe); for small profiler captures")
     return ap.parse_args()
 
 
@@ -77,18 +79,17 @@ def measured_peaks():
 
 
 def recorded_traffic(workload: str, kernel: str):
-    """dram bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources; else None."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes (read + write) per launch of `kernel` on the full-size
+    `workload`, from profiles/dram_traffic.txt (lines: workload kernel
+    source_hash bytes), if it was taken on the current kernel sources; else
+    None."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(p):
         return None
-    try:
-        d = json.load(open(p))
-        e = d.get(workload, {})
-        if e.get("kernel") == kernel and e.get("source_hash") == kernel_source_hash():
-            return float(e["dram_bytes_per_launch"])
-    except Exception:
-        return None
+    for line in open(p):
+        f = line.split()
+        if len(f) == 4 and not line.startswith("#") and f[0] == workload and f[1] == kernel:
+            return float(f[3]) if f[2] == kernel_source_hash() else None
     return None
 
 
@@ -172,13 +173,22 @@ def cpu_oracle_rate(w: workloads.Workload, v, g, budget_s: float):
     return units / secs, oracle.num_threads(), desc, secs
 
 
+def workload_for(args) -> workloads.Workload:
+    w = workloads.WORKLOADS[args.workload]
+    if args.shape:
+        B, L, D = (int(x) for x in args.shape.split(","))
+        from dataclasses import replace
+        w = replace(w, B=B, L=L, D=D)
+    return w
+
+
 def run_reference(args, rank, world):
     """The oracle (plain CPU direct sum) timed on the host cores as the
     reference arm, on the same workload and metric."""
     if rank != 0:
         return
-    w = workloads.WORKLOADS[args.workload]
-    v, g = workloads.generate(w)
+    w = workload_for(args)
+    v, g = workloads.generate(w, B=w.B, L=w.L, D=w.D)
     per_step = max(0.05, 120.0 / max(1, args.steps + args.warmup))
     import oracle
     fv = workloads.bf16_to_f32(v) if w.dtype == "bf16" else v
@@ -235,7 +245,7 @@ def run_ours(args, rank, world, local):
         if pg is not None:
             pg.barrier()
 
-    w = workloads.WORKLOADS[args.workload]
+    w = workload_for(args)
     v_np, g_np = workloads.generate(w, seed=w.seed + 1000 * rank)
     tdt = {"f32": torch.float32, "bf16": torch.bfloat16, "i32": torch.int32}[w.dtype]
 
@@ -302,7 +312,7 @@ def run_ours(args, rank, world, local):
     e2e_gbs = w.units * world * e2e_steps * 3 * w.elem_bytes / (ems * 1e-3) / 1e9
 
     peak, peak_src = measured_peaks()
-    kernel = {"f32": "fftconv_fused_kernel", "bf16": "fftconv_fused_kernel", "i32": "ntt_conv_kernel"}[w.dtype]
+    kernel = "ntt_conv_kernel" if w.dtype == "i32" else ("fftconv_fused_kernel" if w.L <= 1024 else "bigconv_kernel")
     per_launch_bytes = 3 * w.units * w.elem_bytes
     achieved = per_launch_bytes / (ms_per_step * 1e-3) / 1e9
     line = {
@@ -318,7 +328,7 @@ def run_ours(args, rank, world, local):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
                      "kernel": kernel, "algorithmic_bytes_per_launch": per_launch_bytes,
-                     "traffic": recorded_traffic(w.name, kernel)},
+                     "traffic": None if args.shape else recorded_traffic(w.name, kernel)},
         "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": 2 * w.units * w.elem_bytes,
                 "d2h_bytes_per_step": w.units * w.elem_bytes, "steps": e2e_steps,
                 "path": "causal_conv_from_host (pinned host buffers)"},
