@@ -61,6 +61,28 @@ def dist_env():
     return rank, world, local
 
 
+def rank_seed(w: workloads.Workload, rank: int) -> int:
+    """Each rank convolves its own batch: the workload's seed for rank 0, a
+    distinct one for the others (weak scaling, no data shared across ranks)."""
+    return w.seed + 1000 * rank
+
+
+def max_over_ranks(value: float, pg, device=None) -> float:
+    """Max of a per-rank timing over the process group (identity without one)."""
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(units_per_rank: int, world: int, steps: int, ms: float, bytes_per_unit: int):
+    """Whole-job outputs/s and algorithmic GB/s from the max-over-ranks time."""
+    units = units_per_rank * world * steps
+    return units / (ms * 1e-3), units * bytes_per_unit / (ms * 1e-3) / 1e9
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
@@ -246,7 +268,7 @@ def run_ours(args, rank, world, local):
             pg.barrier()
 
     w = workload_for(args)
-    v_np, g_np = workloads.generate(w, seed=w.seed + 1000 * rank)
+    v_np, g_np = workloads.generate(w, seed=rank_seed(w, rank))
     tdt = {"f32": torch.float32, "bf16": torch.bfloat16, "i32": torch.int32}[w.dtype]
 
     def to_t(x):
@@ -279,14 +301,10 @@ def run_ours(args, rank, world, local):
         end.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-    ms = start.elapsed_time(end)
-    if pg is not None:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), pg, dev)
     ms_per_step = ms / args.steps
     units_total = w.units * world * args.steps
-    gbs = units_total * 3 * w.elem_bytes / (ms * 1e-3) / 1e9
+    ups, gbs = throughput(w.units, world, args.steps, ms, 3 * w.elem_bytes)
 
     # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -304,12 +322,8 @@ def run_ours(args, rank, world, local):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    ems = e0.elapsed_time(e1)
-    if pg is not None:
-        t = torch.tensor([ems], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ems = float(t.item())
-    e2e_gbs = w.units * world * e2e_steps * 3 * w.elem_bytes / (ems * 1e-3) / 1e9
+    ems = max_over_ranks(e0.elapsed_time(e1), pg, dev)
+    _, e2e_gbs = throughput(w.units, world, e2e_steps, ems, 3 * w.elem_bytes)
 
     peak, peak_src = measured_peaks()
     kernel = "ntt_conv_kernel" if w.dtype == "i32" else ("fftconv_fused_kernel" if w.L <= 1024 else "bigconv_kernel")
@@ -323,7 +337,7 @@ def run_ours(args, rank, world, local):
                    "transform_len": 2 ** math.ceil(math.log2(2 * w.L)),
                    "l2": f"inputs larger than L2: {n_sets} rotating (v,g,r) sets of {set_bytes / 2 ** 20:.0f} MiB",
                    "parallelism": f"dp{world} (independent batches, no collective)"},
-        "outputs_per_s": units_total / (ms * 1e-3),
+        "outputs_per_s": ups,
         "hbm_frac": gbs / world / peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
@@ -336,8 +350,8 @@ def run_ours(args, rank, world, local):
         "clocks": clk.report(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        ups, cores, desc, secs = cpu_oracle_rate(w, v_np, g_np, budget_s=15.0)
-        line["cpu_baseline"] = {"value": ups * 3 * w.elem_bytes / 1e9, "unit": "GB/s", "cores": cores,
+        cpu_ups, cores, desc, secs = cpu_oracle_rate(w, v_np, g_np, budget_s=15.0)
+        line["cpu_baseline"] = {"value": cpu_ups * 3 * w.elem_bytes / 1e9, "unit": "GB/s", "cores": cores,
                                 "kind": "oracle", "sample": desc, "seconds": secs}
     if rank == 0:
         print(json.dumps(line), flush=True)

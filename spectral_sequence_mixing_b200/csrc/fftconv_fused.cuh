@@ -75,9 +75,13 @@ struct FusedCfg {
     static constexpr int N = N1 * N2;
     static constexpr int LMAX = N / 2;
     static constexpr int M2 = N2 / 2;
+    static constexpr int H = N2 / 2;   // half column (first radix-2 split)
+    static constexpr int MH = M2 / 2;  // half of the inverse column
     static constexpr int LOG_N2 = ilog2(N2);
-    static constexpr int LOG_M2 = ilog2(M2);
-    static constexpr int THREADS = ROWS * N2;
+    static constexpr int LOG_H = ilog2(H);
+    static constexpr int LOG_MH = ilog2(MH);
+    static constexpr int THREADS = ROWS * 2 * N2;  // two threads per (row, n2) / column pair / (m2, h)
+    static constexpr int NWARPS = THREADS / 32;
     // Shared-memory strides in float2 units.  With 8-byte accesses a
     // half-warp is conflict-free when its 16 lanes hit distinct (word mod 16):
     // SF_N = 1 (mod 16) serves the F1 stores / F3 loads, SI_M = 2 (mod 16) and
@@ -86,12 +90,13 @@ struct FusedCfg {
     static constexpr int SI_M = N1 + 2;
     static constexpr int SC = N + N2 + 16 / ROWS;
     static constexpr int HEAD = kHeadT0;
-    // staging: [LMAX][ROWS] elements of IO for v, then for g
     static constexpr size_t XBYTES = (size_t)ROWS * SC * 8;
-    static constexpr size_t HBYTES = (size_t)ROWS * HEAD * 8;
+    static constexpr size_t HBYTES = (size_t)ROWS * HEAD * 8;  // direct-sum results r_t, t < HEAD, [ROWS][2*HEAD] floats
+    // staging: [LMAX][ROWS] elements of IO for v, then for g
     static constexpr size_t SBYTES = (size_t)2 * LMAX * ROWS * sizeof(IO);
-    static constexpr int NWARPS = THREADS / 32;
-    static constexpr size_t RBYTES = (size_t)(NWARPS * ROWS + ROWS) * 8;  // norm partials, per-row scale
+    // norm partials [NWARPS][ROWS] float2, per-row scale [ROWS] float (padded),
+    // rotations [(2h+s)][H+1] float2 (padded so the four (h, s) lane groups hit distinct banks)
+    static constexpr size_t RBYTES = (size_t)(NWARPS * ROWS) * 8 + (size_t)ROWS * 8 + (size_t)4 * (N2 / 2 + 1) * 8;
     static constexpr size_t SMEM_BYTES = XBYTES + HBYTES + SBYTES + RBYTES;
     // Twiddle table layout (float2, built on the host in fp64), theta = omega_2N:
     //   T1[k1*N2 + n2]           = theta^(n2 (2 k1 + 1))         k1 < N1, n2 < N2
@@ -100,10 +105,12 @@ struct FusedCfg {
     static constexpr int TW_P = N;
     static constexpr int TW_Q = N + N / 2;
     static constexpr int TW_SIZE = 2 * N;
-    static_assert(N2 % 16 == 0 && N1 <= 64, "register DFT sizes 16..32 supported");
+    static_assert(N2 == 16 || N2 == 32, "register DFT sizes 16..32 supported");
+    static_assert(THREADS == 256, "lane maps assume 8 warps per CTA");
     static_assert(SC >= N2 * SF_N && SC >= M2 * SI_M, "exchange buffers must fit the row stride");
-    static_assert(16 % ROWS == 0 && (32 / ROWS) % 2 == 0, "ROWS must divide 16");
-    static_assert(HEAD % N2 == 0 && HEAD <= LMAX, "head must be whole n1 blocks of a row");
+    static_assert(16 % ROWS == 0 && 4 * ROWS <= 32, "ROWS must divide 16 and leave room for (h, s) lane bits");
+    static_assert(HEAD == 32 && HEAD <= LMAX && HEAD % N2 == 0, "the direct head is one warp per row");
+    static_assert(ROWS <= NWARPS, "one warp per row computes the direct head");
     // bytes per t per array in staging, and the cp.async chunk covering them
     static constexpr int CH = ROWS * (int)sizeof(IO);
     static constexpr int CHUNK = CH < 16 ? CH : 16;
@@ -197,21 +204,44 @@ __device__ __forceinline__ void stage_tile(const IO *__restrict__ v, const IO *_
     cp_async_commit();
 }
 
+__device__ __forceinline__ float2 shfl_xor2(float2 a, int m) {
+    return make_float2(__shfl_xor_sync(0xffffffffu, a.x, m), __shfl_xor_sync(0xffffffffu, a.y, m));
+}
+
+// Named barrier over `count` threads (a multiple of 32), id 1..15.
+__device__ __forceinline__ void bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
+}
+
 template <int N2, int ROWS, int MINB, typename IO>
-__global__ void __launch_bounds__(ROWS *N2, MINB)
+__global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
     fftconv_fused_kernel(const IO *__restrict__ v, const IO *__restrict__ g, IO *__restrict__ r, int L, int D,
                          int groups_per_batch, int num_tiles, int vec_ok, const float2 *__restrict__ tw) {
     using C = FusedCfg<N2, ROWS, IO>;
-    constexpr int N1 = C::N1, N = C::N, M2 = C::M2, SC = C::SC, SF_N = C::SF_N, SI_M = C::SI_M;
-    constexpr int HEAD = C::HEAD, LMAX = C::LMAX;
+    constexpr int N1 = C::N1, N = C::N, M2 = C::M2, H = C::H, MH = C::MH;
+    constexpr int SC = C::SC, SF_N = C::SF_N, SI_M = C::SI_M, HEAD = C::HEAD, LMAX = C::LMAX;
+    constexpr int THREADS = C::THREADS;
     extern __shared__ float4 smem_raw[];
     float2 *xs = reinterpret_cast<float2 *>(smem_raw);
-    float2 *head = xs + ROWS * SC;
-    IO *sv = reinterpret_cast<IO *>(head + ROWS * HEAD);
+    float *hres = reinterpret_cast<float *>(xs + ROWS * SC);  // [ROWS][2*HEAD]: direct sums r_t, t < HEAD
+    IO *sv = reinterpret_cast<IO *>(hres + ROWS * 2 * HEAD);
     IO *sg = sv + LMAX * ROWS;
     float2 *red = reinterpret_cast<float2 *>(sg + LMAX * ROWS);  // [NWARPS][ROWS] partial norms
     float *alpha_row = reinterpret_cast<float *>(red + C::NWARPS * ROWS);  // [ROWS] balance scale
+    float2 *rot = reinterpret_cast<float2 *>(alpha_row + 2 * ROWS);       // [2h+s][H+1]
     const int tid = threadIdx.x;
+
+    // rot[2h+s][m] = omega_2N1^-((2h+1) m1), m1 = H s + m: untwist of the
+    // odd-frequency grid times the parity rotation of the last inverse step
+    for (int i = tid; i < 4 * H; i += THREADS) {
+        const int hs = i / H, m = i - hs * H, hh = hs >> 1, m1 = H * (hs & 1) + m;
+        rot[hs * (H + 1) + m] = cconj(c_w128[((2 * hh + 1) * m1 * (128 / (2 * N1))) & 127]);
+    }
+    // staging beyond L is never written by the copies: zero it once so loads need no bounds test
+    for (int i = L * ROWS + tid; i < LMAX * ROWS; i += THREADS) {
+        sv[i] = IO(0.f);
+        sg[i] = IO(0.f);
+    }
 
     int tile = blockIdx.x;
     if (tile >= num_tiles) return;
@@ -228,26 +258,34 @@ __global__ void __launch_bounds__(ROWS *N2, MINB)
         __syncthreads();  // staging complete; previous tile's I3 done with xs / head
 
         // ------------------------------------------------------------ F1
+        // thread (e, n2, c): half-spectrum e (k1 = 2k'+e) of column n2 of row c
         {
-            const int c = tid % ROWS, n2 = tid / ROWS;
-#pragma unroll
-            for (int n1 = 0; n1 * N2 < HEAD; ++n1) {
-                const int t = n2 + N2 * n1;
-                const bool ok = t < L;
-                head[c * HEAD + t] = make_float2(ok ? IO_t<IO>::cvt(sv[t * ROWS + c]) : 0.f,
-                                                 ok ? IO_t<IO>::cvt(sg[t * ROWS + c]) : 0.f);
-            }
-            // this thread's inputs z[n2 + N2 n1] and the row's stream norms
+            const int e = tid / (ROWS * N2);  // warp-uniform
+            const int c = tid % ROWS, n2 = (tid / ROWS) % N2;
             float2 zr[N2];
             float nv = 0.f, ng = 0.f;
 #pragma unroll
             for (int n1 = 0; n1 < N2; ++n1) {
                 const int t = n2 + N2 * n1;
-                float2 zv = make_float2(0.f, 0.f);
-                if (t < L) zv = make_float2(IO_t<IO>::cvt(sv[t * ROWS + c]), IO_t<IO>::cvt(sg[t * ROWS + c]));
+                const float2 zv = make_float2(IO_t<IO>::cvt(sv[t * ROWS + c]), IO_t<IO>::cvt(sg[t * ROWS + c]));
                 zr[n1] = zv;
                 nv = fmaf(zv.x, zv.x, nv);
                 ng = fmaf(zv.y, zv.y, ng);
+            }
+            // direct sums r_t = sum_{j<=t} v_j g_{t-j} for t < HEAD: warp w < ROWS
+            // handles row w, lane t
+            if ((tid >> 5) < ROWS) {
+                const int hc = tid >> 5, lt = tid & 31;
+                const float vt = IO_t<IO>::cvt(sv[lt * ROWS + hc]);
+                const float gt = IO_t<IO>::cvt(sg[lt * ROWS + hc]);
+                float acc = 0.f;
+#pragma unroll
+                for (int jj = 0; jj < HEAD; ++jj) {
+                    const float vj = __shfl_sync(0xffffffffu, vt, jj);
+                    const float gtj = __shfl_up_sync(0xffffffffu, gt, jj);
+                    if (lt >= jj) acc = fmaf(vj, gtj, acc);
+                }
+                hres[hc * 2 * HEAD + lt] = acc;
             }
 #pragma unroll
             for (int m = ROWS; m < 32; m <<= 1) {
@@ -258,34 +296,26 @@ __global__ void __launch_bounds__(ROWS *N2, MINB)
             __syncthreads();
             float2 tot = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int w = 0; w < C::NWARPS; ++w) {
+            for (int w = 0; w < C::NWARPS / 2; ++w) {  // the e == 0 warps cover each row once
                 tot.x += red[w * ROWS + c].x;
                 tot.y += red[w * ROWS + c].y;
             }
             const float alpha = balance_scale(tot.x, tot.y);
-            if (n2 == 0) alpha_row[c] = alpha;
-#pragma unroll
-            for (int n1 = 0; n1 < N2; ++n1) zr[n1].y *= alpha;
+            if (tid < ROWS) alpha_row[c] = alpha;
 
-            float2 *xrow = xs + c * SC + n2 * SF_N;
-            const float2 *t1 = tw + n2;
-#pragma unroll 1
-            for (int e = 0; e < 2; ++e) {
-                // x[n1] = z[n2 + N2 n1] * omega_2N1^((2e+1) n1), in bit-reversed slots
-                float2 x[N2];
+            // x[n1] = z[n2 + N2 n1] * omega_2N1^((2e+1) n1), in bit-reversed slots
+            float2 x[N2];
 #pragma unroll
-                for (int n1 = 0; n1 < N2; ++n1) {
-                    const float2 zv = zr[n1];
-                    const float2 w = e ? tw_const(3 * n1, 2 * N1) : tw_const(n1, 2 * N1);
-                    x[bitrev(n1, C::LOG_N2)] = n1 == 0 ? zv : cmul(zv, w);
-                }
-                fft_dit<N2, false>(x);  // x[k'] -> k1 = 2k' + e
-#pragma unroll
-                for (int kp = 0; kp < N2; ++kp) {
-                    const int k1 = 2 * kp + e;
-                    xrow[k1] = cmul(x[kp], __ldg(t1 + k1 * N2));
-                }
+            for (int n1 = 0; n1 < N2; ++n1) {
+                const float2 zv = make_float2(zr[n1].x, alpha * zr[n1].y);
+                const float2 w = e ? tw_const(3 * n1, 2 * N1) : tw_const(n1, 2 * N1);
+                x[bitrev(n1, C::LOG_N2)] = n1 == 0 ? zv : cmul(zv, w);
             }
+            fft_dit<N2, false>(x);  // x[k'] -> k1 = 2k' + e
+            float2 *xrow = xs + c * SC + n2 * SF_N + e;
+            const float2 *t1 = tw + e * N2 + n2;
+#pragma unroll
+            for (int kp = 0; kp < N2; ++kp) xrow[2 * kp] = cmul(x[kp], __ldg(t1 + 2 * kp * N2));
         }
         __syncthreads();  // exchange complete; staging free
 
@@ -299,97 +329,126 @@ __global__ void __launch_bounds__(ROWS *N2, MINB)
         }
 
         // ------------------------------------------------------------ F3
+        // Column pair (j, N1-1-j) of row c is shared by two lanes s = 0, 1 (lane ^ 16).
+        // Lane s keeps the even rows of its own column and receives the odd rows
+        // of the other; that set is closed under both pairings (mirror: row k2 of
+        // one column with row N2-1-k2 of the other; half-length partner: row k2
+        // with row M2-1-k2), so both lanes run the same code.
         {
-            const int c = tid / N2, j = tid % N2;
+            const int c = tid / (2 * N2), rr = tid % (2 * N2);
+            const int s = (rr >> 4) & 1, j = (rr >> 5) * 16 + (rr & 15);
+            const int own_col = s ? N1 - 1 - j : j;
+            const int rec_col = N1 - 1 - own_col;
             float2 *xrow = xs + c * SC;
-            const int ka = j, kb = N1 - 1 - j;
-            float2 A[N2], Bc[N2];
+            float2 own[H], rec[H];
+            {
+                float2 x[N2];
 #pragma unroll
-            for (int n2 = 0; n2 < N2; ++n2) {
-                A[bitrev(n2, C::LOG_N2)] = xrow[n2 * SF_N + ka];
-                Bc[bitrev(n2, C::LOG_N2)] = xrow[n2 * SF_N + kb];
-            }
-            fft_dit<N2, false>(A);   // A[k2]  = Z[ka + N1 k2]
-            fft_dit<N2, false>(Bc);  // Bc[k2] = Z[kb + N1 k2]
-            // mirror of (ka, k2) is (kb, N2-1-k2)
+                for (int n2 = 0; n2 < N2; ++n2) x[n2] = xrow[n2 * SF_N + own_col];
+                // first radix-2 DIF stage over n2: even rows <- x[n] + x[n+H], odd <- (x[n] - x[n+H]) w^n
 #pragma unroll
-            for (int k2 = 0; k2 < N2; ++k2) {
-                const float2 x = spectral_product(A[k2], Bc[N2 - 1 - k2]);
-                A[k2] = x;
-                Bc[N2 - 1 - k2] = cconj(x);
+                for (int n = 0; n < H; ++n) {
+                    const float2 a = x[n], bq = x[n + H];
+                    own[bitrev(n, C::LOG_H)] = cadd(a, bq);
+                    const float2 d = csub(a, bq);
+                    const float2 w = n == 0 ? d : (4 * n == N2 ? make_float2(d.y, -d.x) : cmul(d, tw_const(n, N2)));
+                    rec[bitrev(n, C::LOG_H)] = shfl_xor2(w, 16);  // odd rows of the other column
+                }
             }
-            // half-length partner of (ka, k2) is (kb, M2-1-k2)
+            fft_dit<H, false>(own);  // own[k] = Z[own_col + N1 (2k)]
+            fft_dit<H, false>(rec);  // rec[k] = Z[rec_col + N1 (2k+1)]
+            // spectral product: mirror of (own_col, 2k) is (rec_col, N2-1-2k) = rec[H-1-k]
+#pragma unroll
+            for (int k = 0; k < H; ++k) {
+                const float2 xv = spectral_product(own[k], rec[H - 1 - k]);
+                own[k] = xv;
+                rec[H - 1 - k] = cconj(xv);
+            }
+            // real-inverse packing: partner of (own_col, 2k) is (rec_col, M2-1-2k) = rec[MH-1-k]
             const float2 *ptab = tw + C::TW_P;
 #pragma unroll
-            for (int k2 = 0; k2 < M2; ++k2) {
+            for (int k = 0; k < MH; ++k) {
                 float2 ca, cb;
-                pack_pair(A[k2], Bc[M2 - 1 - k2], __ldg(ptab + k2 * N1 + ka), __ldg(ptab + (M2 - 1 - k2) * N1 + kb),
-                          ca, cb);
-                A[k2] = ca;
-                Bc[M2 - 1 - k2] = cb;
+                pack_pair(own[k], rec[MH - 1 - k], __ldg(ptab + (2 * k) * N1 + own_col),
+                          __ldg(ptab + (M2 - 1 - 2 * k) * N1 + rec_col), ca, cb);
+                own[k] = ca;
+                rec[MH - 1 - k] = cb;
             }
-            // first inverse step: M2-point DFT over k2, then its twiddle
-            float2 ya[M2], yb[M2];
+            // first inverse step (M2-point DFT over k2) split by parity of k2:
+            // E of own column here, O of own column at the partner
+            float2 eo[MH], oo[MH];
 #pragma unroll
-            for (int k2 = 0; k2 < M2; ++k2) {
-                ya[bitrev(k2, C::LOG_M2)] = A[k2];
-                yb[bitrev(k2, C::LOG_M2)] = Bc[k2];
+            for (int k = 0; k < MH; ++k) {
+                eo[bitrev(k, C::LOG_MH)] = own[k];
+                oo[bitrev(k, C::LOG_MH)] = rec[k];
             }
-            fft_dit<M2, true>(ya);
-            fft_dit<M2, true>(yb);
+            fft_dit<MH, true>(eo);  // E of own_col
+            fft_dit<MH, true>(oo);  // O of rec_col
+            float2 y[M2];
+#pragma unroll
+            for (int m = 0; m < MH; ++m) {
+                const float2 op = shfl_xor2(oo[m], 16);  // O of own_col
+                const float2 t = m == 0 ? op : cmul_conj(op, tw_const(m, M2));
+                y[m] = cadd(eo[m], t);
+                y[m + MH] = csub(eo[m], t);
+            }
             const float2 *qtab = tw + C::TW_Q;
-            __syncwarp();  // the inverse buffer aliases this row's forward buffer
+            if (N2 > 16)
+                bar_sync(1 + c, 2 * N2);  // both warps of the row are done reading it
+            else
+                __syncwarp();
+            xrow[own_col] = y[0];
 #pragma unroll
-            for (int m2 = 0; m2 < M2; ++m2) {
-                xrow[m2 * SI_M + ka] = cmul(ya[m2], __ldg(qtab + m2 * N1 + ka));
-                xrow[m2 * SI_M + kb] = cmul(yb[m2], __ldg(qtab + m2 * N1 + kb));
-            }
+            for (int m2 = 1; m2 < M2; ++m2) xrow[m2 * SI_M + own_col] = cmul(y[m2], __ldg(qtab + m2 * N1 + own_col));
         }
         __syncthreads();
 
         // ------------------------------------------------------------ I3
+        // thread (m2, s, h, c): the N1-point inverse DFT over k1 = 2i + h of row
+        // m2 of row c; lane s takes the even (s=0) or odd (s=1) i.
         {
-            const int c = tid % ROWS, u = tid / ROWS;
-            const int m2 = u >> 1, h = u & 1;
-            const float2 *xi = xs + c * SC + m2 * SI_M + h;
-            float2 x[N2];
+            const int c = tid % ROWS, h = (tid / ROWS) & 1, s = (tid / (2 * ROWS)) & 1, m2 = tid / (4 * ROWS);
+            const float2 *xi = xs + c * SC + m2 * SI_M + 2 * s + h;
+            float2 x[H];
 #pragma unroll
-            for (int i = 0; i < N2; ++i) x[bitrev(i, C::LOG_N2)] = xi[2 * i];
-            fft_dit<N2, true>(x);
-            // untwist and odd-k1 rotation: times omega_2N1^-((2h+1) m1)
+            for (int i = 0; i < H; ++i) x[bitrev(i, C::LOG_H)] = xi[4 * i];
+            fft_dit<H, true>(x);  // E (s = 0) or O (s = 1), m in [0, H)
+            // out[m] = E[m] + w^-m O[m] (m < H), out[m+H] = E[m] - w^-m O[m]; lane s keeps m1 = H s + m
+            const float sg1 = s ? -1.f : 1.f;
+            float2 out[H];
 #pragma unroll
-            for (int m1 = 1; m1 < N2; ++m1) {
-                const float2 w = h ? tw_const(3 * m1, 2 * N1) : tw_const(m1, 2 * N1);
-                x[m1] = cmul_conj(x[m1], w);
+            for (int m = 0; m < H; ++m) {
+                float2 mine = x[m];
+                if (m > 0) {
+                    const float2 w = tw_const(m, N2);
+                    const float2 ws = s ? w : make_float2(1.f, 0.f);
+                    mine = cmul_conj(mine, ws);
+                }
+                const float2 other = shfl_xor2(mine, 2 * ROWS);
+                float2 o = make_float2(fmaf(sg1, mine.x, other.x), fmaf(sg1, mine.y, other.y));
+                out[m] = cmul(o, rot[(2 * h + s) * (H + 1) + m]);
             }
+            // combine the two parities h: lane h keeps m in [h H/2, (h+1) H/2)
             const int d = d0 + c;
             const bool dok = d < D;
-            IO *rp = r + boff + d;
-            const float s = 1.f / (4.f * (float)N * alpha_row[c]);
-            const float2 *hrow = head + c * HEAD;
+            const float sc = 1.f / (4.f * (float)N * alpha_row[c]);
+            const int t0 = 2 * m2 + N2 * (H * s + (H / 2) * h);
+            IO *rp = r + boff + d + (int64_t)t0 * D;
+            const int64_t step = (int64_t)N2 * D;
 #pragma unroll
-            for (int i = 0; i < N2 / 2; ++i) {
-                const float2 send = h ? x[i] : x[N2 / 2 + i];
-                const float2 own = h ? x[N2 / 2 + i] : x[i];
-                float2 o;
-                o.x = own.x + __shfl_xor_sync(0xffffffffu, send.x, ROWS);
-                o.y = own.y + __shfl_xor_sync(0xffffffffu, send.y, ROWS);
-                const int m1 = i + h * (N2 / 2);
-                const int t = 2 * m2 + N2 * m1;
-                float r0 = o.x * s, r1 = o.y * s;
+            for (int i = 0; i < H / 2; ++i) {
+                const float2 send = h ? out[i] : out[H / 2 + i];
+                const float2 keep = h ? out[H / 2 + i] : out[i];
+                const float2 o = cadd(keep, shfl_xor2(send, ROWS));
+                const int t = t0 + N2 * i;
+                float r0 = o.x * sc, r1 = o.y * sc;
                 if (i * N2 < HEAD && t < HEAD) {
-                    float a0 = 0.f, a1 = 0.f;
-                    for (int jj = 0; jj <= t; ++jj) {
-                        const float vj = hrow[jj].x;
-                        a0 = fmaf(vj, hrow[t - jj].y, a0);
-                        a1 = fmaf(vj, hrow[t + 1 - jj].y, a1);
-                    }
-                    a1 = fmaf(hrow[t + 1].x, hrow[0].y, a1);
-                    r0 = a0;
-                    r1 = a1;
+                    r0 = hres[c * 2 * HEAD + t];
+                    r1 = hres[c * 2 * HEAD + t + 1];
                 }
-                if (dok && t < L) IO_t<IO>::st(rp + (int64_t)t * D, r0);
-                if (dok && t + 1 < L) IO_t<IO>::st(rp + (int64_t)(t + 1) * D, r1);
+                if (dok && t < L) IO_t<IO>::st(rp, r0);
+                if (dok && t + 1 < L) IO_t<IO>::st(rp + D, r1);
+                rp += step;
             }
         }
     }
