@@ -64,6 +64,11 @@ def _bind(lib):
     lib.oracle_conv_i32in.restype = None
     lib.oracle_conv_i32in_points.argtypes = [_PTR, _PTR, _I64, _I64, _I64, _PTR, _I64, _PTR]
     lib.oracle_conv_i32in_points.restype = None
+    lib.oracle_conv_bwd_f32in.argtypes = [_PTR, _PTR, _PTR, _I64, _I64, _I64, _PTR, _PTR, _PTR, _PTR]
+    lib.oracle_conv_bwd_f32in.restype = None
+    lib.oracle_conv_bwd_f32in_points.argtypes = [_PTR, _PTR, _PTR, _I64, _I64, _I64, _PTR, _I64, _PTR, _PTR,
+                                                 _PTR, _PTR]
+    lib.oracle_conv_bwd_f32in_points.restype = None
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
@@ -156,6 +161,33 @@ def causal_conv_int_points(v: np.ndarray, g: np.ndarray, pts: np.ndarray, lib=No
     r = np.empty(pts.shape[0], np.int64)
     lib.oracle_conv_i32in_points(_ptr(v), _ptr(g), B, L, D, _ptr(pts), pts.shape[0], _ptr(r))
     return r
+
+
+def causal_conv_bwd(dr: np.ndarray, v: np.ndarray, g: np.ndarray, lib=None):
+    """Gradients of the causal convolution (float inputs widened exactly to
+    double): returns (dv, den_dv, dg, den_dg), each float64 [B, L, D], with
+    dv_j = sum_{t>=j} dr_t g_{t-j} and dg_k = sum_{t>=k} dr_t v_{t-k}."""
+    lib = lib or load()
+    B, L, D = _check3(v, g)
+    if dr.shape != v.shape:
+        raise ValueError("dr must have the shape of v")
+    dr, v, g = (np.ascontiguousarray(x, np.float32) for x in (dr, v, g))
+    out = [np.empty((B, L, D), np.float64) for _ in range(4)]
+    lib.oracle_conv_bwd_f32in(_ptr(dr), _ptr(v), _ptr(g), B, L, D, *(_ptr(o) for o in out))
+    return tuple(out)
+
+
+def causal_conv_bwd_points(dr, v, g, pts, lib=None):
+    lib = lib or load()
+    B, L, D = _check3(v, g)
+    pts = np.ascontiguousarray(pts, np.int64).reshape(-1, 3)
+    if pts.size and ((pts.min(0) < 0).any() or (pts.max(0) >= np.array([B, L, D])).any()):
+        raise ValueError("sample point out of range")
+    dr, v, g = (np.ascontiguousarray(x, np.float32) for x in (dr, v, g))
+    out = [np.empty(pts.shape[0], np.float64) for _ in range(4)]
+    lib.oracle_conv_bwd_f32in_points(_ptr(dr), _ptr(v), _ptr(g), B, L, D, _ptr(pts), pts.shape[0],
+                                     *(_ptr(o) for o in out))
+    return tuple(out)
 
 
 def centered_mod(x: np.ndarray, p: int) -> np.ndarray:

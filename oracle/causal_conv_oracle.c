@@ -26,8 +26,18 @@
  * (b, t, d) sits at (b*L + t)*D + d.  Points for the sampled variants are
  * given as n triples (b, t, d), flattened.
  *
+ * Backward (gradient of a scalar loss through r, given dr = dLoss/dr): the
+ * derivatives of the sum above are, per row,
+ *
+ *     dv_j = sum_{t=j}^{L-1} dr_t * g_{t-j},     dg_k = sum_{t=k}^{L-1} dr_t * v_{t-k},
+ *
+ * again evaluated term by term (ascending t) in double, with the matching
+ * error-bound denominators sum |dr_t g_{t-j}| and sum |dr_t v_{t-k}|.
+ *
  * Parity pins: see tests/test_oracle_pins.py (delta inputs, closed-form sums,
- * commutativity/bilinearity/shift, causality, wrap-around, brute force).
+ * commutativity/bilinearity/shift, causality, wrap-around, brute force, and
+ * for the backward: the adjoint identity, numpy.convolve on reversed rows,
+ * torch autograd).
  */
 #include <stdint.h>
 #include <math.h>
@@ -136,6 +146,47 @@ void oracle_conv_i32in_points(const int32_t *v, const int32_t *g, int64_t B, int
 #pragma omp parallel for schedule(dynamic, 4)
     for (int64_t i = 0; i < n; ++i)
         r[i] = point_i32in(v, g, L, D, pts[3 * i], pts[3 * i + 1], pts[3 * i + 2]);
+}
+
+/* ---- backward ---------------------------------------------------------- */
+
+/* dv[b,j,d] (with den) for one point: sum over t >= j of dr_t g_{t-j}. */
+static void point_bwd_f32in(const float *dr, const float *k, int64_t L, int64_t D,
+                            int64_t b, int64_t j, int64_t d, double *out, double *den)
+{
+    double acc = 0.0, mag = 0.0;
+    for (int64_t t = j; t < L; ++t) {
+        double p = (double)dr[IDX(b, t, d)] * (double)k[IDX(b, t - j, d)];
+        acc += p;
+        mag += fabs(p);
+    }
+    *out = acc;
+    *den = mag;
+}
+
+/* Full gradients: dv from (dr, g), dg from (dr, v). */
+void oracle_conv_bwd_f32in(const float *dr, const float *v, const float *g, int64_t B, int64_t L, int64_t D,
+                           double *dv, double *den_dv, double *dg, double *den_dg)
+{
+    int64_t n = B * L * D;
+#pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t d = i % D, j = (i / D) % L, b = i / (D * L);
+        point_bwd_f32in(dr, g, L, D, b, j, d, &dv[i], &den_dv[i]);
+        point_bwd_f32in(dr, v, L, D, b, j, d, &dg[i], &den_dg[i]);
+    }
+}
+
+void oracle_conv_bwd_f32in_points(const float *dr, const float *v, const float *g, int64_t B, int64_t L,
+                                  int64_t D, const int64_t *pts, int64_t n, double *dv, double *den_dv,
+                                  double *dg, double *den_dg)
+{
+    (void)B;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t i = 0; i < n; ++i) {
+        point_bwd_f32in(dr, g, L, D, pts[3 * i], pts[3 * i + 1], pts[3 * i + 2], &dv[i], &den_dv[i]);
+        point_bwd_f32in(dr, v, L, D, pts[3 * i], pts[3 * i + 1], pts[3 * i + 2], &dg[i], &den_dg[i]);
+    }
 }
 
 /* Number of OpenMP threads the loops above use (for the baseline report). */

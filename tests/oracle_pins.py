@@ -35,8 +35,8 @@ def load_golden(path: str = GOLDEN):
             if not line or line.startswith("#"):
                 continue
             key, *rest = line.split()
-            if key == "case":
-                cur = {"name": rest[0], "shape": tuple(int(x) for x in rest[1:4])}
+            if key in ("case", "bwdcase"):
+                cur = {"name": rest[0], "kind": key, "shape": tuple(int(x) for x in rest[1:4])}
                 cases.append(cur)
             else:
                 cur[key] = np.array([float(x) for x in rest], np.float64).reshape(cur["shape"])
@@ -51,6 +51,10 @@ def _rng(seed):
 
 def pin_golden(lib):
     for c in load_golden():
+        if c["kind"] == "bwdcase":
+            dv, _, dg, _ = oracle.causal_conv_bwd(c["dr"], c["v"], c["g"], lib=lib)
+            assert np.array_equal(dv, c["dv"]) and np.array_equal(dg, c["dg"]), (c["name"], dv.ravel(), dg.ravel())
+            continue
         r, den = oracle.causal_conv(c["v"], c["g"], lib=lib)
         assert np.array_equal(r, c["r"]), (c["name"], r.ravel(), c["r"].ravel())
         assert np.array_equal(den, c["den"]), (c["name"], den.ravel(), c["den"].ravel())
@@ -220,8 +224,75 @@ def pin_points_match_full(lib):
     assert np.array_equal(oracle.causal_conv_int_points(vi, gi, pts, lib=lib), ri[pts[:, 0], pts[:, 1], pts[:, 2]])
 
 
+# ---------------------------------------------------------- backward pins
+
+def pin_bwd_adjoint(lib):
+    """<dr, r(v, g)> = <dv, v> = <dg, g>: the gradient of the bilinear form
+    sum_t dr_t r_t, checked against the (separately pinned) forward."""
+    B, L, D = 2, 97, 3
+    rng = _rng(20)
+    dr, v, g = (rng.standard_normal((B, L, D)).astype(np.float32) for _ in range(3))
+    r, _ = oracle.causal_conv(v, g, lib=lib)
+    dv, _, dg, _ = oracle.causal_conv_bwd(dr, v, g, lib=lib)
+    for b in range(B):
+        for d in range(D):
+            lhs = float(np.dot(dr[b, :, d].astype(np.float64), r[b, :, d]))
+            assert abs(lhs - np.dot(dv[b, :, d], v[b, :, d].astype(np.float64))) <= 1e-11 * (1 + abs(lhs))
+            assert abs(lhs - np.dot(dg[b, :, d], g[b, :, d].astype(np.float64))) <= 1e-11 * (1 + abs(lhs))
+
+
+def pin_bwd_numpy_reversal(lib):
+    """dv = rev(convolve(rev(dr), g)[:L]) with numpy's convolution."""
+    B, L, D = 1, 64, 4
+    rng = _rng(21)
+    dr, v, g = (rng.standard_normal((B, L, D)).astype(np.float32) for _ in range(3))
+    dv, den_dv, dg, _ = oracle.causal_conv_bwd(dr, v, g, lib=lib)
+    for d in range(D):
+        rdr = dr[0, ::-1, d].astype(np.float64)
+        ref_v = np.convolve(rdr, g[0, :, d].astype(np.float64))[:L][::-1]
+        ref_g = np.convolve(rdr, v[0, :, d].astype(np.float64))[:L][::-1]
+        assert np.allclose(dv[0, :, d], ref_v, rtol=0, atol=1e-12 * den_dv.max())
+        assert np.allclose(dg[0, :, d], ref_g, rtol=0, atol=1e-12 * den_dv.max() + 1e-12 * np.abs(ref_g).max())
+        ad = np.convolve(np.abs(rdr), np.abs(g[0, :, d].astype(np.float64)))[:L][::-1]
+        assert np.allclose(den_dv[0, :, d], ad, rtol=1e-13, atol=0)
+
+
+def pin_bwd_autograd(lib):
+    """torch autograd (fp64, CPU) through a forward built from torch's conv1d."""
+    import torch
+    B, L, D = 1, 40, 3
+    rng = _rng(22)
+    dr, v, g = (rng.standard_normal((B, L, D)).astype(np.float32) for _ in range(3))
+    tv = torch.tensor(v, dtype=torch.float64, requires_grad=True)
+    tg = torch.tensor(g, dtype=torch.float64, requires_grad=True)
+    # r[b, t, d] = sum_j v[b, j, d] g[b, t-j, d]: depthwise conv1d of left-padded v with flipped g
+    x = tv.permute(0, 2, 1).reshape(1, B * D, L)
+    w = tg.permute(0, 2, 1).reshape(B * D, 1, L).flip(-1)
+    r = torch.nn.functional.conv1d(torch.nn.functional.pad(x, (L - 1, 0)), w, groups=B * D)
+    r = r.reshape(B, D, L).permute(0, 2, 1)
+    (r * torch.tensor(dr, dtype=torch.float64)).sum().backward()
+    dv, _, dg, _ = oracle.causal_conv_bwd(dr, v, g, lib=lib)
+    assert np.allclose(dv, tv.grad.numpy(), rtol=1e-12, atol=1e-12)
+    assert np.allclose(dg, tg.grad.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def pin_bwd_delta(lib):
+    B, L, D = 1, 33, 2
+    rng = _rng(23)
+    v, g = (rng.standard_normal((B, L, D)).astype(np.float32) for _ in range(2))
+    dr = np.zeros((B, L, D), np.float32)
+    dr[:, L - 1, :] = 1.0  # only the last output matters: dv_j = g_{L-1-j}
+    dv, _, dg, _ = oracle.causal_conv_bwd(dr, v, g, lib=lib)
+    assert np.array_equal(dv, g[:, ::-1, :].astype(np.float64))
+    assert np.array_equal(dg, v[:, ::-1, :].astype(np.float64))
+    pts = np.array([(0, j, d) for j in range(L) for d in range(D)], np.int64)
+    pv, _, pg, _ = oracle.causal_conv_bwd_points(dr, v, g, pts, lib=lib)
+    assert np.array_equal(pv, dv.reshape(-1)) and np.array_equal(pg, dg.reshape(-1))
+
+
 PINS = [pin_golden, pin_delta, pin_closed_forms, pin_numpy_convolve, pin_fft_independent,
-        pin_symmetries, pin_causality, pin_den, pin_points_match_full]
+        pin_symmetries, pin_causality, pin_den, pin_points_match_full,
+        pin_bwd_adjoint, pin_bwd_numpy_reversal, pin_bwd_autograd, pin_bwd_delta]
 
 
 def run_all(lib):

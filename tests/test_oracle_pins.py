@@ -37,6 +37,10 @@ MUTANTS = {
                           "#define IDX(b, t, d) (((int64_t)(b) * D + (d)) * L + (t))"),
     "den_signed": ("mag += fabs(p);", "mag += p;"),
     "int_narrow_accumulator": ("int64_t acc = 0;", "int16_t acc = 0;"),
+    "bwd_dropped_term": ("for (int64_t t = j; t < L; ++t) {", "for (int64_t t = j + 1; t < L; ++t) {"),
+    "bwd_correlation_flip": ("(double)k[IDX(b, t - j, d)]", "(double)k[IDX(b, L - 1 - (t - j), d)]"),
+    "bwd_swapped_kernels": ("point_bwd_f32in(dr, g, L, D, b, j, d, &dv[i], &den_dv[i]);",
+                            "point_bwd_f32in(dr, v, L, D, b, j, d, &dv[i], &den_dv[i]);"),
 }
 
 
