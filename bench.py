@@ -49,6 +49,9 @@ def parse_args():
     ap.add_argument("--workload", default="small_f32", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--path", choices=["fwd", "bwd", "decode"], default="fwd",
+                    help="fwd: the causal convolution (default line); bwd: its gradients (dv, dg); "
+                         "decode: one autoregressive step at t = L-1 from [B, L, D] caches")
     ap.add_argument("--shape", default=None,
                     help="B,L,D override of the workload's sizes (same recipe); for small profiler captures")
     return ap.parse_args()
@@ -283,7 +286,28 @@ def run_ours(args, rank, world, local):
     sets = [(v0, g0, torch.empty_like(v0))] + [(v0.clone(), g0.clone(), torch.empty_like(v0)) for _ in
                                                 range(n_sets - 1)]
     stream = torch.cuda.current_stream(dev)
-    fn = ssm.causal_conv
+    if args.path == "fwd":
+        def fn(a, b, out, stream):
+            ssm.causal_conv(a, b, out=out, stream=stream)
+        bytes_per_step, launches_per_step = 3 * w.units * w.elem_bytes, 1
+    elif args.path == "bwd":
+        # dr is the third buffer of the set; dv, dg get their own buffers
+        bwd_out = [(torch.empty_like(v0), torch.empty_like(v0)) for _ in range(n_sets)]
+
+        def fn(a, b, out, stream, _k=[0]):
+            dv, dg = bwd_out[_k[0] % n_sets]
+            _k[0] += 1
+            ssm.causal_conv_bwd(out, a, b, dv=dv, dg=dg, stream=stream)
+        for _, _, c in sets:
+            c.copy_(sets[0][0])
+        bytes_per_step, launches_per_step = 5 * w.units * w.elem_bytes, 2
+    else:
+        dec_ws = torch.empty(ssm.decode_workspace_bytes(v0.dtype, w.B, w.D, w.L - 1), dtype=torch.uint8, device=dev)
+        dec_out = torch.empty((w.B, w.D), dtype=v0.dtype, device=dev)
+
+        def fn(a, b, out, stream):
+            ssm.causal_conv_decode(a, b, w.L - 1, out=dec_out, workspace=dec_ws, stream=stream)
+        bytes_per_step, launches_per_step = (2 * w.L + 1) * w.B * w.D * w.elem_bytes, 2
 
     for i in range(args.warmup):
         a, b, c = sets[i % n_sets]
@@ -303,8 +327,9 @@ def run_ours(args, rank, world, local):
         barrier()
     ms = max_over_ranks(start.elapsed_time(end), pg, dev)
     ms_per_step = ms / args.steps
-    units_total = w.units * world * args.steps
-    ups, gbs = throughput(w.units, world, args.steps, ms, 3 * w.elem_bytes)
+    units_step = w.units if args.path != "decode" else w.B * w.D
+    ups, _ = throughput(units_step, world, args.steps, ms, 1)
+    gbs = bytes_per_step * world * args.steps / (ms * 1e-3) / 1e9
 
     # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -327,13 +352,15 @@ def run_ours(args, rank, world, local):
 
     peak, peak_src = measured_peaks()
     kernel = "ntt_conv_kernel" if w.dtype == "i32" else ("fftconv_fused_kernel" if w.L <= 1024 else "bigconv_kernel")
-    per_launch_bytes = 3 * w.units * w.elem_bytes
-    achieved = per_launch_bytes / (ms_per_step * 1e-3) / 1e9
+    if args.path == "decode":
+        kernel = "decode_partial_kernel"
+    per_launch_bytes = bytes_per_step // launches_per_step if args.path == "bwd" else bytes_per_step
+    achieved = bytes_per_step / (ms_per_step * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": {"f32": "f32", "bf16": "f32", "i32": "u32"}[w.dtype], "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "L": w.L, "D": w.D, "io_dtype": w.dtype,
+        "config": {"workload": w.name, "path": args.path, "B": w.B, "L": w.L, "D": w.D, "io_dtype": w.dtype,
                    "transform_len": 2 ** math.ceil(math.log2(2 * w.L)),
                    "l2": f"inputs larger than L2: {n_sets} rotating (v,g,r) sets of {set_bytes / 2 ** 20:.0f} MiB",
                    "parallelism": f"dp{world} (independent batches, no collective)"},
@@ -342,13 +369,16 @@ def run_ours(args, rank, world, local):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
                      "kernel": kernel, "algorithmic_bytes_per_launch": per_launch_bytes,
-                     "traffic": None if args.shape else recorded_traffic(w.name, kernel)},
+                     "traffic": None if (args.shape or args.path != "fwd") else recorded_traffic(w.name, kernel)},
         "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": 2 * w.units * w.elem_bytes,
                 "d2h_bytes_per_step": w.units * w.elem_bytes, "steps": e2e_steps,
                 "path": "causal_conv_from_host (pinned host buffers)"},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * launches_per_step,
         "clocks": clk.report(),
     }
+    if args.path != "fwd":  # the host-buffer leg and CPU baseline describe the forward line only
+        line.pop("e2e")
+        args.no_cpu_baseline = True
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu_ups, cores, desc, secs = cpu_oracle_rate(w, v_np, g_np, budget_s=15.0)
         line["cpu_baseline"] = {"value": cpu_ups * 3 * w.elem_bytes / 1e9, "unit": "GB/s", "cores": cores,

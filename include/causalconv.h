@@ -110,6 +110,60 @@ CC_API int causal_ntt_conv_i32(const int32_t *v, const int32_t *g, int32_t *r,
                         void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * causal_fftconv_bwd_f32 -- gradients of the causal convolution for training
+ * (the models on "Caracal: Causal Architecture via Spectral Mixing" train with
+ * next-token cross-entropy, "Loss / training strategy").  Given
+ * dr = dLoss/dr, per (b, d) row:
+ *
+ *     dv[b, j, d] = sum_{t=j..L-1} dr[b, t, d] * g[b, t-j, d]
+ *     dg[b, k, d] = sum_{t=k..L-1} dr[b, t, d] * v[b, t-k, d]
+ *
+ * Both are anti-causal correlations; with rev(x)_t = x_{L-1-t} they equal
+ * rev(conv(rev(dr), g)) and rev(conv(rev(dr), v)), which is how they are
+ * computed: two launches of the forward kernels with time-reversed input and
+ * output indexing (no extra copies).
+ *   dr, v, g  [B, L, D] float32 (device); dv, dg [B, L, D] float32 outputs
+ *   (device), overlapping none of the inputs or each other.
+ * Accuracy, ranges, workspace and errors as causal_fftconv_f32, with the
+ * bound taken against sum_t |dr_t g_{t-j}| (resp. |dr_t v_{t-k}|).
+ */
+CC_API int causal_fftconv_bwd_f32(const float *dr, const float *v, const float *g, float *dv, float *dg,
+                                  int64_t B, int64_t L, int64_t D,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/* causal_fftconv_bwd_bf16 -- as causal_fftconv_bwd_f32 with bfloat16 I/O. */
+CC_API int causal_fftconv_bwd_bf16(const uint16_t *dr, const uint16_t *v, const uint16_t *g, uint16_t *dv,
+                                   uint16_t *dg, int64_t B, int64_t L, int64_t D,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * causal_conv_decode_f32 -- one autoregressive step: the output of the newest
+ * position t from cached value and gate streams (next-token prediction in
+ * "Caracal: Causal Architecture via Spectral Mixing", framework figure):
+ *
+ *     r[b, d] = sum_{j=0..t} v[b, j, d] * g[b, t-j, d]
+ *
+ *   v, g   [B, Lcap, D] float32 caches (device), positions 0..t filled
+ *   r      [B, D] float32 output (device), overlapping neither cache
+ *   t      0 <= t < Lcap, the same position for every batch row
+ *   workspace  device scratch of at least causal_conv_decode_workspace_bytes()
+ *              bytes (fp64 partial sums of the split reduction; required)
+ * Direct O(t) summation (no transform), split over j across the GPU, fp64
+ * accumulation, fixed-order reduction: deterministic and within one float
+ * rounding of the exact sum.  B <= 65535.  Errors as causal_fftconv_f32;
+ * int32 is CC_ERR_UNSUPPORTED.
+ */
+CC_API int causal_conv_decode_f32(const float *v, const float *g, float *r, int64_t B, int64_t Lcap, int64_t D,
+                                  int64_t t, void *workspace, size_t workspace_bytes, void *stream);
+
+/* causal_conv_decode_bf16 -- as causal_conv_decode_f32 with bfloat16 caches and output. */
+CC_API int causal_conv_decode_bf16(const uint16_t *v, const uint16_t *g, uint16_t *r, int64_t B, int64_t Lcap,
+                                   int64_t D, int64_t t, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes causal_conv_decode_* needs for (B, D, t); (size_t)-1 if invalid. */
+CC_API size_t causal_conv_decode_workspace_bytes(int dtype, int64_t B, int64_t D, int64_t t);
+
+/*
  * causal_conv_from_host -- the same convolution for HOST buffers: enqueues on
  * `stream` the copy of v_host and g_host into the caller's device buffers
  * v_dev and g_dev, the convolution into r_dev, and the copy of r_dev back

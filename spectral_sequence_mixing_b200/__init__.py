@@ -21,7 +21,8 @@ from . import _lib
 from ._lib import (CC_DTYPE_BF16, CC_DTYPE_F32, CC_DTYPE_I32, CausalConvError, load, strerror)
 
 __all__ = [
-    "causal_fftconv_f32", "causal_fftconv_bf16", "causal_ntt_conv_i32", "causal_conv",
+    "causal_fftconv_f32", "causal_fftconv_bf16", "causal_ntt_conv_i32", "causal_conv", "causal_conv_bwd",
+    "causal_conv_decode", "decode_workspace_bytes",
     "causal_conv_from_host", "workspace_bytes", "max_len", "ntt_params", "strerror",
     "CausalConvError", "CC_DTYPE_F32", "CC_DTYPE_BF16", "CC_DTYPE_I32",
 ]
@@ -93,6 +94,65 @@ def causal_conv(v: torch.Tensor, g: torch.Tensor, out=None, workspace=None, stre
     if v.dtype not in _DT:
         raise TypeError(f"unsupported dtype {v.dtype}")
     return _run(_DT[v.dtype], v, g, out, workspace, stream)
+
+
+def causal_conv_bwd(dr: torch.Tensor, v: torch.Tensor, g: torch.Tensor, dv=None, dg=None, workspace=None,
+                    stream=None):
+    """Gradients (dv, dg) of the causal convolution given dr = dLoss/dr
+    (float32 or bfloat16 [B, L, D]):  dv_j = sum_{t>=j} dr_t g_{t-j},
+    dg_k = sum_{t>=k} dr_t v_{t-k}."""
+    dtype = v.dtype
+    if dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"unsupported dtype {dtype}")
+    for name, t in (("dr", dr), ("v", v), ("g", g)):
+        _check(t, name, dtype, v.shape)
+        if not t.is_cuda or t.device != v.device:
+            raise ValueError("dr, v, g must be CUDA tensors on the same device")
+    dv = torch.empty_like(v) if dv is None else dv
+    dg = torch.empty_like(v) if dg is None else dg
+    _check(dv, "dv", dtype, v.shape)
+    _check(dg, "dg", dtype, v.shape)
+    B, L, D = v.shape
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    fn = "causal_fftconv_bwd_f32" if dtype == torch.float32 else "causal_fftconv_bwd_bf16"
+    with torch.cuda.device(v.device):
+        st = getattr(load(), fn)(dr.data_ptr(), v.data_ptr(), g.data_ptr(), dv.data_ptr(), dg.data_ptr(), B, L, D,
+                                 ws_ptr, ws_bytes, _stream_ptr(stream))
+    if st != 0:
+        raise CausalConvError(st, fn)
+    return dv, dg
+
+
+def decode_workspace_bytes(dtype: torch.dtype, B: int, D: int, t: int) -> int:
+    return int(load().causal_conv_decode_workspace_bytes(_DT[dtype], B, D, t))
+
+
+def causal_conv_decode(v_cache: torch.Tensor, g_cache: torch.Tensor, t: int, out=None, workspace=None,
+                       stream=None) -> torch.Tensor:
+    """Output [B, D] of position t from [B, Lcap, D] caches:
+    r[b, d] = sum_{j<=t} v[b, j, d] g[b, t-j, d].  `workspace` (a uint8 CUDA
+    tensor of decode_workspace_bytes bytes) is allocated here when not given."""
+    dtype = v_cache.dtype
+    if dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"unsupported dtype {dtype}")
+    _check(v_cache, "v_cache", dtype)
+    _check(g_cache, "g_cache", dtype, v_cache.shape)
+    B, Lcap, D = v_cache.shape
+    if out is None:
+        out = torch.empty((B, D), dtype=dtype, device=v_cache.device)
+    nbytes = decode_workspace_bytes(dtype, B, D, t)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=v_cache.device)
+    fn = "causal_conv_decode_f32" if dtype == torch.float32 else "causal_conv_decode_bf16"
+    with torch.cuda.device(v_cache.device):
+        st = getattr(load(), fn)(v_cache.data_ptr(), g_cache.data_ptr(), out.data_ptr(), B, Lcap, D, int(t),
+                                 workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                 _stream_ptr(stream))
+    if st != 0:
+        raise CausalConvError(st, fn)
+    return out
 
 
 def causal_conv_from_host(v_host: torch.Tensor, g_host: torch.Tensor, r_host: torch.Tensor, v_dev: torch.Tensor,

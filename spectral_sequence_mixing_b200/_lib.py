@@ -22,6 +22,11 @@ SIGNATURES = {
     "causal_fftconv_f32": (ctypes.c_int, _CONV),
     "causal_fftconv_bf16": (ctypes.c_int, _CONV),
     "causal_ntt_conv_i32": (ctypes.c_int, _CONV),
+    "causal_fftconv_bwd_f32": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
+    "causal_fftconv_bwd_bf16": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
+    "causal_conv_decode_f32": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
+    "causal_conv_decode_bf16": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
+    "causal_conv_decode_workspace_bytes": (_SZ, [ctypes.c_int, _I64, _I64, _I64]),
     "causal_conv_from_host": (ctypes.c_int, [ctypes.c_int, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "causal_conv_workspace_bytes": (_SZ, [ctypes.c_int, _I64, _I64, _I64]),
     "causal_conv_max_len": (_I64, [ctypes.c_int]),

@@ -9,6 +9,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <initializer_list>
 #include <mutex>
 #include <vector>
 
@@ -16,6 +17,7 @@
 #include "fftconv_fused.cuh"
 #include "bigconv.cuh"
 #include "ntt.cuh"
+#include "decode.cuh"
 
 namespace ccv {
 
@@ -151,10 +153,11 @@ static int64_t max_len(int dtype) {
     }
 }
 
-static bool ranges_overlap(const void *a, const void *b, size_t bytes) {
+static bool ranges_overlap(const void *a, size_t a_bytes, const void *b, size_t b_bytes) {
     const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
-    return x < y + bytes && y < x + bytes;
+    return x < y + b_bytes && y < x + a_bytes;
 }
+static bool ranges_overlap(const void *a, const void *b, size_t bytes) { return ranges_overlap(a, bytes, b, bytes); }
 
 static int check_shape(int dtype, int64_t B, int64_t L, int64_t D, size_t *bytes) {
     const size_t es = dtype_size(dtype);
@@ -180,30 +183,44 @@ static int check_device_ptr(const void *p, int dev) {
     return CC_OK;
 }
 
-static int check_common(int dtype, const void *v, const void *g, const void *r, int64_t B, int64_t L, int64_t D,
-                        size_t ws_bytes, int *dev_out) {
+// Checks that need no CUDA call: null pointers, sizes, aliasing, workspace.
+static int check_host(int dtype, const void *v, const void *g, const void *r, int64_t B, int64_t L, int64_t D,
+                      size_t ws_bytes) {
     if (!v || !g || !r) return CC_ERR_INVALID_ARG;
     size_t bytes = 0;
     int st = check_shape(dtype, B, L, D, &bytes);
     if (st != CC_OK) return st;
     if (ranges_overlap(r, v, bytes) || ranges_overlap(r, g, bytes)) return CC_ERR_ALIAS;
     if (ws_bytes < causal_conv_workspace_bytes(dtype, B, L, D)) return CC_ERR_WORKSPACE;
+    return CC_OK;
+}
+
+// Every pointer is device memory of the current device (cudaPointerGetAttributes).
+static int check_device(std::initializer_list<const void *> ptrs, int *dev_out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
         return CC_ERR_CUDA;
     }
-    if ((st = check_device_ptr(v, dev)) != CC_OK) return st;
-    if ((st = check_device_ptr(g, dev)) != CC_OK) return st;
-    if ((st = check_device_ptr(r, dev)) != CC_OK) return st;
+    for (const void *p : ptrs) {
+        const int st = check_device_ptr(p, dev);
+        if (st != CC_OK) return st;
+    }
     *dev_out = dev;
     return CC_OK;
+}
+
+static int check_common(int dtype, const void *v, const void *g, const void *r, int64_t B, int64_t L, int64_t D,
+                        size_t ws_bytes, int *dev_out) {
+    const int st = check_host(dtype, v, g, r, B, L, D, ws_bytes);
+    if (st != CC_OK) return st;
+    return check_device({v, g, r}, dev_out);
 }
 
 // ------------------------------------------------------------------ launch
 template <class Cfg, int MINB, typename IO>
 static int launch_fused(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, const float2 *tw,
-                        cudaStream_t s, int dev) {
+                        cudaStream_t s, int dev, int rev) {
     const int64_t groups = (D + Cfg::ROWS - 1) / Cfg::ROWS;
     const int64_t tiles = B * groups;
     if (tiles > INT32_MAX) return CC_ERR_UNSUPPORTED;
@@ -218,13 +235,13 @@ static int launch_fused(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, i
     // whole-chunk async copies need full, aligned channel groups
     const bool vec = (D % Cfg::ROWS) == 0 && ((uintptr_t)v % Cfg::CHUNK) == 0 && ((uintptr_t)g % Cfg::CHUNK) == 0;
     kern<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(v, g, r, (int)L, (int)D, (int)groups, (int)tiles,
-                                                              vec ? 1 : 0, tw);
+                                                              vec ? 1 : 0, rev, tw);
     return cudaGetLastError() == cudaSuccess ? CC_OK : CC_ERR_CUDA;
 }
 
 template <class Cfg, int MINB, typename IO>
 static int launch_big(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, const float2 *tw,
-                      cudaStream_t s) {
+                      cudaStream_t s, int rev) {
     const int64_t rows = B * D;
     if (rows * Cfg::CL > INT32_MAX) return CC_ERR_UNSUPPORTED;
     auto kern = bigconv_kernel<Cfg::R0, Cfg::RA, Cfg::RB, Cfg::RC, Cfg::CL, Cfg::T, MINB, IO>;
@@ -240,7 +257,7 @@ static int launch_big(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, v, g, r, (int)L, (int)D, tw);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, v, g, r, (int)L, (int)D, rev, tw);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return CC_ERR_CUDA;
@@ -250,25 +267,73 @@ static int launch_big(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int
 
 template <typename IO>
 static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, cudaStream_t s,
-                            int dev) {
+                            int dev, int rev = 0) {
     void *tw = nullptr;
     if (L <= CfgS<IO>::LMAX) {
         if (cudaGetSymbolAddress(&tw, g_tw_s) != cudaSuccess) return CC_ERR_CUDA;
-        return launch_fused<CfgS<IO>, kMinbS>(v, g, r, B, L, D, (const float2 *)tw, s, dev);
+        return launch_fused<CfgS<IO>, kMinbS>(v, g, r, B, L, D, (const float2 *)tw, s, dev, rev);
     }
     if (L <= CfgM<IO>::LMAX) {
         if (cudaGetSymbolAddress(&tw, g_tw_m) != cudaSuccess) return CC_ERR_CUDA;
-        return launch_fused<CfgM<IO>, kMinbM>(v, g, r, B, L, D, (const float2 *)tw, s, dev);
+        return launch_fused<CfgM<IO>, kMinbM>(v, g, r, B, L, D, (const float2 *)tw, s, dev, rev);
     }
     if (L <= BigL<IO>::LMAX) {
         if (cudaGetSymbolAddress(&tw, g_tw_bl) != cudaSuccess) return CC_ERR_CUDA;
-        return launch_big<BigL<IO>, kMinbBigL>(v, g, r, B, L, D, (const float2 *)tw, s);
+        return launch_big<BigL<IO>, kMinbBigL>(v, g, r, B, L, D, (const float2 *)tw, s, rev);
     }
     if (L <= BigX<IO>::LMAX) {
         if (cudaGetSymbolAddress(&tw, g_tw_bx) != cudaSuccess) return CC_ERR_CUDA;
-        return launch_big<BigX<IO>, kMinbBigX>(v, g, r, B, L, D, (const float2 *)tw, s);
+        return launch_big<BigX<IO>, kMinbBigX>(v, g, r, B, L, D, (const float2 *)tw, s, rev);
     }
     return CC_ERR_UNSUPPORTED;
+}
+
+// Backward: dv = rev(conv(rev(dr), g)), dg = rev(conv(rev(dr), v)).
+template <typename IO>
+static int fftconv_bwd(const IO *dr, const IO *v, const IO *g, IO *dv, IO *dg, int64_t B, int64_t L, int64_t D,
+                       cudaStream_t s, int dev) {
+    int st = fftconv_dispatch<IO>(dr, g, dv, B, L, D, s, dev, 3);
+    if (st != CC_OK) return st;
+    return fftconv_dispatch<IO>(dr, v, dg, B, L, D, s, dev, 3);
+}
+
+static int check_bwd(int dtype, const void *dr, const void *v, const void *g, const void *dv, const void *dg,
+                     int64_t B, int64_t L, int64_t D, size_t ws_bytes, int *dev) {
+    if (!dv || !dg) return CC_ERR_INVALID_ARG;
+    int st = check_host(dtype, dr, g, dv, B, L, D, ws_bytes);
+    if (st != CC_OK) return st;
+    if ((st = check_host(dtype, dr, v, dg, B, L, D, ws_bytes)) != CC_OK) return st;
+    const size_t bytes = (size_t)(B * L * D) * dtype_size(dtype);
+    if (ranges_overlap(dv, dg, bytes) || ranges_overlap(dv, v, bytes) || ranges_overlap(dg, g, bytes)) return CC_ERR_ALIAS;
+    return check_device({dr, v, g, dv, dg}, dev);
+}
+
+// ---------------------------------------------------------------- decode
+static int check_decode(int dtype, const void *v, const void *g, const void *r, int64_t B, int64_t Lcap, int64_t D,
+                        int64_t t, const void *ws, size_t ws_bytes) {
+    const size_t es = dtype_size(dtype);
+    if (es == 0 || !v || !g || !r) return CC_ERR_INVALID_ARG;
+    if (B < 1 || Lcap < 1 || D < 1 || t < 0 || t >= Lcap) return CC_ERR_INVALID_ARG;
+    if (B > 65535 || Lcap > INT32_MAX || D > INT32_MAX) return CC_ERR_INVALID_ARG;
+    const int64_t lim = INT64_MAX / (int64_t)es;
+    if (Lcap > lim / D || B > lim / (Lcap * D)) return CC_ERR_INVALID_ARG;
+    if (dtype == CC_DTYPE_I32) return CC_ERR_UNSUPPORTED;
+    const size_t cache_bytes = (size_t)(B * Lcap * D) * es, out_bytes = (size_t)(B * D) * es;
+    if (ranges_overlap(r, out_bytes, v, cache_bytes) || ranges_overlap(r, out_bytes, g, cache_bytes))
+        return CC_ERR_ALIAS;
+    const size_t need = (size_t)decode_splits(B, D, t) * (size_t)(B * D) * sizeof(double);
+    if (!ws || ws_bytes < need) return CC_ERR_WORKSPACE;
+    return CC_OK;
+}
+
+template <typename IO>
+static int decode_entry(int dtype, const IO *v, const IO *g, IO *r, int64_t B, int64_t Lcap, int64_t D, int64_t t,
+                        void *workspace, size_t workspace_bytes, void *stream) {
+    int st = check_decode(dtype, v, g, r, B, Lcap, D, t, workspace, workspace_bytes);
+    if (st != CC_OK) return st;
+    int dev;
+    if ((st = check_device({v, g, r, workspace}, &dev)) != CC_OK) return st;
+    return decode_launch<IO>(v, g, r, B, Lcap, D, t, (double *)workspace, (cudaStream_t)stream);
 }
 
 }  // namespace ccv
@@ -328,6 +393,46 @@ int causal_ntt_conv_i32(const int32_t *v, const int32_t *g, int32_t *r, int64_t 
     if (st != CC_OK) return st;
     if (ensure_init(dev) != cudaSuccess) return CC_ERR_CUDA;
     return ntt_dispatch(v, g, r, B, L, D, (cudaStream_t)stream);
+}
+
+int causal_fftconv_bwd_f32(const float *dr, const float *v, const float *g, float *dv, float *dg, int64_t B,
+                           int64_t L, int64_t D, void *workspace, size_t workspace_bytes, void *stream) {
+    (void)workspace;
+    int dev;
+    int st = check_bwd(CC_DTYPE_F32, dr, v, g, dv, dg, B, L, D, workspace_bytes, &dev);
+    if (st != CC_OK) return st;
+    if (ensure_init(dev) != cudaSuccess) return CC_ERR_CUDA;
+    return fftconv_bwd<float>(dr, v, g, dv, dg, B, L, D, (cudaStream_t)stream, dev);
+}
+
+int causal_fftconv_bwd_bf16(const uint16_t *dr, const uint16_t *v, const uint16_t *g, uint16_t *dv, uint16_t *dg,
+                            int64_t B, int64_t L, int64_t D, void *workspace, size_t workspace_bytes, void *stream) {
+    (void)workspace;
+    int dev;
+    int st = check_bwd(CC_DTYPE_BF16, dr, v, g, dv, dg, B, L, D, workspace_bytes, &dev);
+    if (st != CC_OK) return st;
+    if (ensure_init(dev) != cudaSuccess) return CC_ERR_CUDA;
+    typedef __nv_bfloat16 bf;
+    return fftconv_bwd<bf>((const bf *)dr, (const bf *)v, (const bf *)g, (bf *)dv, (bf *)dg, B, L, D,
+                           (cudaStream_t)stream, dev);
+}
+
+size_t causal_conv_decode_workspace_bytes(int dtype, int64_t B, int64_t D, int64_t t) {
+    if (dtype_size(dtype) == 0 || B < 1 || D < 1 || t < 0 || B > 65535 || D > INT32_MAX || t >= INT32_MAX)
+        return (size_t)-1;
+    return (size_t)decode_splits(B, D, t) * (size_t)(B * D) * sizeof(double);
+}
+
+int causal_conv_decode_f32(const float *v, const float *g, float *r, int64_t B, int64_t Lcap, int64_t D, int64_t t,
+                           void *workspace, size_t workspace_bytes, void *stream) {
+    return decode_entry<float>(CC_DTYPE_F32, v, g, r, B, Lcap, D, t, workspace, workspace_bytes, stream);
+}
+
+int causal_conv_decode_bf16(const uint16_t *v, const uint16_t *g, uint16_t *r, int64_t B, int64_t Lcap, int64_t D,
+                            int64_t t, void *workspace, size_t workspace_bytes, void *stream) {
+    typedef __nv_bfloat16 bf;
+    return decode_entry<bf>(CC_DTYPE_BF16, (const bf *)v, (const bf *)g, (bf *)r, B, Lcap, D, t, workspace,
+                            workspace_bytes, stream);
 }
 
 int causal_conv_from_host(int dtype, const void *v_host, const void *g_host, void *r_host, void *v_dev, void *g_dev,

@@ -162,7 +162,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // plain loads (2-byte elements) are used.
 template <class C, typename IO>
 __device__ __forceinline__ void stage_tile(const IO *__restrict__ v, const IO *__restrict__ g, IO *sv, IO *sg,
-                                           int64_t boff, int d0, int L, int D, bool vec) {
+                                           int64_t boff, int d0, int L, int D, bool vec, bool rev_a) {
     constexpr int ROWS = C::ROWS;
     const int tid = threadIdx.x;
     const IO *vb = v + boff + d0;
@@ -172,16 +172,17 @@ __device__ __forceinline__ void stage_tile(const IO *__restrict__ v, const IO *_
         for (int e = tid; e < L * C::NCHUNK; e += C::THREADS) {
             const int t = e / C::NCHUNK, q = e - t * C::NCHUNK;
             const int64_t o = (int64_t)t * D + q * EPC;
+            const int64_t ov = (int64_t)(rev_a ? L - 1 - t : t) * D + q * EPC;
             IO *dv = sv + t * ROWS + q * EPC;
             IO *dg = sg + t * ROWS + q * EPC;
             if (C::CHUNK == 16) {
-                cp_async16(dv, vb + o);
+                cp_async16(dv, vb + ov);
                 cp_async16(dg, gb + o);
             } else if (C::CHUNK == 8) {
-                cp_async8(dv, vb + o);
+                cp_async8(dv, vb + ov);
                 cp_async8(dg, gb + o);
             } else {
-                cp_async4(dv, vb + o);
+                cp_async4(dv, vb + ov);
                 cp_async4(dg, gb + o);
             }
         }
@@ -191,11 +192,12 @@ __device__ __forceinline__ void stage_tile(const IO *__restrict__ v, const IO *_
             const int t = e / ROWS, c = e - t * ROWS;
             if (c < nc) {
                 const int64_t o = (int64_t)t * D + c;
+                const int64_t ov = (int64_t)(rev_a ? L - 1 - t : t) * D + c;
                 if (sizeof(IO) == 4) {
-                    cp_async4(sv + e, vb + o);
+                    cp_async4(sv + e, vb + ov);
                     cp_async4(sg + e, gb + o);
                 } else {
-                    sv[e] = IO_t<IO>::ld(vb + o);
+                    sv[e] = IO_t<IO>::ld(vb + ov);
                     sg[e] = IO_t<IO>::ld(gb + o);
                 }
             }
@@ -216,9 +218,11 @@ __device__ __forceinline__ void bar_sync(int id, int count) {
 template <int N2, int ROWS, int MINB, typename IO>
 __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
     fftconv_fused_kernel(const IO *__restrict__ v, const IO *__restrict__ g, IO *__restrict__ r, int L, int D,
-                         int groups_per_batch, int num_tiles, int vec_ok, const float2 *__restrict__ tw) {
+                         int groups_per_batch, int num_tiles, int vec_ok, int rev, const float2 *__restrict__ tw) {
+    // rev bit 0: read v reversed in time (v_t -> v_{L-1-t}); bit 1: write r reversed
     using C = FusedCfg<N2, ROWS, IO>;
     constexpr int N1 = C::N1, N = C::N, M2 = C::M2, H = C::H, MH = C::MH;
+    const bool rev_a = rev & 1, rev_out = (rev >> 1) & 1;
     constexpr int SC = C::SC, SF_N = C::SF_N, SI_M = C::SI_M, HEAD = C::HEAD, LMAX = C::LMAX;
     constexpr int THREADS = C::THREADS;
     extern __shared__ float4 smem_raw[];
@@ -247,7 +251,7 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
     if (tile >= num_tiles) return;
     {
         const int b = tile / groups_per_batch, d0 = (tile - b * groups_per_batch) * ROWS;
-        stage_tile<C, IO>(v, g, sv, sg, (int64_t)b * L * D, d0, L, D, vec_ok && d0 + ROWS <= D);
+        stage_tile<C, IO>(v, g, sv, sg, (int64_t)b * L * D, d0, L, D, vec_ok && d0 + ROWS <= D, rev_a);
     }
 
     for (; tile < num_tiles; tile += gridDim.x) {
@@ -324,7 +328,7 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
             const int nt = tile + gridDim.x;
             if (nt < num_tiles) {
                 const int nb = nt / groups_per_batch, nd0 = (nt - nb * groups_per_batch) * ROWS;
-                stage_tile<C, IO>(v, g, sv, sg, (int64_t)nb * L * D, nd0, L, D, vec_ok && nd0 + ROWS <= D);
+                stage_tile<C, IO>(v, g, sv, sg, (int64_t)nb * L * D, nd0, L, D, vec_ok && nd0 + ROWS <= D, rev_a);
             }
         }
 
@@ -433,8 +437,9 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
             const bool dok = d < D;
             const float sc = 1.f / (4.f * (float)N * alpha_row[c]);
             const int t0 = 2 * m2 + N2 * (H * s + (H / 2) * h);
-            IO *rp = r + boff + d + (int64_t)t0 * D;
-            const int64_t step = (int64_t)N2 * D;
+            const int64_t dir = rev_out ? -1 : 1;  // output time direction
+            IO *rp = r + boff + d + (int64_t)(rev_out ? L - 1 - t0 : t0) * D;
+            const int64_t step = dir * N2 * D;
 #pragma unroll
             for (int i = 0; i < H / 2; ++i) {
                 const float2 send = h ? out[i] : out[H / 2 + i];
@@ -447,7 +452,7 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
                     r1 = hres[c * 2 * HEAD + t + 1];
                 }
                 if (dok && t < L) IO_t<IO>::st(rp, r0);
-                if (dok && t + 1 < L) IO_t<IO>::st(rp + D, r1);
+                if (dok && t + 1 < L) IO_t<IO>::st(rp + dir * D, r1);
                 rp += step;
             }
         }

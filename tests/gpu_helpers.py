@@ -49,3 +49,11 @@ def float_violations(r_gpu, r_ref, den, tol, floor=0.0):
     with np.errstate(divide="ignore", invalid="ignore"):
         ratio = np.where(bound > 0, err / bound, np.where(err > 0, np.inf, 0.0))
     return int((err > bound).sum()), float(ratio.max() if ratio.size else 0.0)
+
+
+def run_gpu_bwd(dr, v, g, dtype: str):
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    dv, dg = ssm.causal_conv_bwd(to_dev(dr, dtype), to_dev(v, dtype), to_dev(g, dtype))
+    torch.cuda.synchronize()
+    return from_dev(dv, dtype), from_dev(dg, dtype)

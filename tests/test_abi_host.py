@@ -115,3 +115,42 @@ def test_from_host_rejects_null_host_pointers(lib):
     assert lib.causal_conv_from_host(0, None, B_, C, A, B_, C, 1, 16, 4, None, 0, None) == 1
     assert lib.causal_conv_from_host(9, A, B_, C, A + 0x1000000, B_ + 0x1000000, C + 0x1000000, 1, 16, 4, None, 0,
                                      None) == 1
+
+
+def test_bwd_host_side_argument_errors(lib):
+    f = lib.causal_fftconv_bwd_f32
+    D_, E_ = 0x40000000, 0x50000000
+    assert f(A, B_, C, None, E_, 1, 16, 4, None, 0, None) == 1        # null dv
+    assert f(A, B_, C, D_, None, 1, 16, 4, None, 0, None) == 1        # null dg
+    assert f(A, B_, C, D_, E_, 0, 16, 4, None, 0, None) == 1          # B < 1
+    assert f(A, B_, C, A + 8, E_, 1, 16, 4, None, 0, None) == 3       # dv overlaps dr
+    assert f(A, B_, C, D_, B_ + 8, 1, 16, 4, None, 0, None) == 3      # dg overlaps v
+    assert f(A, B_, C, D_, D_ + 8, 1, 16, 4, None, 0, None) == 3      # dv overlaps dg
+
+
+def test_decode_host_side_checks(lib):
+    f = lib.causal_conv_decode_f32
+    ws = lib.causal_conv_decode_workspace_bytes(0, 8, 768, 1023)
+    assert 0 < ws < 2 ** 32 and ws % (8 * 768 * 8) == 0
+    assert lib.causal_conv_decode_workspace_bytes(0, 8, 768, -1) == ctypes.c_size_t(-1).value
+    big = 1 << 30
+    W = 0x60000000
+    assert f(None, B_, C, 1, 16, 4, 3, W, big, None) == 1            # null cache
+    assert f(A, B_, C, 1, 16, 4, 16, W, big, None) == 1              # t >= Lcap
+    assert f(A, B_, C, 1, 16, 4, -1, W, big, None) == 1              # t < 0
+    assert f(A, B_, C, 70000, 16, 4, 3, W, big, None) == 1           # B > 65535
+    assert f(A, B_, A + 8, 1, 16, 4, 3, W, big, None) == 3           # output inside a cache
+    assert f(A, B_, C, 1, 16, 4, 3, None, 0, None) == 4              # workspace missing
+    assert f(A, B_, C, 1, 16, 4, 3, W, 8, None) == 4                 # workspace too small
+    assert lib.causal_conv_decode_bf16(A, B_, C, 1, 16, 4, 3, W, 8, None) == 4
+
+
+def test_decode_alias_is_range_exact(lib):
+    """An output just past the end of a cache is not an overlap; one inside is."""
+    f = lib.causal_conv_decode_f32
+    B, L, D = 1, 16, 4
+    cache = B * L * D * 4
+    W = 0x60000000
+    assert f(A, B_, A + cache, B, L, D, 3, W, 8, None) == 4      # passes the alias check, fails on workspace
+    assert f(A, B_, A + cache - 4, B, L, D, 3, W, 8, None) == 3  # last cache element overlaps
+    assert f(A, B_, A - B * D * 4, B, L, D, 3, W, 8, None) == 4  # output right before the cache

@@ -242,3 +242,87 @@ def test_rejects_host_pointer_on_device_entry():
     d2 = torch.zeros(1, 16, 4, device="cuda")
     assert lib.causal_fftconv_f32(h.data_ptr(), d.data_ptr(), d2.data_ptr(), 1, 16, 4, None, 0, None) == 6
     assert lib.causal_fftconv_f32(d.data_ptr(), d2.data_ptr(), h.data_ptr(), 1, 16, 4, None, 0, None) == 6
+
+
+# ---------------------------------------------------------------- backward
+from gpu_helpers import run_gpu_bwd  # noqa: E402
+
+BWD_SHAPES = [(1, 1, 1), (2, 33, 5), (3, 200, 19), (2, 1000, 37), (1, 1024, 8), (1, 2000, 3), (1, 4096, 2)]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", BWD_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_bwd_parity_full_oracle(shape, dtype):
+    """dv_j = sum_{t>=j} dr_t g_{t-j}, dg_k = sum_{t>=k} dr_t v_{t-k} (training gradients)."""
+    rng = np.random.Generator(np.random.PCG64(300 + sum(shape)))
+    dr, v, g = (rng.standard_normal(shape).astype(np.float32) for _ in range(3))
+    tol = F32_TOL
+    if dtype == "bf16":
+        dr, v, g = (workloads.bf16_round(x) for x in (dr, v, g))
+        tol = BF16_TOL
+    dv, dg = run_gpu_bwd(dr, v, g, dtype)
+    ref_dv, den_dv, ref_dg, den_dg = oracle.causal_conv_bwd(*(as_f32(x, dtype) for x in (dr, v, g)))
+    for name, got, ref, den in (("dv", dv, ref_dv, den_dv), ("dg", dg, ref_dg, den_dg)):
+        n_bad, worst = float_violations(as_f32(got, dtype) if dtype == "bf16" else got, ref, den, tol)
+        assert n_bad == 0, f"{name}: {n_bad} violations, worst ratio {worst:.3g}"
+
+
+@pytest.mark.parametrize("shape", [(1, 20000, 2), (8, 1024, 768)], ids=lambda s: "x".join(map(str, s)))
+def test_bwd_sampled_oracle(shape):
+    """Cluster path (L > 4096) and the small_f32 shape, on sampled outputs."""
+    B, L, D = shape
+    rng = np.random.Generator(np.random.PCG64(400 + L))
+    dr, v, g = (rng.standard_normal(shape).astype(np.float32) for _ in range(3))
+    dv, dg = run_gpu_bwd(dr, v, g, "f32")
+    pts = workloads.sample_points(B, L, D, 2048, seed=8)
+    ref_dv, den_dv, ref_dg, den_dg = oracle.causal_conv_bwd_points(dr, v, g, pts)
+    ix = (pts[:, 0], pts[:, 1], pts[:, 2])
+    for name, got, ref, den in (("dv", dv[ix], ref_dv, den_dv), ("dg", dg[ix], ref_dg, den_dg)):
+        n_bad, worst = float_violations(got, ref, den, F32_TOL)
+        assert n_bad == 0, f"{name}: {n_bad} violations, worst ratio {worst:.3g}"
+
+
+def test_bwd_consistent_with_forward_adjoint():
+    """<dr, r(v, g)> = <dv, v> = <dg, g> with the GPU forward and backward."""
+    import spectral_sequence_mixing_b200 as ssm
+    rng = np.random.Generator(np.random.PCG64(5))
+    shape = (2, 700, 16)
+    dr, v, g = (rng.standard_normal(shape).astype(np.float32) for _ in range(3))
+    r = run_gpu(v, g, "f32").astype(np.float64)
+    dv, dg = run_gpu_bwd(dr, v, g, "f32")
+    lhs = np.einsum("btd,btd->bd", dr.astype(np.float64), r)
+    for grad, x in ((dv, v), (dg, g)):
+        rhs = np.einsum("btd,btd->bd", grad.astype(np.float64), x.astype(np.float64))
+        assert np.allclose(lhs, rhs, rtol=1e-4, atol=1e-3)
+
+
+# ---------------------------------------------------------------- decode step
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("case", [(2, 64, 5, 0), (2, 64, 5, 1), (3, 300, 37, 63), (3, 300, 37, 64),
+                                  (1, 5000, 19, 4999), (8, 1024, 768, 1023), (8, 1024, 768, 500)],
+                         ids=lambda c: "x".join(map(str, c)))
+def test_decode_step_matches_oracle(case, dtype):
+    """One decode step equals the causal sum at position t, bit-identically
+    across calls (fixed-order fp64 reduction)."""
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    B, Lcap, D, t = case
+    rng = np.random.Generator(np.random.PCG64(sum(case)))
+    v = rng.standard_normal((B, Lcap, D)).astype(np.float32)
+    g = rng.standard_normal((B, Lcap, D)).astype(np.float32)
+    tol = F32_TOL
+    if dtype == "bf16":
+        v, g = workloads.bf16_round(v), workloads.bf16_round(g)
+        tol = BF16_TOL
+    tv, tg = to_dev(v, dtype), to_dev(g, dtype)
+    r1 = ssm.causal_conv_decode(tv, tg, t)
+    r2 = ssm.causal_conv_decode(tv, tg, t)
+    torch.cuda.synchronize()
+    assert torch.equal(r1.view(torch.int16) if dtype == "bf16" else r1, r2.view(torch.int16) if dtype == "bf16" else r2)
+    got = as_f32(from_dev(r1, dtype), dtype)
+    pts = np.array([(b, t, d) for b in range(B) for d in range(D)], np.int64)
+    ref, den = oracle.causal_conv_points(as_f32(v, dtype), as_f32(g, dtype), pts)
+    n_bad, worst = float_violations(got.reshape(-1), ref, den, tol)
+    assert n_bad == 0, f"{n_bad} violations, worst ratio {worst:.3g}"
+    if dtype == "f32":  # fp64 accumulation, one rounding to float at the end
+        assert np.all(np.abs(got.reshape(-1) - ref) <= 6.0e-8 * np.abs(ref) + 1e-12 * den)
