@@ -52,7 +52,8 @@ typedef enum {
     CC_ERR_ALIAS = 3,       /* r overlaps v or g                                */
     CC_ERR_WORKSPACE = 4,   /* workspace smaller than causal_conv_workspace_bytes */
     CC_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed      */
-    CC_ERR_NOT_DEVICE = 6   /* a pointer is not device memory of the current device */
+    CC_ERR_NOT_DEVICE = 6,  /* a pointer is not device memory of the current device */
+    CC_ERR_SCRATCH_LIMIT = 7 /* beyond the fixed scratch of causal_conv_decode_f32_noalloc */
 } cc_status;
 
 typedef enum {
@@ -159,6 +160,34 @@ CC_API int causal_conv_decode_f32(const float *v, const float *g, float *r, int6
 /* causal_conv_decode_bf16 -- as causal_conv_decode_f32 with bfloat16 caches and output. */
 CC_API int causal_conv_decode_bf16(const uint16_t *v, const uint16_t *g, uint16_t *r, int64_t B, int64_t Lcap,
                                    int64_t D, int64_t t, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * causal_conv_decode_f32_noalloc -- causal_conv_decode_f32 for callers that
+ * cannot allocate device memory: code that runs inside an engine which owns
+ * all device memory through its own pool and forbids allocations behind its
+ * back, or code on a path that must not pay the device-wide synchronisation
+ * cudaFree implies.  The pages have no counterpart; this is a library entry
+ * point, not part of the method.
+ *
+ * Arguments and result are those of causal_conv_decode_f32 without the
+ * workspace: the caller still passes the caches v, g and the output r.  The
+ * fp64 partial sums go to one static device buffer of 8 MiB inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  The first call on a device looks the buffer's address up (once,
+ * with that device current); make that first call before any stream capture.
+ * The function calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Limit: a problem whose partial sums need more than 8 MiB, i.e. for which
+ * causal_conv_decode_workspace_bytes(CC_DTYPE_F32, B, D, t) > 8388608 (the
+ * small_f32 shape B = 8, D = 768, t = 1023 needs 768 KiB), returns
+ * CC_ERR_SCRATCH_LIMIT before anything is enqueued.  Every call on a device
+ * shares the one buffer and leaves its partial sums there; nothing in it has
+ * to start at zero (each call writes every slot it reads), but calls whose
+ * work overlaps on the GPU (other streams, other host threads) race on the
+ * buffer: order them.
+ */
+CC_API int causal_conv_decode_f32_noalloc(const float *v, const float *g, float *r, int64_t B, int64_t Lcap,
+                                          int64_t D, int64_t t, void *stream);
 
 /* Workspace bytes causal_conv_decode_* needs for (B, D, t); (size_t)-1 if invalid. */
 CC_API size_t causal_conv_decode_workspace_bytes(int dtype, int64_t B, int64_t D, int64_t t);

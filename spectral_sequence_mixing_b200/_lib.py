@@ -11,6 +11,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libcausalconv.so")
 
 CC_OK, CC_ERR_INVALID_ARG, CC_ERR_UNSUPPORTED, CC_ERR_ALIAS, CC_ERR_WORKSPACE, CC_ERR_CUDA, CC_ERR_NOT_DEVICE = range(7)
+CC_ERR_SCRATCH_LIMIT = 7
 CC_DTYPE_F32, CC_DTYPE_BF16, CC_DTYPE_I32 = 0, 1, 2
 
 # name -> (restype, argtypes); every symbol include/causalconv.h declares.
@@ -27,6 +28,7 @@ SIGNATURES = {
     "causal_conv_decode_f32": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "causal_conv_decode_bf16": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "causal_conv_decode_workspace_bytes": (_SZ, [ctypes.c_int, _I64, _I64, _I64]),
+    "causal_conv_decode_f32_noalloc": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _I64, _P]),
     "causal_conv_from_host": (ctypes.c_int, [ctypes.c_int, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "causal_conv_workspace_bytes": (_SZ, [ctypes.c_int, _I64, _I64, _I64]),
     "causal_conv_max_len": (_I64, [ctypes.c_int]),

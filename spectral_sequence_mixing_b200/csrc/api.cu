@@ -336,6 +336,34 @@ static int decode_entry(int dtype, const IO *v, const IO *g, IO *r, int64_t B, i
     return decode_launch<IO>(v, g, r, B, Lcap, D, t, (double *)workspace, (cudaStream_t)stream);
 }
 
+// ------------------------------------------------- decode without allocation
+// Fixed scratch for causal_conv_decode_f32_noalloc: the fp64 partial sums of
+// the split reduction live here instead of in a caller workspace.  Every GPU
+// that loads this library holds these 8 MiB until the process exits.
+constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;
+static __device__ __align__(256) double g_noalloc_scratch[kNoAllocScratchBytes / sizeof(double)];
+
+// Device address of g_noalloc_scratch per device.  In host code the symbol
+// only names a host-side stand-in, so the address is looked up with the
+// device current on first use and cached.
+static std::mutex g_noalloc_mu;
+static double *g_noalloc_ptr[128];
+
+static int noalloc_scratch(int dev, double **out) {
+    if (dev < 0 || dev >= 128) return CC_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return CC_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = (double *)p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return CC_OK;
+}
+
 }  // namespace ccv
 
 using namespace ccv;
@@ -360,6 +388,7 @@ const char *causal_conv_strerror(int status) {
         case CC_ERR_WORKSPACE: return "workspace smaller than causal_conv_workspace_bytes()";
         case CC_ERR_CUDA: return "CUDA runtime error or kernel launch failure";
         case CC_ERR_NOT_DEVICE: return "pointer is not device memory of the current device";
+        case CC_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the fixed 8 MiB buffer of the no-allocation entry point";
         default: return "unknown status";
     }
 }
@@ -433,6 +462,25 @@ int causal_conv_decode_bf16(const uint16_t *v, const uint16_t *g, uint16_t *r, i
     typedef __nv_bfloat16 bf;
     return decode_entry<bf>(CC_DTYPE_BF16, (const bf *)v, (const bf *)g, (bf *)r, B, Lcap, D, t, workspace,
                             workspace_bytes, stream);
+}
+
+int causal_conv_decode_f32_noalloc(const float *v, const float *g, float *r, int64_t B, int64_t Lcap, int64_t D,
+                                   int64_t t, void *stream) {
+    // Same checks as causal_conv_decode_f32 with the library's own scratch
+    // standing in for the workspace; a problem whose partial sums exceed the
+    // fixed scratch is refused before anything is enqueued.
+    if (!v || !g || !r) return CC_ERR_INVALID_ARG;
+    if (B < 1 || D < 1 || t < 0 || B > 65535 || D > INT32_MAX || t >= INT32_MAX) return CC_ERR_INVALID_ARG;
+    const size_t need = (size_t)decode_splits(B, D, t) * (size_t)(B * D) * sizeof(double);
+    if (need > kNoAllocScratchBytes) return CC_ERR_SCRATCH_LIMIT;
+    // the fixed scratch stands in for the workspace argument (non-null, large enough)
+    int st = check_decode(CC_DTYPE_F32, v, g, r, B, Lcap, D, t, &need, kNoAllocScratchBytes);
+    if (st != CC_OK) return st;
+    int dev;
+    if ((st = check_device({v, g, r}, &dev)) != CC_OK) return st;
+    double *scratch = nullptr;
+    if ((st = noalloc_scratch(dev, &scratch)) != CC_OK) return st;
+    return decode_launch<float>(v, g, r, B, Lcap, D, t, scratch, (cudaStream_t)stream);
 }
 
 int causal_conv_from_host(int dtype, const void *v_host, const void *g_host, void *r_host, void *v_dev, void *g_dev,
