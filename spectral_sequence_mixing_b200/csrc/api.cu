@@ -64,14 +64,22 @@ static std::vector<float2> fused_twiddles() {
 
 template <class Cfg>
 static std::vector<float2> big_twiddles() {
+    // factor tables, see BigCfg
     constexpr int S = Cfg::S, SL = Cfg::SL, R0 = Cfg::R0, RA = Cfg::RA, RB = Cfg::RB, RC = Cfg::RC;
+    constexpr int Q0 = Cfg::Q0, QA = Cfg::QA, STA = Cfg::STA;
     std::vector<float2> t(Cfg::TW_SIZE);
-    for (int k0 = 0; k0 < R0; ++k0)
-        for (int n = 0; n < SL; ++n) t[Cfg::TW0 + k0 * SL + n] = omega((int64_t)n * (2 * k0 + 1), 2 * (int64_t)S);
-    for (int k = 0; k < RA; ++k)
-        for (int lo = 0; lo < RB * RC; ++lo) t[Cfg::TWA + k * (RB * RC) + lo] = omega((int64_t)lo * k, SL);
+    const int64_t S2 = 2 * (int64_t)S;
+    for (int k0 = 0; k0 < R0; ++k0) {
+        for (int nl = 0; nl < Q0; ++nl) t[Cfg::T0A + k0 * Q0 + nl] = omega((int64_t)nl * (2 * k0 + 1), S2);
+        for (int nh = 0; nh < SL / Q0; ++nh)
+            t[Cfg::T0B + k0 * (SL / Q0) + nh] = omega((int64_t)Q0 * nh * (2 * k0 + 1), S2);
+    }
+    for (int k = 0; k < RA; ++k) {
+        for (int ll = 0; ll < QA; ++ll) t[Cfg::TAA + k * QA + ll] = omega((int64_t)ll * k, SL);
+        for (int lh = 0; lh < STA / QA; ++lh) t[Cfg::TAB + k * (STA / QA) + lh] = omega((int64_t)QA * lh * k, SL);
+    }
     for (int k = 0; k < RB; ++k)
-        for (int lo = 0; lo < RC; ++lo) t[Cfg::TWB + k * RC + lo] = omega((int64_t)lo * k, RB * RC);
+        for (int lo = 0; lo < RC; ++lo) t[Cfg::TB + k * RC + lo] = omega((int64_t)lo * k, RB * RC);
     return t;
 }
 

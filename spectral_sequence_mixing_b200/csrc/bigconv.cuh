@@ -51,12 +51,22 @@ struct BigCfg {
     static constexpr int WORDS = SC + SC / 16;  // padded float2 words
     static constexpr int PER0 = COLS0 / T;  // pass-0 columns per thread
     static constexpr size_t SMEM_BYTES = (size_t)WORDS * 8 + (size_t)HEAD * 8 + (size_t)(T / 32 + 1) * 8;
-    // twiddle tables (float2): TW0[k0*SL + n] = theta^(n (2 k0 + 1)),
-    // TWA[k*(RB RC) + lo] = omega_SL^(lo k), TWB[k*RC + lo] = omega_(RB RC)^(lo k)
-    static constexpr int TW0 = 0;
-    static constexpr int TWA = S;
-    static constexpr int TWB = S + SL;
-    static constexpr int TW_SIZE = S + SL + RB * RC;
+    // Twiddle tables (float2), each factored into two small tables that stay
+    // in L1 (value = product of two correctly rounded unit numbers):
+    //   pass 0:  theta^(n (2 k0 + 1)), n = nh Q0 + nl
+    //            = T0A[k0][nl] * T0B[k0][nh],  T0A = theta^(nl (2k0+1)), T0B = theta^(Q0 nh (2k0+1))
+    //   pass A:  omega_SL^(lo k), lo = lh QA + ll
+    //            = TAa[k][ll] * TAb[k][lh]
+    //   pass B:  omega_(RB RC)^(lo k) = TB[k][lo]   (only when RC > 1)
+    static constexpr int STA = RB * RC;  // slot stride of pass A
+    static constexpr int Q0 = SL < 64 ? SL : 64;
+    static constexpr int QA = STA < 32 ? STA : 32;
+    static constexpr int T0A = 0;
+    static constexpr int T0B = T0A + R0 * Q0;
+    static constexpr int TAA = T0B + R0 * (SL / Q0);
+    static constexpr int TAB = TAA + RA * QA;
+    static constexpr int TB = TAB + RA * (STA / QA);
+    static constexpr int TW_SIZE = TB + RB * RC;
     static constexpr int LAST_R = RC > 1 ? RC : RB;
     static_assert(CL == 1 || CL == R0, "a cluster splits the most significant digit");
     static_assert(LAST_R == 16, "innermost radix must be 16 (conflict-free padded layout)");
@@ -66,39 +76,72 @@ struct BigCfg {
 
 __device__ __forceinline__ int bc_pad(int p) { return p + (p >> 4); }
 
+// Distributed shared memory: 32-bit shared-window addresses of the same
+// offset in another CTA of the cluster, and 8-byte loads / stores there.
+__device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ uint32_t cluster_map(uint32_t addr, int rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster(uint32_t addr, float2 v) {
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};\n" ::"r"(addr), "f"(v.x), "f"(v.y) : "memory");
+}
+__device__ __forceinline__ float2 ld_cluster(uint32_t addr) {
+    float2 v;
+    asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];\n" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
+    return v;
+}
+
 // One local forward (INV=false) or inverse (INV=true) pass over a digit of
-// radix R and slot stride ST inside sub-arrays of SL slots; W = twiddle table
-// omega_(R*ST)^(lo*k) laid out [k][lo] (nullptr when ST == 1).
-template <int R, int ST, int SL, int SC, int T, bool INV>
-__device__ __forceinline__ void bc_local_pass(float2 *xs, const float2 *__restrict__ W) {
+// radix R and slot stride ST inside sub-arrays of SL slots.  The twiddle
+// omega_(R ST)^(lo k) is Wa[k][lo % Q] * Wb[k][lo / Q] (Wb unused when
+// ST <= Q; no twiddle when ST == 1).  With ST a multiple of 16 (or 1 and
+// R == 16) the padded address of element j is pad(base) + j * PST, a
+// compile-time offset.
+template <int R, int ST, int Q, int SL, int SC, int T, bool INV>
+__device__ __forceinline__ void bc_local_pass(float2 *xs, const float2 *__restrict__ Wa,
+                                              const float2 *__restrict__ Wb) {
     constexpr int NDFT = SC / R;
     constexpr int LOG_R = ilog2(R);
+    constexpr int PST = ST == 1 ? 1 : ST + ST / 16;
+    static_assert(ST == 1 ? R == 16 : ST % 16 == 0, "linear padded addressing");
 #pragma unroll 1
     for (int q = threadIdx.x; q < NDFT; q += T) {
         const int sub = q / (SL / R), w = q - sub * (SL / R);
         const int hi = w / ST, lo = w - hi * ST;
-        const int base = sub * SL + hi * R * ST + lo;
+        float2 *xp = xs + bc_pad(sub * SL + hi * R * ST + lo);
+        const float2 *wa = Wa + (lo % Q);
+        const float2 *wb = Wb + (lo / Q);
         float2 x[R];
         if (!INV) {
 #pragma unroll
-            for (int j = 0; j < R; ++j) x[bitrev(j, LOG_R)] = xs[bc_pad(base + j * ST)];
+            for (int j = 0; j < R; ++j) x[bitrev(j, LOG_R)] = xp[j * PST];
             fft_dit<R, false>(x);
             if (ST > 1) {
 #pragma unroll
-                for (int k = 1; k < R; ++k) x[k] = cmul(x[k], __ldg(W + k * ST + lo));
+                for (int k = 1; k < R; ++k) {
+                    float2 w2 = __ldg(wa + k * Q);
+                    if (ST > Q) w2 = cmul(w2, __ldg(wb + k * (ST / Q)));
+                    x[k] = cmul(x[k], w2);
+                }
             }
 #pragma unroll
-            for (int k = 0; k < R; ++k) xs[bc_pad(base + k * ST)] = x[k];
+            for (int k = 0; k < R; ++k) xp[k * PST] = x[k];
         } else {
 #pragma unroll
             for (int k = 0; k < R; ++k) {
-                float2 y = xs[bc_pad(base + k * ST)];
-                if (ST > 1 && k > 0) y = cmul_conj(y, __ldg(W + k * ST + lo));
+                float2 y = xp[k * PST];
+                if (ST > 1 && k > 0) {
+                    float2 w2 = __ldg(wa + k * Q);
+                    if (ST > Q) w2 = cmul(w2, __ldg(wb + k * (ST / Q)));
+                    y = cmul_conj(y, w2);
+                }
                 x[bitrev(k, LOG_R)] = y;
             }
             fft_dit<R, true>(x);
 #pragma unroll
-            for (int j = 0; j < R; ++j) xs[bc_pad(base + j * ST)] = x[j];
+            for (int j = 0; j < R; ++j) xp[j * PST] = x[j];
         }
     }
 }
@@ -128,13 +171,35 @@ __global__ void __launch_bounds__(T, MINB)
             __syncthreads();
     };
     if constexpr (CL > 1) cluster_sync();  // all CTAs of the cluster resident before any remote store
-    // generic pointer to slot s of the row (any CTA of the cluster)
-    auto slot_ptr = [&](int s) -> float2 * {
-        const int k0 = s / SL;
+    // Slot (k0, n) of the row lives in CTA k0 / K0C at local offset
+    // (k0 % K0C) SL + n; with a cluster it is reached through the shared
+    // window address of that CTA (same layout in every CTA).
+    const uint32_t xs_addr = smem_addr(xs);
+    auto slot_addr = [&](int k0, int n) -> uint32_t {
         const int owner = k0 / C::K0C;
-        float2 *p = xs + bc_pad((k0 - owner * C::K0C) * SL + (s - k0 * SL));
-        if constexpr (CL > 1) return cg::this_cluster().map_shared_rank(p, owner);
-        return p;
+        const uint32_t local = xs_addr + 8u * (uint32_t)bc_pad((k0 - owner * C::K0C) * SL + n);
+        if constexpr (CL > 1) return cluster_map(local, owner);
+        return local;
+    };
+    auto slot_st = [&](uint32_t a, float2 val) {
+        if constexpr (CL > 1)
+            st_cluster(a, val);
+        else
+            asm volatile("st.shared.v2.f32 [%0], {%1, %2};\n" ::"r"(a), "f"(val.x), "f"(val.y) : "memory");
+    };
+    auto slot_ld = [&](uint32_t a) -> float2 {
+        float2 val;
+        if constexpr (CL > 1)
+            val = ld_cluster(a);
+        else
+            asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];\n" : "=f"(val.x), "=f"(val.y) : "r"(a) : "memory");
+        return val;
+    };
+    // theta^(n (2 k0 + 1)) from the two factor tables
+    auto tw0 = [&](int k0, int n) -> float2 {
+        const float2 a = __ldg(tw + C::T0A + k0 * C::Q0 + (n % C::Q0));
+        if constexpr (SL > C::Q0) return cmul(a, __ldg(tw + C::T0B + k0 * (SL / C::Q0) + (n / C::Q0)));
+        return a;
     };
 
     // ---- load the padded input of this CTA's pass-0 columns; stream norms for balancing
@@ -198,22 +263,19 @@ __global__ void __launch_bounds__(T, MINB)
         }
         fft_dit<R0, false, true>(x);
 #pragma unroll
-        for (int k0 = 0; k0 < R0; ++k0) {
-            const float2 y = cmul(x[k0], __ldg(tw + C::TW0 + k0 * SL + n));
-            *slot_ptr(k0 * SL + n) = y;
-        }
+        for (int k0 = 0; k0 < R0; ++k0) slot_st(slot_addr(k0, n), cmul(x[k0], tw0(k0, n)));
     }
     cluster_sync();
 
     // ---- forward local passes
-    bc_local_pass<RA, RB * RC, SL, SC, T, false>(xs, tw + C::TWA);
+    bc_local_pass<RA, C::STA, C::QA, SL, SC, T, false>(xs, tw + C::TAA, tw + C::TAB);
     __syncthreads();
     if constexpr (RC > 1) {
-        bc_local_pass<RB, RC, SL, SC, T, false>(xs, tw + C::TWB);
+        bc_local_pass<RB, RC, RC, SL, SC, T, false>(xs, tw + C::TB, tw + C::TB);
         __syncthreads();
-        bc_local_pass<RC, 1, SL, SC, T, false>(xs, nullptr);
+        bc_local_pass<RC, 1, 1, SL, SC, T, false>(xs, tw, tw);
     } else {
-        bc_local_pass<RB, 1, SL, SC, T, false>(xs, nullptr);
+        bc_local_pass<RB, 1, 1, SL, SC, T, false>(xs, tw, tw);
     }
     cluster_sync();
 
@@ -226,7 +288,8 @@ __global__ void __launch_bounds__(T, MINB)
             const int o = tid + i * T;               // own offset
             const int s = rank * SC + o;             // global slot (k0-major within the cluster)
             const float2 zk = xs[bc_pad(o)];
-            const float2 zm = *slot_ptr(S - 1 - s);
+            const int sm = S - 1 - s;
+            const float2 zm = slot_ld(slot_addr(sm / SL, sm % SL));
             xv[i] = spectral_product(zk, zm);
         }
         cluster_sync();  // every mirror read done before any slot is overwritten
@@ -237,14 +300,14 @@ __global__ void __launch_bounds__(T, MINB)
 
     // ---- inverse local passes
     if constexpr (RC > 1) {
-        bc_local_pass<RC, 1, SL, SC, T, true>(xs, nullptr);
+        bc_local_pass<RC, 1, 1, SL, SC, T, true>(xs, tw, tw);
         __syncthreads();
-        bc_local_pass<RB, RC, SL, SC, T, true>(xs, tw + C::TWB);
+        bc_local_pass<RB, RC, RC, SL, SC, T, true>(xs, tw + C::TB, tw + C::TB);
     } else {
-        bc_local_pass<RB, 1, SL, SC, T, true>(xs, nullptr);
+        bc_local_pass<RB, 1, 1, SL, SC, T, true>(xs, tw, tw);
     }
     __syncthreads();
-    bc_local_pass<RA, RB * RC, SL, SC, T, true>(xs, tw + C::TWA);
+    bc_local_pass<RA, C::STA, C::QA, SL, SC, T, true>(xs, tw + C::TAA, tw + C::TAB);
     cluster_sync();
 
     // ---- inverse pass 0: twiddle, inverse R0-point DFT (outputs n0 < R0/2), untwist, store t < L
@@ -256,8 +319,7 @@ __global__ void __launch_bounds__(T, MINB)
             float2 x[R0];
 #pragma unroll
             for (int k0 = 0; k0 < R0; ++k0) {
-                const float2 y = *slot_ptr(k0 * SL + n);
-                x[bitrev(k0, LOG_R0)] = cmul_conj(y, __ldg(tw + C::TW0 + k0 * SL + n));
+                x[bitrev(k0, LOG_R0)] = cmul_conj(slot_ld(slot_addr(k0, n)), tw0(k0, n));
             }
             fft_dit<R0, true, false, true>(x);
 #pragma unroll
