@@ -228,6 +228,21 @@ CC_API const char *causal_conv_strerror(int status);
  */
 CC_API int causal_ntt_params(int64_t N, uint32_t out[6]);
 
+/*
+ * causal_conv_fault_flags -- the library's per-device fault word.  The pages
+ * have no counterpart: it reports waits inside the kernels that ran out of
+ * time.  Every wait in the kernels (on an asynchronous copy, an mbarrier) is
+ * bounded to about two seconds; a wait that runs out sets a bit here and its
+ * kernel returns early, leaving its outputs incomplete, instead of hanging the
+ * device.  Bit 0: a TMA staging copy did not complete.
+ *   device  CUDA device ordinal;
+ *   flags   host pointer, receives the word;
+ *   clear   non-zero: reset the word to 0 after reading it.
+ * Synchronises the device (the word is read after all queued work ends).
+ * Returns CC_OK, CC_ERR_INVALID_ARG (NULL flags, bad device) or CC_ERR_CUDA.
+ */
+CC_API int causal_conv_fault_flags(int device, unsigned int *flags, int clear);
+
 #ifdef __cplusplus
 }
 #endif

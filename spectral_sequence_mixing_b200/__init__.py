@@ -23,7 +23,7 @@ from ._lib import (CC_DTYPE_BF16, CC_DTYPE_F32, CC_DTYPE_I32, CausalConvError, l
 __all__ = [
     "causal_fftconv_f32", "causal_fftconv_bf16", "causal_ntt_conv_i32", "causal_conv", "causal_conv_bwd",
     "causal_conv_decode", "decode_workspace_bytes",
-    "causal_conv_from_host", "workspace_bytes", "max_len", "ntt_params", "strerror",
+    "causal_conv_from_host", "workspace_bytes", "max_len", "ntt_params", "strerror", "fault_flags",
     "CausalConvError", "CC_DTYPE_F32", "CC_DTYPE_BF16", "CC_DTYPE_I32",
 ]
 
@@ -194,3 +194,14 @@ def ntt_params(N: int) -> dict:
     if st != 0:
         raise CausalConvError(st, "causal_ntt_params")
     return dict(zip(("p", "omega", "omega_inv", "n_inv", "p_inv_mod_2_32", "r2_mod_p"), list(out)))
+
+
+def fault_flags(device: int | None = None, clear: bool = False) -> int:
+    """The per-device word of kernel waits that ran out of time (0 = none);
+    synchronises the device."""
+    dev = torch.cuda.current_device() if device is None else int(device)
+    out = ctypes.c_uint(0)
+    st = load().causal_conv_fault_flags(dev, ctypes.byref(out), 1 if clear else 0)
+    if st != 0:
+        raise CausalConvError(st, "causal_conv_fault_flags")
+    return int(out.value)

@@ -34,6 +34,7 @@ SIGNATURES = {
     "causal_conv_max_len": (_I64, [ctypes.c_int]),
     "causal_conv_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "causal_ntt_params": (ctypes.c_int, [_I64, ctypes.POINTER(ctypes.c_uint32)]),
+    "causal_conv_fault_flags": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_uint), ctypes.c_int]),
 }
 
 _lib = None

@@ -3,7 +3,9 @@
 // Host side: argument checks, one-time per-device constant/twiddle setup,
 // and dispatch to the sm_100a kernels.  The library allocates no device
 // memory: its tables are static __device__ arrays filled on first use.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 #include <math.h>
 #include <stdint.h>
 #include <string.h>
@@ -225,6 +227,43 @@ static int check_common(int dtype, const void *v, const void *g, const void *r, 
     return check_device({v, g, r}, dev_out);
 }
 
+// ------------------------------------------------------------------ tensor maps
+// cuTensorMapEncodeTiled from the driver, looked up once (no link against libcuda).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+// 3-D map over a channel-last [B, L, D] tensor (dims innermost first: D, L, B)
+// with boxes of [box_t][box_d]; elements outside the tensor read as zero.
+// False when the layout cannot be described (strides or base not 16-byte aligned).
+template <typename IO>
+static bool encode_btd_map(CUtensorMap *m, const IO *base, int64_t B, int64_t L, int64_t D, int box_d, int box_t) {
+    const size_t es = sizeof(IO);
+    if (((uintptr_t)base & 15) != 0 || (D * (int64_t)es) % 16 != 0) return false;
+    if (D > (int64_t)UINT32_MAX || L > (int64_t)UINT32_MAX || B > (int64_t)UINT32_MAX) return false;
+    if ((int64_t)es * D * L >= ((int64_t)1 << 40)) return false;
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)L, (cuuint64_t)B};
+    const cuuint64_t strides[2] = {(cuuint64_t)(D * es), (cuuint64_t)(D * L * es)};
+    const cuuint32_t box[3] = {(cuuint32_t)box_d, (cuuint32_t)box_t, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapDataType dt = sizeof(IO) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    return enc(m, dt, 3, const_cast<IO *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ launch
 template <class Cfg, int MINB, typename IO>
 static int launch_fused(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, const float2 *tw,
@@ -242,8 +281,15 @@ static int launch_fused(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, i
     const int64_t grid = std::min<int64_t>(tiles, (int64_t)per_sm * g_num_sms[dev]);
     // whole-chunk async copies need full, aligned channel groups
     const bool vec = (D % Cfg::ROWS) == 0 && ((uintptr_t)v % Cfg::CHUNK) == 0 && ((uintptr_t)g % Cfg::CHUNK) == 0;
+    // TMA boxes when a tile row is whole 16-byte units and v is read forward in time
+    CUtensorMap tmv, tmg;
+    memset(&tmv, 0, sizeof(tmv));
+    memset(&tmg, 0, sizeof(tmg));
+    const bool tma = Cfg::TMA_OK && (rev & 1) == 0 &&
+                     encode_btd_map<IO>(&tmv, v, B, L, D, Cfg::ROWS, Cfg::BOXT) &&
+                     encode_btd_map<IO>(&tmg, g, B, L, D, Cfg::ROWS, Cfg::BOXT);
     kern<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(v, g, r, (int)L, (int)D, (int)groups, (int)tiles,
-                                                              vec ? 1 : 0, rev, tw);
+                                                              vec ? 1 : 0, rev, tw, tmv, tmg, tma ? 1 : 0);
     return cudaGetLastError() == cudaSuccess ? CC_OK : CC_ERR_CUDA;
 }
 
@@ -538,6 +584,32 @@ int causal_ntt_params(int64_t N, uint32_t out[6]) {
     out[3] = p.ninv;
     out[4] = p.pinv;
     out[5] = p.r2;
+    return CC_OK;
+}
+
+int causal_conv_fault_flags(int device, unsigned int *flags, int clear) {
+    if (!flags) return CC_ERR_INVALID_ARG;
+    int n = 0;
+    if (cudaGetDeviceCount(&n) != cudaSuccess || device < 0 || device >= n) {
+        cudaGetLastError();
+        return CC_ERR_INVALID_ARG;
+    }
+    int prev = 0;
+    if (cudaGetDevice(&prev) != cudaSuccess || cudaSetDevice(device) != cudaSuccess) {
+        cudaGetLastError();
+        return CC_ERR_CUDA;
+    }
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(flags, g_cc_fault, sizeof(unsigned int));
+    if (e == cudaSuccess && clear) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_cc_fault, &zero, sizeof(zero));
+    }
+    cudaSetDevice(prev);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return CC_ERR_CUDA;
+    }
     return CC_OK;
 }
 

@@ -40,13 +40,20 @@
 // kHeadT0 inputs.
 //
 // Pipeline: each CTA loops over tiles; the next tile's v and g are copied
-// into a staging buffer with cp.async while the current tile runs F3 and I3.
+// into a staging buffer while the current tile runs F3 and I3.  The copy is a
+// handful of TMA boxes issued by one thread (completion counted on an
+// mbarrier; the copy engine zero-fills t >= L and d >= D) whenever a tile row
+// is a multiple of 16 bytes and the tensors allow a tensor map; otherwise the
+// threads issue cp.async pieces.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "fft_reg.cuh"
+#include "tma.cuh"
 
 namespace ccv {
 
@@ -86,18 +93,30 @@ struct FusedCfg {
     // half-warp is conflict-free when its 16 lanes hit distinct (word mod 16):
     // SF_N = 1 (mod 16) serves the F1 stores / F3 loads, SI_M = 2 (mod 16) and
     // SC = 16/ROWS (mod 16) serve the F3 stores / I3 loads.
+    // With ROWS = 2 a half-warp of I3 also spans two m2 rows, which then
+    // need SI_M = 4 (mod 16).
     static constexpr int SF_N = N1 + 1;
-    static constexpr int SI_M = N1 + 2;
+    static constexpr int SI_M = N1 + (ROWS == 2 ? 4 : 2);
     static constexpr int SC = N + N2 + 16 / ROWS;
     static constexpr int HEAD = kHeadT0;
+    // the direct head of each row is split over HP warps by ranges of j
+    static constexpr int HP = NWARPS / ROWS;
     static constexpr size_t XBYTES = (size_t)ROWS * SC * 8;
-    static constexpr size_t HBYTES = (size_t)ROWS * HEAD * 8;  // direct-sum results r_t, t < HEAD, [ROWS][2*HEAD] floats
+    static constexpr size_t HBYTES = ((size_t)ROWS * HP * HEAD * 4 + 15) / 16 * 16;  // [ROWS][HP][HEAD] partial sums
     // staging: [LMAX][ROWS] elements of IO for v, then for g
     static constexpr size_t SBYTES = (size_t)2 * LMAX * ROWS * sizeof(IO);
     // norm partials [NWARPS][ROWS] float2, per-row scale [ROWS] float (padded),
     // rotations [(2h+s)][H+1] float2 (padded so the four (h, s) lane groups hit distinct banks)
     static constexpr size_t RBYTES = (size_t)(NWARPS * ROWS) * 8 + (size_t)ROWS * 8 + (size_t)4 * (N2 / 2 + 1) * 8;
-    static constexpr size_t SMEM_BYTES = XBYTES + HBYTES + SBYTES + RBYTES;
+    // staging starts on a 128-byte boundary (TMA destination)
+    static constexpr size_t SOFF = (XBYTES + HBYTES + 127) / 128 * 128;
+    // + one mbarrier (8 bytes, padded)
+    static constexpr size_t SMEM_BYTES = SOFF + SBYTES + RBYTES + 16;
+    // TMA staging: boxes of [BOXT t][ROWS d]; a box row must be a multiple of 16 bytes
+    static constexpr bool TMA_OK = (ROWS * sizeof(IO)) % 16 == 0;
+    static constexpr int BOXT = LMAX < 256 ? LMAX : 256;
+    static constexpr int NBOX = LMAX / BOXT;
+    static constexpr unsigned STAGE_BYTES = (unsigned)SBYTES;
     // Twiddle table layout (float2, built on the host in fp64), theta = omega_2N:
     //   T1[k1*N2 + n2]           = theta^(n2 (2 k1 + 1))         k1 < N1, n2 < N2
     //   P [N + k2*N1 + k1]       = theta^-(2 (k1 + N1 k2) + 1)   k2 < M2
@@ -106,17 +125,17 @@ struct FusedCfg {
     static constexpr int TW_Q = N + N / 2;
     static constexpr int TW_SIZE = 2 * N;
     static_assert(N2 == 16 || N2 == 32, "register DFT sizes 16..32 supported");
-    static_assert(THREADS == 256, "lane maps assume 8 warps per CTA");
+    static_assert(THREADS == 128 || THREADS == 256, "lane maps assume 4 or 8 warps per CTA");
+    static_assert(NWARPS % ROWS == 0 && HEAD % HP == 0, "head split");
     static_assert(SC >= N2 * SF_N && SC >= M2 * SI_M, "exchange buffers must fit the row stride");
     static_assert(16 % ROWS == 0 && 4 * ROWS <= 32, "ROWS must divide 16 and leave room for (h, s) lane bits");
-    static_assert(HEAD == 32 && HEAD <= LMAX && HEAD % N2 == 0, "the direct head is one warp per row");
-    static_assert(ROWS <= NWARPS, "one warp per row computes the direct head");
+    static_assert(HEAD == 32 && HEAD <= LMAX && HEAD % N2 == 0, "the direct head spans one warp of t");
     // bytes per t per array in staging, and the cp.async chunk covering them
     static constexpr int CH = ROWS * (int)sizeof(IO);
     static constexpr int CHUNK = CH < 16 ? CH : 16;
     static constexpr int NCHUNK = CH / CHUNK;
     static_assert(CH % CHUNK == 0 && (CHUNK == 4 || CHUNK == 8 || CHUNK == 16), "staging chunking");
-    static_assert((XBYTES + HBYTES) % 16 == 0 && (LMAX * CH) % 16 == 0, "staging must be 16-byte aligned");
+    static_assert((LMAX * CH) % 128 == 0 && LMAX % BOXT == 0, "staging boxes must stay 128-byte aligned");
 };
 
 // X' = -i (Zk + conj Zm)(Zk - conj Zm) = 4 V_k G_k for z = v + i g, Zm = mirror bin.
@@ -218,8 +237,12 @@ __device__ __forceinline__ void bar_sync(int id, int count) {
 template <int N2, int ROWS, int MINB, typename IO>
 __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
     fftconv_fused_kernel(const IO *__restrict__ v, const IO *__restrict__ g, IO *__restrict__ r, int L, int D,
-                         int groups_per_batch, int num_tiles, int vec_ok, int rev, const float2 *__restrict__ tw) {
+                         int groups_per_batch, int num_tiles, int vec_ok, int rev, const float2 *__restrict__ tw,
+                         const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmg,
+                         int use_tma) {
     // rev bit 0: read v reversed in time (v_t -> v_{L-1-t}); bit 1: write r reversed
+    // use_tma: stage tiles with TMA boxes from tmv / tmg (3-D maps over {D, L, B}),
+    // otherwise with cp.async from the pointers
     using C = FusedCfg<N2, ROWS, IO>;
     constexpr int N1 = C::N1, N = C::N, M2 = C::M2, H = C::H, MH = C::MH;
     const bool rev_a = rev & 1, rev_out = (rev >> 1) & 1;
@@ -227,13 +250,33 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
     constexpr int THREADS = C::THREADS;
     extern __shared__ float4 smem_raw[];
     float2 *xs = reinterpret_cast<float2 *>(smem_raw);
-    float *hres = reinterpret_cast<float *>(xs + ROWS * SC);  // [ROWS][2*HEAD]: direct sums r_t, t < HEAD
-    IO *sv = reinterpret_cast<IO *>(hres + ROWS * 2 * HEAD);
+    float *hres = reinterpret_cast<float *>(xs + ROWS * SC);  // [ROWS][HP][HEAD]: partial direct sums, t < HEAD
+    IO *sv = reinterpret_cast<IO *>(reinterpret_cast<char *>(smem_raw) + C::SOFF);
     IO *sg = sv + LMAX * ROWS;
     float2 *red = reinterpret_cast<float2 *>(sg + LMAX * ROWS);  // [NWARPS][ROWS] partial norms
     float *alpha_row = reinterpret_cast<float *>(red + C::NWARPS * ROWS);  // [ROWS] balance scale
     float2 *rot = reinterpret_cast<float2 *>(alpha_row + 2 * ROWS);       // [2h+s][H+1]
+    uint64_t *bar = reinterpret_cast<uint64_t *>(rot + 4 * (H + 1));      // staging-complete barrier
     const int tid = threadIdx.x;
+    const bool tma = C::TMA_OK && use_tma && (smem_u32(sv) & 127) == 0;
+    unsigned phase = 0;
+    // stage tile `t` (v and g, t < LMAX, zero-filled past L and D) into sv / sg
+    auto issue = [&](int t) {
+        const int b = t / groups_per_batch, d0 = (t - b * groups_per_batch) * ROWS;
+        if (tma) {
+            if (tid == 0) {
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
+#pragma unroll
+                for (int k = 0; k < C::NBOX; ++k) {
+                    tma_load_3d(sv + k * C::BOXT * ROWS, &tmv, d0, k * C::BOXT, b, bar);
+                    tma_load_3d(sg + k * C::BOXT * ROWS, &tmg, d0, k * C::BOXT, b, bar);
+                }
+            }
+        } else {
+            stage_tile<C, IO>(v, g, sv, sg, (int64_t)b * L * D, d0, L, D, vec_ok && d0 + ROWS <= D, rev_a);
+        }
+    };
 
     // rot[2h+s][m] = omega_2N1^-((2h+1) m1), m1 = H s + m: untwist of the
     // odd-frequency grid times the parity rotation of the last inverse step
@@ -241,25 +284,42 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
         const int hs = i / H, m = i - hs * H, hh = hs >> 1, m1 = H * (hs & 1) + m;
         rot[hs * (H + 1) + m] = cconj(c_w128[((2 * hh + 1) * m1 * (128 / (2 * N1))) & 127]);
     }
-    // staging beyond L is never written by the copies: zero it once so loads need no bounds test
-    for (int i = L * ROWS + tid; i < LMAX * ROWS; i += THREADS) {
-        sv[i] = IO(0.f);
-        sg[i] = IO(0.f);
+    if (tma) {
+        if (tid == 0) mbar_init(bar, 1);
+    } else {
+        // staging beyond L is never written by the copies: zero it once so loads need no bounds test
+        for (int i = L * ROWS + tid; i < LMAX * ROWS; i += THREADS) {
+            sv[i] = IO(0.f);
+            sg[i] = IO(0.f);
+        }
     }
+    __syncthreads();
 
     int tile = blockIdx.x;
     if (tile >= num_tiles) return;
-    {
-        const int b = tile / groups_per_batch, d0 = (tile - b * groups_per_batch) * ROWS;
-        stage_tile<C, IO>(v, g, sv, sg, (int64_t)b * L * D, d0, L, D, vec_ok && d0 + ROWS <= D, rev_a);
-    }
+    issue(tile);
 
     for (; tile < num_tiles; tile += gridDim.x) {
         const int b = tile / groups_per_batch;
         const int d0 = (tile - b * groups_per_batch) * ROWS;
         const int64_t boff = (int64_t)b * L * D;
-        cp_async_wait_all();
-        __syncthreads();  // staging complete; previous tile's I3 done with xs / head
+        bool staged = true;
+        if (tma) {
+            staged = mbar_wait_bounded(bar, phase);
+            phase ^= 1u;
+        } else {
+            cp_async_wait_all();
+        }
+        // staging complete; previous tile's I3 done with xs / head
+        if (__syncthreads_or(!staged)) {
+            // a copy did not complete in time: flag it, give the copies in
+            // flight one more bounded wait, and stop
+            if (tid == 0) {
+                atomicOr(&g_cc_fault, kFaultTmaWait);
+                mbar_wait_bounded(bar, phase ^ 1u);
+            }
+            return;
+        }
 
         // ------------------------------------------------------------ F1
         // thread (e, n2, c): half-spectrum e (k1 = 2k'+e) of column n2 of row c
@@ -276,20 +336,22 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
                 nv = fmaf(zv.x, zv.x, nv);
                 ng = fmaf(zv.y, zv.y, ng);
             }
-            // direct sums r_t = sum_{j<=t} v_j g_{t-j} for t < HEAD: warp w < ROWS
-            // handles row w, lane t
-            if ((tid >> 5) < ROWS) {
-                const int hc = tid >> 5, lt = tid & 31;
+            // direct sums r_t = sum_{j<=t} v_j g_{t-j} for t < HEAD: warp w takes
+            // row w % ROWS, lane t, and the j range of part w / ROWS
+            {
+                constexpr int HP = C::HP, JP = HEAD / HP;
+                const int w = tid >> 5, hc = w % ROWS, hp = w / ROWS, lt = tid & 31;
                 const float vt = IO_t<IO>::cvt(sv[lt * ROWS + hc]);
                 const float gt = IO_t<IO>::cvt(sg[lt * ROWS + hc]);
                 float acc = 0.f;
 #pragma unroll
-                for (int jj = 0; jj < HEAD; ++jj) {
-                    const float vj = __shfl_sync(0xffffffffu, vt, jj);
-                    const float gtj = __shfl_up_sync(0xffffffffu, gt, jj);
-                    if (lt >= jj) acc = fmaf(vj, gtj, acc);
+                for (int jj = 0; jj < JP; ++jj) {
+                    const int j = hp * JP + jj;
+                    const float vj = __shfl_sync(0xffffffffu, vt, j);
+                    const float gtj = __shfl_up_sync(0xffffffffu, gt, j);
+                    if (lt >= j) acc = fmaf(vj, gtj, acc);
                 }
-                hres[hc * 2 * HEAD + lt] = acc;
+                hres[(hc * HP + hp) * HEAD + lt] = acc;
             }
 #pragma unroll
             for (int m = ROWS; m < 32; m <<= 1) {
@@ -307,30 +369,31 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
             const float alpha = balance_scale(tot.x, tot.y);
             if (tid < ROWS) alpha_row[c] = alpha;
 
-            // x[n1] = z[n2 + N2 n1] * omega_2N1^((2e+1) n1), in bit-reversed slots
-            float2 x[N2];
+            // x[n1] = z[n2 + N2 n1] * omega_2N1^((2e+1) n1), in bit-reversed slots;
+            // e is warp-uniform, so each warp runs the branch with its twist as constants
+            auto half_spectrum = [&](auto e_const) {
+                constexpr int E = decltype(e_const)::value;
+                float2 x[N2];
 #pragma unroll
-            for (int n1 = 0; n1 < N2; ++n1) {
-                const float2 zv = make_float2(zr[n1].x, alpha * zr[n1].y);
-                const float2 w = e ? tw_const(3 * n1, 2 * N1) : tw_const(n1, 2 * N1);
-                x[bitrev(n1, C::LOG_N2)] = n1 == 0 ? zv : cmul(zv, w);
-            }
-            fft_dit<N2, false>(x);  // x[k'] -> k1 = 2k' + e
-            float2 *xrow = xs + c * SC + n2 * SF_N + e;
-            const float2 *t1 = tw + e * N2 + n2;
+                for (int n1 = 0; n1 < N2; ++n1) {
+                    const float2 zv = make_float2(zr[n1].x, alpha * zr[n1].y);
+                    x[bitrev(n1, C::LOG_N2)] = n1 == 0 ? zv : cmul(zv, tw_const((2 * E + 1) * n1, 2 * N1));
+                }
+                fft_dit<N2, false>(x);  // x[k'] -> k1 = 2k' + e
+                float2 *xrow = xs + c * SC + n2 * SF_N + E;
+                const float2 *t1 = tw + E * N2 + n2;
 #pragma unroll
-            for (int kp = 0; kp < N2; ++kp) xrow[2 * kp] = cmul(x[kp], __ldg(t1 + 2 * kp * N2));
+                for (int kp = 0; kp < N2; ++kp) xrow[2 * kp] = cmul(x[kp], __ldg(t1 + 2 * kp * N2));
+            };
+            if (e)
+                half_spectrum(std::integral_constant<int, 1>{});
+            else
+                half_spectrum(std::integral_constant<int, 0>{});
         }
         __syncthreads();  // exchange complete; staging free
 
         // prefetch the next tile while this one finishes
-        {
-            const int nt = tile + gridDim.x;
-            if (nt < num_tiles) {
-                const int nb = nt / groups_per_batch, nd0 = (nt - nb * groups_per_batch) * ROWS;
-                stage_tile<C, IO>(v, g, sv, sg, (int64_t)nb * L * D, nd0, L, D, vec_ok && nd0 + ROWS <= D, rev_a);
-            }
-        }
+        if (tile + (int)gridDim.x < num_tiles) issue(tile + gridDim.x);
 
         // ------------------------------------------------------------ F3
         // Column pair (j, N1-1-j) of row c is shared by two lanes s = 0, 1 (lane ^ 16).
@@ -448,8 +511,13 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
                 const int t = t0 + N2 * i;
                 float r0 = o.x * sc, r1 = o.y * sc;
                 if (i * N2 < HEAD && t < HEAD) {
-                    r0 = hres[c * 2 * HEAD + t];
-                    r1 = hres[c * 2 * HEAD + t + 1];
+                    r0 = 0.f;
+                    r1 = 0.f;
+#pragma unroll
+                    for (int p = 0; p < C::HP; ++p) {
+                        r0 += hres[(c * C::HP + p) * HEAD + t];
+                        r1 += hres[(c * C::HP + p) * HEAD + t + 1];
+                    }
                 }
                 if (dok && t < L) IO_t<IO>::st(rp, r0);
                 if (dok && t + 1 < L) IO_t<IO>::st(rp + dir * D, r1);
@@ -457,7 +525,7 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
             }
         }
     }
-    cp_async_wait_all();
+    if (!tma) cp_async_wait_all();
 }
 
 }  // namespace ccv

@@ -154,3 +154,10 @@ def test_decode_alias_is_range_exact(lib):
     assert f(A, B_, A + cache, B, L, D, 3, W, 8, None) == 4      # passes the alias check, fails on workspace
     assert f(A, B_, A + cache - 4, B, L, D, 3, W, 8, None) == 3  # last cache element overlaps
     assert f(A, B_, A - B * D * 4, B, L, D, 3, W, 8, None) == 4  # output right before the cache
+
+
+def test_fault_flags_host_checks(lib):
+    import ctypes
+    assert lib.causal_conv_fault_flags(0, None, 0) == 1                      # NULL flags
+    out = ctypes.c_uint(7)
+    assert lib.causal_conv_fault_flags(-1, ctypes.byref(out), 0) == 1       # bad device

@@ -25,8 +25,12 @@ def _rand_float(shape, seed, scale_g=1.0):
 
 
 # shapes spanning several tiles with ragged tails in L (vs N/2) and D (vs the channel tile)
+# (D * element size a multiple of 16 bytes selects the TMA staging: (3, 200, 36)
+# and (2, 130, 24) end in a partial channel group the copy engine zero-fills,
+# (1, 513, 4) and (2, 700, 20) have many zero-filled time steps past L)
 FLOAT_SHAPES = [(1, 1, 1), (1, 2, 3), (1, 3, 2), (2, 31, 5), (1, 32, 4), (1, 33, 7), (3, 200, 19), (1, 256, 8),
-                (2, 257, 9), (2, 513, 5), (2, 1000, 37), (1, 1024, 12)]
+                (2, 257, 9), (2, 513, 5), (2, 1000, 37), (1, 1024, 12), (3, 200, 36), (2, 130, 24), (1, 513, 4),
+                (2, 700, 20)]
 
 
 @pytest.mark.parametrize("shape", FLOAT_SHAPES, ids=lambda s: "x".join(map(str, s)))
@@ -46,6 +50,38 @@ def test_bf16_parity_full_oracle(shape):
     r_ref, den = oracle.causal_conv(as_f32(vb, "bf16"), as_f32(gb, "bf16"))
     n_bad, worst = float_violations(as_f32(r, "bf16"), r_ref, den, BF16_TOL)
     assert n_bad == 0, f"{n_bad} elements beyond the bf16 bound, worst ratio {worst:.3g}"
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_unaligned_base_pointers(dtype):
+    """Tensors starting 4 (f32) or 2 (bf16) bytes past an allocation: no tensor
+    map can describe them, so the threads stage the tiles themselves."""
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    shape = (2, 300, 16)
+    v, g = _rand_float(shape, seed=99, scale_g=0.125)
+    if dtype == "bf16":
+        v, g = workloads.bf16_round(v), workloads.bf16_round(g)
+    n = int(np.prod(shape))
+    tv, tg = to_dev(v.reshape(-1), dtype), to_dev(g.reshape(-1), dtype)
+    bv = torch.empty(n + 1, dtype=tv.dtype, device="cuda")
+    bg = torch.empty(n + 1, dtype=tv.dtype, device="cuda")
+    bv[1:] = tv
+    bg[1:] = tg
+    r = ssm.causal_conv(bv[1:].view(shape), bg[1:].view(shape))
+    torch.cuda.synchronize()
+    r_ref, den = oracle.causal_conv(as_f32(v, dtype), as_f32(g, dtype))
+    n_bad, worst = float_violations(as_f32(from_dev(r, dtype), dtype), r_ref, den,
+                                    F32_TOL if dtype == "f32" else BF16_TOL)
+    assert n_bad == 0, f"{n_bad} elements beyond the bound, worst ratio {worst:.3g}"
+
+
+def test_no_kernel_wait_ran_out():
+    """Every bounded wait in the kernels completed during the tests so far."""
+    import spectral_sequence_mixing_b200 as ssm
+    v, g = _rand_float((4, 1024, 64), seed=5)
+    run_gpu(v, g, "f32")
+    assert ssm.fault_flags() == 0
 
 
 INT_SHAPES = [(1, 1, 1), (1, 2, 3), (2, 33, 5), (2, 1000, 37), (1, 4097, 3), (1, 8192, 2)]
