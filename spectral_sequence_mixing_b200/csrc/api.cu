@@ -115,6 +115,15 @@ static cudaError_t ensure_init(int dev) {
     for (int k = 0; k < 128; ++k) w128[k] = omega(k, 128);
     if ((e = cudaMemcpyToSymbol(c_w128, w128, sizeof(w128))) != cudaSuccess) return e;
     {
+        float2 tw1[2][2][32];
+        for (int sz = 0; sz < 2; ++sz) {
+            const int n2s = sz ? 32 : 16, two_n1 = 4 * n2s;
+            for (int ee = 0; ee < 2; ++ee)
+                for (int n1 = 0; n1 < 32; ++n1) tw1[sz][ee][n1] = omega((int64_t)(2 * ee + 1) * n1, two_n1);
+        }
+        if ((e = cudaMemcpyToSymbol(c_f1_twist, tw1, sizeof(tw1))) != cudaSuccess) return e;
+    }
+    {
         auto t = fused_twiddles<CfgS<float>>();
         if ((e = cudaMemcpyToSymbol(g_tw_s, t.data(), t.size() * sizeof(float2))) != cudaSuccess) return e;
     }

@@ -50,14 +50,16 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include <type_traits>
-
 #include "fft_reg.cuh"
 #include "tma.cuh"
 
 namespace ccv {
 
 constexpr int kHeadT0 = 32;
+
+// F1 input twist omega_2N1^((2e+1) n1) for N2 = 16 (N1 = 32) and N2 = 32
+// (N1 = 64): c_f1_twist[N2 == 32][e][n1], n1 < N2; filled once per device.
+__constant__ float2 c_f1_twist[2][2][32];
 
 template <typename IO>
 struct IO_t;
@@ -369,26 +371,21 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
             const float alpha = balance_scale(tot.x, tot.y);
             if (tid < ROWS) alpha_row[c] = alpha;
 
-            // x[n1] = z[n2 + N2 n1] * omega_2N1^((2e+1) n1), in bit-reversed slots;
-            // e is warp-uniform, so each warp runs the branch with its twist as constants
-            auto half_spectrum = [&](auto e_const) {
-                constexpr int E = decltype(e_const)::value;
-                float2 x[N2];
+            // x[n1] = z[n2 + N2 n1] * omega_2N1^((2e+1) n1), in bit-reversed slots.
+            // e is warp-uniform: the twist comes from a constant table at a
+            // per-warp offset, so both halves share one copy of the code.
+            const float2 *twist = c_f1_twist[N2 == 32 ? 1 : 0][e];
+            float2 x[N2];
 #pragma unroll
-                for (int n1 = 0; n1 < N2; ++n1) {
-                    const float2 zv = make_float2(zr[n1].x, alpha * zr[n1].y);
-                    x[bitrev(n1, C::LOG_N2)] = n1 == 0 ? zv : cmul(zv, tw_const((2 * E + 1) * n1, 2 * N1));
-                }
-                fft_dit<N2, false>(x);  // x[k'] -> k1 = 2k' + e
-                float2 *xrow = xs + c * SC + n2 * SF_N + E;
-                const float2 *t1 = tw + E * N2 + n2;
+            for (int n1 = 0; n1 < N2; ++n1) {
+                const float2 zv = make_float2(zr[n1].x, alpha * zr[n1].y);
+                x[bitrev(n1, C::LOG_N2)] = n1 == 0 ? zv : cmul(zv, twist[n1]);
+            }
+            fft_dit<N2, false>(x);  // x[k'] -> k1 = 2k' + e
+            float2 *xrow = xs + c * SC + n2 * SF_N + e;
+            const float2 *t1 = tw + e * N2 + n2;
 #pragma unroll
-                for (int kp = 0; kp < N2; ++kp) xrow[2 * kp] = cmul(x[kp], __ldg(t1 + 2 * kp * N2));
-            };
-            if (e)
-                half_spectrum(std::integral_constant<int, 1>{});
-            else
-                half_spectrum(std::integral_constant<int, 0>{});
+            for (int kp = 0; kp < N2; ++kp) xrow[2 * kp] = cmul(x[kp], __ldg(t1 + 2 * kp * N2));
         }
         __syncthreads();  // exchange complete; staging free
 
