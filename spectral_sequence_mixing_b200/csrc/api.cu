@@ -87,8 +87,12 @@ static std::vector<float2> big_twiddles() {
 
 template <class Cfg, typename IO, int MINB>
 static cudaError_t set_big_attr() {
-    return cudaFuncSetAttribute(bigconv_kernel<Cfg::R0, Cfg::RA, Cfg::RB, Cfg::RC, Cfg::CL, Cfg::T, MINB, IO>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_BYTES);
+    if constexpr (Cfg::CL == 1)
+        return cudaFuncSetAttribute(bigrow_group_kernel<Cfg::R0, Cfg::RA, Cfg::RB, Cfg::RC, Cfg::T, MINB, IO>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_BYTES);
+    else
+        return cudaFuncSetAttribute(bigconv_kernel<Cfg::R0, Cfg::RA, Cfg::RB, Cfg::RC, Cfg::CL, Cfg::T, MINB, IO>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_BYTES);
 }
 
 static std::mutex g_init_mu;
@@ -328,6 +332,38 @@ static int launch_big(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int
     return CC_OK;
 }
 
+// Rows that fit one CTA, kGroup adjacent channels per cluster.
+template <class Cfg, int MINB, typename IO>
+static int launch_group(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, const float2 *tw,
+                        cudaStream_t s, int rev) {
+    static_assert(Cfg::CL == 1, "one row per CTA");
+    const int64_t gpb = (D + kGroup - 1) / kGroup;
+    if (B * gpb * kGroup > INT32_MAX) return CC_ERR_UNSUPPORTED;
+    auto kern = bigrow_group_kernel<Cfg::R0, Cfg::RA, Cfg::RB, Cfg::RC, Cfg::T, MINB, IO>;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(B * gpb * kGroup));
+    cfg.blockDim = dim3(Cfg::T);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kGroup;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // 16-byte group accesses: every (b, t) row of D elements and the bases 16-byte aligned
+    const bool vec = (D * (int64_t)sizeof(IO)) % 16 == 0 && ((uintptr_t)v % 16) == 0 && ((uintptr_t)g % 16) == 0 &&
+                     ((uintptr_t)r % 16) == 0;
+    const cudaError_t e =
+        cudaLaunchKernelEx(&cfg, kern, v, g, r, (int)L, (int)D, (int)gpb, rev, vec ? 1 : 0, tw);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return CC_ERR_CUDA;
+    }
+    return CC_OK;
+}
+
 template <typename IO>
 static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, cudaStream_t s,
                             int dev, int rev = 0) {
@@ -342,7 +378,7 @@ static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t 
     }
     if (L <= BigL<IO>::LMAX) {
         if (cudaGetSymbolAddress(&tw, g_tw_bl) != cudaSuccess) return CC_ERR_CUDA;
-        return launch_big<BigL<IO>, kMinbBigL>(v, g, r, B, L, D, (const float2 *)tw, s, rev);
+        return launch_group<BigL<IO>, kMinbBigL>(v, g, r, B, L, D, (const float2 *)tw, s, rev);
     }
     if (L <= BigX<IO>::LMAX) {
         if (cudaGetSymbolAddress(&tw, g_tw_bx) != cudaSuccess) return CC_ERR_CUDA;

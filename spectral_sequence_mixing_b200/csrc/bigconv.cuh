@@ -71,7 +71,7 @@ struct BigCfg {
     static_assert(CL == 1 || CL == R0, "a cluster splits the most significant digit");
     static_assert(LAST_R == 16, "innermost radix must be 16 (conflict-free padded layout)");
     static_assert(R0 <= 64 && RA <= 32 && RB <= 32 && RC <= 32, "register DFT sizes");
-    static_assert(SC % T == 0 && COLS0 % T == 0, "pass work split");
+    static_assert(SC % (2 * T) == 0 && COLS0 % T == 0, "pass work split");
 };
 
 __device__ __forceinline__ int bc_pad(int p) { return p + (p >> 4); }
@@ -279,24 +279,24 @@ __global__ void __launch_bounds__(T, MINB)
     }
     cluster_sync();
 
-    // ---- spectral product X' = 4 V G at every own slot, from Z_s and Z_{S-1-s}
+    // ---- spectral product X' = 4 V G.  The pair (s, S-1-s) is handled by the
+    // thread that owns s at local offset o < SC/2 (the mirror then sits at a
+    // local offset >= SC/2, here or in CTA R0-1-rank): it reads both bins and
+    // writes X'_s and X'_{S-1-s} = conj(X'_s), so every slot is read and
+    // written by one thread only.
     {
-        constexpr int PER = SC / T;
-        float2 xv[PER];
-#pragma unroll
-        for (int i = 0; i < PER; ++i) {
-            const int o = tid + i * T;               // own offset
-            const int s = rank * SC + o;             // global slot (k0-major within the cluster)
-            const float2 zk = xs[bc_pad(o)];
-            const int sm = S - 1 - s;
-            const float2 zm = slot_ld(slot_addr(sm / SL, sm % SL));
-            xv[i] = spectral_product(zk, zm);
+        constexpr int PER2 = SC / (2 * T);
+#pragma unroll 4
+        for (int i = 0; i < PER2; ++i) {
+            const int o = tid + i * T;
+            const int sm = S - 1 - (rank * SC + o);
+            const uint32_t am = slot_addr(sm / SL, sm % SL);
+            const float2 xk = spectral_product(xs[bc_pad(o)], slot_ld(am));
+            xs[bc_pad(o)] = xk;
+            slot_st(am, cconj(xk));
         }
-        cluster_sync();  // every mirror read done before any slot is overwritten
-#pragma unroll
-        for (int i = 0; i < PER; ++i) xs[bc_pad(tid + i * T)] = xv[i];
     }
-    __syncthreads();
+    cluster_sync();
 
     // ---- inverse local passes
     if constexpr (RC > 1) {
@@ -339,6 +339,248 @@ __global__ void __launch_bounds__(T, MINB)
         }
     }
     cluster_sync();  // keep this CTA's shared memory alive until the cluster is done with it
+}
+
+// ---------------------------------------------------------------------------
+// Channel groups: rows that fit one CTA, kGroup adjacent channels of one
+// batch per cluster (one channel per CTA).  Reading one channel of a
+// channel-last tensor touches a separate 2..4-byte piece of memory per time
+// step; a group reads all kGroup channels of a time step in one 16..32-byte
+// piece instead.  CTA q of the cluster loads time steps
+// [q LMAX/kGroup, (q+1) LMAX/kGroup) of the whole group and writes
+// (v_t, g_t) of channel c straight into slot t of CTA c (distributed shared
+// memory), which is where the row's pass 0 reads its input (t = n0 SL + n is
+// slot (n0, n), the column pass 0 rewrites in place).  The last inverse pass
+// leaves r_t in slot t the same way, and CTA q gathers its time steps of all
+// kGroup channels for the stores.
+constexpr int kGroup = 8;
+
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+    float x;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(x) : "r"(addr) : "memory");
+    return x;
+}
+
+// kGroup consecutive channels at p[0..nch) (zeros beyond nch, or everywhere when !inb).
+template <typename IO>
+__device__ __forceinline__ void load_group(const IO *__restrict__ p, int nch, bool vec, bool inb, float (&o)[kGroup]) {
+#pragma unroll
+    for (int c = 0; c < kGroup; ++c) o[c] = 0.f;
+    if (!inb) return;
+    if (vec) {
+        if constexpr (sizeof(IO) == 2) {
+            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(p));
+            const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int c = 0; c < kGroup; ++c) o[c] = __uint_as_float(((u[c / 2] >> (16 * (c & 1))) & 0xffffu) << 16);
+        } else {
+            const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+            const float4 bq = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+            o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+            o[4] = bq.x; o[5] = bq.y; o[6] = bq.z; o[7] = bq.w;
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < kGroup; ++c)
+            if (c < nch) o[c] = IO_t<IO>::cvt(IO_t<IO>::ld(p + c));
+    }
+}
+
+template <typename IO>
+__device__ __forceinline__ void store_group(IO *__restrict__ p, int nch, bool vec, const float (&o)[kGroup]) {
+    if (vec) {
+        if constexpr (sizeof(IO) == 2) {
+            uint32_t u[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                u[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o[2 * i])) |
+                       ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(o[2 * i + 1])) << 16);
+            *reinterpret_cast<uint4 *>(p) = make_uint4(u[0], u[1], u[2], u[3]);
+        } else {
+            reinterpret_cast<float4 *>(p)[0] = make_float4(o[0], o[1], o[2], o[3]);
+            reinterpret_cast<float4 *>(p)[1] = make_float4(o[4], o[5], o[6], o[7]);
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < kGroup; ++c)
+            if (c < nch) IO_t<IO>::st(p + c, o[c]);
+    }
+}
+
+template <int R0, int RA, int RB, int RC, int T, int MINB, typename IO>
+__global__ void __launch_bounds__(T, MINB)
+    bigrow_group_kernel(const IO *__restrict__ v, const IO *__restrict__ g, IO *__restrict__ r, int L, int D,
+                        int groups_per_batch, int rev, int vec_ok, const float2 *__restrict__ tw) {
+    // rev bit 0: read v reversed in time; bit 1: write r reversed.  vec_ok:
+    // whole groups may use 16-byte accesses (D and the base pointers allow it).
+    using C = BigCfg<R0, RA, RB, RC, 1, T, IO>;
+    constexpr int S = C::S, SL = C::SL, HEAD = C::HEAD, LMAX = C::LMAX;
+    constexpr int LOG_R0 = ilog2(R0);
+    static_assert(LMAX % kGroup == 0, "time steps split evenly over the group");
+    extern __shared__ float4 bsm_raw[];
+    float2 *xs = reinterpret_cast<float2 *>(bsm_raw);
+    float2 *head = xs + C::WORDS;
+    const int tid = threadIdx.x;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    const int grp = blockIdx.x / kGroup;
+    const int b = grp / groups_per_batch, d0 = (grp - b * groups_per_batch) * kGroup;
+    const int nch = min(kGroup, D - d0);
+    const bool vec = vec_ok && nch == kGroup;
+    const int64_t gbase = (int64_t)b * L * D + d0;  // element (b, 0, d0)
+    const uint32_t xs_addr = smem_addr(xs);
+    cluster.sync();  // every CTA of the cluster runs before the first remote store
+
+    // ---- cooperative load of time steps [t0, t0 + LMAX/kGroup), zeros past L
+    {
+        constexpr int TC = LMAX / kGroup;
+        const int t0 = rank * TC;
+        uint32_t dst[kGroup];
+#pragma unroll
+        for (int c = 0; c < kGroup; ++c) dst[c] = cluster_map(xs_addr, c);
+#pragma unroll 2
+        for (int t = t0 + tid; t < t0 + TC; t += T) {
+            float vv[kGroup], gg[kGroup];
+            const bool inb = t < L;
+            load_group<IO>(v + gbase + (int64_t)((rev & 1) ? L - 1 - t : t) * D, nch, vec, inb, vv);
+            load_group<IO>(g + gbase + (int64_t)t * D, nch, vec, inb, gg);
+            const uint32_t off = 8u * (uint32_t)bc_pad(t);
+#pragma unroll
+            for (int c = 0; c < kGroup; ++c) st_cluster(dst[c] + off, make_float2(vv[c], gg[c]));
+        }
+    }
+    cluster.sync();
+
+    // ---- this CTA's row: input of the pass-0 columns, norms for balancing
+    float2 zin[C::PER0][R0 / 2];
+    float nv = 0.f, ng = 0.f;
+#pragma unroll
+    for (int p = 0; p < C::PER0; ++p) {
+        const int n = tid + p * T;
+#pragma unroll
+        for (int n0 = 0; n0 < R0 / 2; ++n0) {
+            const int t = n0 * SL + n;
+            const float2 z = xs[bc_pad(t)];
+            if (t < HEAD) head[t] = z;
+            zin[p][n0] = z;
+            nv = fmaf(z.x, z.x, nv);
+            ng = fmaf(z.y, z.y, ng);
+        }
+    }
+    float alpha;
+    {
+        float2 *red = head + HEAD;
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+            nv += __shfl_xor_sync(0xffffffffu, nv, m);
+            ng += __shfl_xor_sync(0xffffffffu, ng, m);
+        }
+        if ((tid & 31) == 0) red[tid >> 5] = make_float2(nv, ng);
+        __syncthreads();
+        float2 tot = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < T / 32; ++w) {
+            tot.x += red[w].x;
+            tot.y += red[w].y;
+        }
+        alpha = balance_scale(tot.x, tot.y);
+    }
+    auto tw0 = [&](int k0, int n) -> float2 {
+        const float2 a = __ldg(tw + C::T0A + k0 * C::Q0 + (n % C::Q0));
+        if constexpr (SL > C::Q0) return cmul(a, __ldg(tw + C::T0B + k0 * (SL / C::Q0) + (n / C::Q0)));
+        return a;
+    };
+
+    // ---- forward pass 0 (in place per column n: reads slots (n0, n), writes (k0, n))
+#pragma unroll
+    for (int p = 0; p < C::PER0; ++p) {
+        const int n = tid + p * T;
+        float2 x[R0];
+#pragma unroll
+        for (int n0 = 0; n0 < R0 / 2; ++n0) {
+            const float2 z = make_float2(zin[p][n0].x, alpha * zin[p][n0].y);
+            x[bitrev(n0, LOG_R0)] = n0 == 0 ? z : cmul(z, tw_const(n0, 2 * R0));
+        }
+        fft_dit<R0, false, true>(x);
+#pragma unroll
+        for (int k0 = 0; k0 < R0; ++k0) xs[bc_pad(k0 * SL + n)] = cmul(x[k0], tw0(k0, n));
+    }
+    __syncthreads();
+
+    // ---- forward local passes, spectral product, inverse local passes
+    bc_local_pass<RA, C::STA, C::QA, SL, S, T, false>(xs, tw + C::TAA, tw + C::TAB);
+    __syncthreads();
+    if constexpr (RC > 1) {
+        bc_local_pass<RB, RC, RC, SL, S, T, false>(xs, tw + C::TB, tw + C::TB);
+        __syncthreads();
+        bc_local_pass<RC, 1, 1, SL, S, T, false>(xs, tw, tw);
+    } else {
+        bc_local_pass<RB, 1, 1, SL, S, T, false>(xs, tw, tw);
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int i = 0; i < S / (2 * T); ++i) {  // pair (o, S-1-o), o < S/2
+        const int o = tid + i * T;
+        const float2 xk = spectral_product(xs[bc_pad(o)], xs[bc_pad(S - 1 - o)]);
+        xs[bc_pad(o)] = xk;
+        xs[bc_pad(S - 1 - o)] = cconj(xk);
+    }
+    __syncthreads();
+    if constexpr (RC > 1) {
+        bc_local_pass<RC, 1, 1, SL, S, T, true>(xs, tw, tw);
+        __syncthreads();
+        bc_local_pass<RB, RC, RC, SL, S, T, true>(xs, tw + C::TB, tw + C::TB);
+    } else {
+        bc_local_pass<RB, 1, 1, SL, S, T, true>(xs, tw, tw);
+    }
+    __syncthreads();
+    bc_local_pass<RA, C::STA, C::QA, SL, S, T, true>(xs, tw + C::TAA, tw + C::TAB);
+    __syncthreads();
+
+    // ---- inverse pass 0: twiddle, inverse R0-point DFT (outputs n0 < R0/2),
+    // untwist; r_t (t < L) is left in slot t of the same column
+    {
+        const float sc = 1.f / (4.f * (float)S * alpha);
+#pragma unroll 1
+        for (int n = tid; n < SL; n += T) {
+            float2 x[R0];
+#pragma unroll
+            for (int k0 = 0; k0 < R0; ++k0) x[bitrev(k0, LOG_R0)] = cmul_conj(xs[bc_pad(k0 * SL + n)], tw0(k0, n));
+            fft_dit<R0, true, false, true>(x);
+#pragma unroll
+            for (int n0 = 0; n0 < R0 / 2; ++n0) {
+                const int t = n0 * SL + n;
+                if (t >= L) continue;
+                const float2 w = tw_const(n0, 2 * R0);
+                float out = (n0 == 0 ? x[0].x : fmaf(x[n0].x, w.x, x[n0].y * w.y)) * sc;
+                if (t < HEAD) {
+                    float a = 0.f;
+                    for (int j = 0; j <= t; ++j) a = fmaf(head[j].x, head[t - j].y, a);
+                    out = a;
+                }
+                xs[bc_pad(t)].x = out;
+            }
+        }
+    }
+    cluster.sync();
+
+    // ---- cooperative store of time steps [t0, t1) of the group
+    {
+        const int TS = (L + kGroup - 1) / kGroup;
+        const int t0 = rank * TS, t1 = min(L, t0 + TS);
+        uint32_t src[kGroup];
+#pragma unroll
+        for (int c = 0; c < kGroup; ++c) src[c] = cluster_map(xs_addr, c);
+#pragma unroll 2
+        for (int t = t0 + tid; t < t1; t += T) {
+            float o[kGroup];
+            const uint32_t off = 8u * (uint32_t)bc_pad(t);
+#pragma unroll
+            for (int c = 0; c < kGroup; ++c) o[c] = ld_cluster_f32(src[c] + off);
+            store_group<IO>(r + gbase + (int64_t)((rev & 2) ? L - 1 - t : t) * D, nch, vec, o);
+        }
+    }
+    cluster.sync();  // remote reads of this CTA's slots are done before it exits
 }
 
 }  // namespace ccv

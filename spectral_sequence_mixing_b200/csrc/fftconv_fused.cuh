@@ -127,7 +127,7 @@ struct FusedCfg {
     static constexpr int TW_Q = N + N / 2;
     static constexpr int TW_SIZE = 2 * N;
     static_assert(N2 == 16 || N2 == 32, "register DFT sizes 16..32 supported");
-    static_assert(THREADS == 128 || THREADS == 256, "lane maps assume 4 or 8 warps per CTA");
+    static_assert(THREADS == 128 || THREADS == 256 || THREADS == 512, "lane maps assume 4, 8 or 16 warps per CTA");
     static_assert(NWARPS % ROWS == 0 && HEAD % HP == 0, "head split");
     static_assert(SC >= N2 * SF_N && SC >= M2 * SI_M, "exchange buffers must fit the row stride");
     static_assert(16 % ROWS == 0 && 4 * ROWS <= 32, "ROWS must divide 16 and leave room for (h, s) lane bits");

@@ -52,13 +52,14 @@ def test_bf16_parity_full_oracle(shape):
     assert n_bad == 0, f"{n_bad} elements beyond the bf16 bound, worst ratio {worst:.3g}"
 
 
+@pytest.mark.parametrize("shape", [(2, 300, 16), (1, 2000, 16)], ids=lambda s: "x".join(map(str, s)))
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_unaligned_base_pointers(dtype):
+def test_unaligned_base_pointers(dtype, shape):
     """Tensors starting 4 (f32) or 2 (bf16) bytes past an allocation: no tensor
-    map can describe them, so the threads stage the tiles themselves."""
+    map (fused kernel) and no 16-byte group access (channel-group clusters)
+    can describe them, so element-wise paths run."""
     import torch
     import spectral_sequence_mixing_b200 as ssm
-    shape = (2, 300, 16)
     v, g = _rand_float(shape, seed=99, scale_g=0.125)
     if dtype == "bf16":
         v, g = workloads.bf16_round(v), workloads.bf16_round(g)
@@ -133,7 +134,9 @@ def test_ntt_wraps_to_centered_residue():
 
 
 # rows longer than one fused tile: one row per CTA (L <= 4096) or per 8-CTA cluster (L <= 65536)
-BIG_SHAPES = [(1, 1025, 3), (2, 2000, 5), (1, 4096, 4)]
+# rows of one CTA run in clusters of 8 adjacent channels: partial groups
+# (D < 8, D = 12), whole groups with 16-byte accesses (D = 16, 24)
+BIG_SHAPES = [(1, 1025, 3), (2, 2000, 5), (1, 4096, 4), (1, 2000, 16), (2, 1500, 24), (1, 4096, 12)]
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
