@@ -15,6 +15,12 @@
 //
 // Layout: one CTA per row, both transforms resident in shared memory (two
 // arrays of N words, one pad word per 32 so every pass is conflict-free).
+// The CTAs of a cluster take kNttGroup adjacent channels of one batch: CTA q
+// reads time steps [q LMAX/kNttGroup, (q+1) LMAX/kNttGroup) of all of them
+// with one 16-byte access per time step and array, and writes each
+// channel's residues into the owning CTA's arrays (distributed shared
+// memory), at the slots the first pass reads; the last pass leaves the
+// outputs in place and CTA q stores its time steps of the whole group.
 // N = 16 x 32 x 32, index n = nA*1024 + nB*32 + nC; three in-place passes
 // (16-point over nA, 32-point over nB, 32-point over nC) with the inter-pass
 // twiddles of the four-step decomposition.  The forward passes are
@@ -24,6 +30,7 @@
 // product and the first inverse pass run back to back in registers.
 #pragma once
 
+#include <cooperative_groups.h>
 #include <stdint.h>
 
 namespace ccv {
@@ -33,6 +40,7 @@ constexpr int kNttN = 16384;
 constexpr int64_t kNttMaxL = kNttN / 2;
 constexpr int kNttThreads = 512;
 constexpr int kNttWordsPerArray = kNttN + kNttN / 32;
+constexpr int kNttGroup = 4;  // channels per cluster (4 x 4 bytes per time step)
 constexpr size_t kNttSmemBytes = 2u * kNttWordsPerArray * 4u;
 
 struct NttParams {
@@ -153,32 +161,87 @@ __device__ __forceinline__ void ntt_dit_inv(uint32_t (&x)[R]) {
 
 __device__ __forceinline__ int pad_idx(int s) { return s + (s >> 5); }
 
-// One CTA per (b, d) row.  smem: V[N + N/32], G[N + N/32] (padded words).
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t x) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;\n" ::"r"(addr), "r"(x) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
+    uint32_t x;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];\n" : "=r"(x) : "r"(addr) : "memory");
+    return x;
+}
+
+// One CTA per (b, d) row, kNttGroup rows per cluster.  smem: V[N + N/32],
+// G[N + N/32] (padded words).  vec_ok: 16-byte group accesses are aligned.
 __global__ void __launch_bounds__(kNttThreads, 1)
     ntt_conv_kernel(const int32_t *__restrict__ v, const int32_t *__restrict__ g, int32_t *__restrict__ r, int L,
-                    int D) {
+                    int D, int groups_per_batch, int vec_ok) {
     extern __shared__ uint32_t nsm[];
     uint32_t *sv = nsm;
     uint32_t *sg = nsm + kNttWordsPerArray;
     const int tid = threadIdx.x;
-    const int b = blockIdx.x / D, d = blockIdx.x - b * D;
-    const int64_t base = (int64_t)b * L * D + d;
+    cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    const int grp = blockIdx.x / kNttGroup;
+    const int b = grp / groups_per_batch, d0 = (grp - b * groups_per_batch) * kNttGroup;
+    const int nch = min(kNttGroup, D - d0);
+    const bool vec = vec_ok && nch == kNttGroup;
+    const int64_t gbase = (int64_t)b * L * D + d0;  // element (b, 0, d0)
+    const uint32_t sv_addr = (uint32_t)__cvta_generic_to_shared(sv);
+    const uint32_t sg_addr = (uint32_t)__cvta_generic_to_shared(sg);
+    cluster.sync();  // every CTA of the cluster runs before the first remote store
 
-    // F1: 16-point DIF over nA for each n2 (inputs with nA >= 8 are padding zeros)
+    // Load: residues of time steps [t0, t0 + TC) of the group, zeros past L,
+    // into slot t of each channel's CTA
+    {
+        constexpr int TC = (int)kNttMaxL / kNttGroup;
+        const int t0 = rank * TC;
+        uint32_t dv[kNttGroup], dg[kNttGroup];
+#pragma unroll
+        for (int c = 0; c < kNttGroup; ++c) {
+            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(dv[c]) : "r"(sv_addr), "r"(c));
+            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(dg[c]) : "r"(sg_addr), "r"(c));
+        }
+#pragma unroll 2
+        for (int t = t0 + tid; t < t0 + TC; t += kNttThreads) {
+            int32_t a[kNttGroup] = {0, 0, 0, 0}, q[kNttGroup] = {0, 0, 0, 0};
+            if (t < L) {
+                const int32_t *pv = v + gbase + (int64_t)t * D;
+                const int32_t *pg = g + gbase + (int64_t)t * D;
+                if (vec) {
+                    const int4 x = __ldg(reinterpret_cast<const int4 *>(pv));
+                    const int4 y = __ldg(reinterpret_cast<const int4 *>(pg));
+                    a[0] = x.x; a[1] = x.y; a[2] = x.z; a[3] = x.w;
+                    q[0] = y.x; q[1] = y.y; q[2] = y.z; q[3] = y.w;
+                } else {
+#pragma unroll
+                    for (int c = 0; c < kNttGroup; ++c)
+                        if (c < nch) {
+                            a[c] = __ldg(pv + c);
+                            q[c] = __ldg(pg + c);
+                        }
+                }
+            }
+            const uint32_t off = 4u * (uint32_t)pad_idx(t);
+#pragma unroll
+            for (int c = 0; c < kNttGroup; ++c) {
+                st_cluster_u32(dv[c] + off, n_from_int(a[c]));
+                st_cluster_u32(dg[c] + off, n_from_int(q[c]));
+            }
+        }
+    }
+    cluster.sync();
+
+    // F1: 16-point DIF over nA for each n2 (inputs with nA >= 8 are padding
+    // zeros); column n2 is read (slots of t = nA 1024 + n2) and rewritten in place
 #pragma unroll 1
     for (int rep = 0; rep < 2; ++rep) {
         const int n2 = tid + rep * kNttThreads;
         uint32_t xv[16], xg[16];
 #pragma unroll
         for (int nA = 0; nA < 16; ++nA) {
-            const int t = nA * 1024 + n2;
-            uint32_t a = 0, q = 0;
-            if (nA < 8 && t < L) {
-                a = n_from_int(__ldg(v + base + (int64_t)t * D));
-                q = n_from_int(__ldg(g + base + (int64_t)t * D));
-            }
-            xv[nA] = a;
-            xg[nA] = q;
+            const int s = pad_idx(nA * 1024 + n2);
+            xv[nA] = nA < 8 ? sv[s] : 0u;
+            xg[nA] = nA < 8 ? sg[s] : 0u;
         }
         ntt_dif<16, 8>(xv);
         ntt_dif<16, 8>(xg);
@@ -247,7 +310,8 @@ __global__ void __launch_bounds__(kNttThreads, 1)
     }
     __syncthreads();
 
-    // I1: twiddle, inverse 16-point DIT over the nA slots keeping nA < 8, scale, lift, store
+    // I1: twiddle, inverse 16-point DIT over the nA slots keeping nA < 8,
+    // scale, lift; r_t is left in slot t of the same column
     const uint32_t sc = c_nscale, scs = c_nscale_s;
 #pragma unroll 1
     for (int rep = 0; rep < 2; ++rep) {
@@ -261,11 +325,36 @@ __global__ void __launch_bounds__(kNttThreads, 1)
         }
         ntt_dit_inv<16, 8>(x);
 #pragma unroll
-        for (int nA = 0; nA < 8; ++nA) {
-            const int t = nA * 1024 + n2;
-            if (t < L) r[base + (int64_t)t * D] = n_centered(n_mul_shoup(x[nA], sc, scs));
+        for (int nA = 0; nA < 8; ++nA)
+            sv[pad_idx(nA * 1024 + n2)] = (uint32_t)n_centered(n_mul_shoup(x[nA], sc, scs));
+    }
+    cluster.sync();
+
+    // Store: time steps [t0, t1) of the group, gathered from the channels' CTAs
+    {
+        const int TS = (L + kNttGroup - 1) / kNttGroup;
+        const int t0 = rank * TS, t1 = min(L, t0 + TS);
+        uint32_t src[kNttGroup];
+#pragma unroll
+        for (int c = 0; c < kNttGroup; ++c)
+            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(src[c]) : "r"(sv_addr), "r"(c));
+#pragma unroll 2
+        for (int t = t0 + tid; t < t1; t += kNttThreads) {
+            const uint32_t off = 4u * (uint32_t)pad_idx(t);
+            uint32_t o[kNttGroup];
+#pragma unroll
+            for (int c = 0; c < kNttGroup; ++c) o[c] = ld_cluster_u32(src[c] + off);
+            int32_t *pr = r + gbase + (int64_t)t * D;
+            if (vec) {
+                *reinterpret_cast<int4 *>(pr) = make_int4((int)o[0], (int)o[1], (int)o[2], (int)o[3]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < kNttGroup; ++c)
+                    if (c < nch) pr[c] = (int32_t)o[c];
+            }
         }
     }
+    cluster.sync();  // remote reads of this CTA's slots are done before it exits
 }
 
 static inline uint32_t h_bitrev(uint32_t x, int bits) {
@@ -322,10 +411,26 @@ static cudaError_t ntt_init_device() {
 static int ntt_dispatch(const int32_t *v, const int32_t *g, int32_t *r, int64_t B, int64_t L, int64_t D,
                         cudaStream_t s) {
     if (L > kNttMaxL) return 2;  // CC_ERR_UNSUPPORTED
-    const int64_t blocks = B * D;
-    if (blocks > INT32_MAX) return 2;
-    ntt_conv_kernel<<<(unsigned)blocks, kNttThreads, kNttSmemBytes, s>>>(v, g, r, (int)L, (int)D);
-    return cudaGetLastError() == cudaSuccess ? 0 : 5;  // CC_OK / CC_ERR_CUDA
+    const int64_t gpb = (D + kNttGroup - 1) / kNttGroup;
+    if (B * gpb * kNttGroup > INT32_MAX) return 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(B * gpb * kNttGroup));
+    cfg.blockDim = dim3(kNttThreads);
+    cfg.dynamicSmemBytes = kNttSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kNttGroup;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int vec = (D % 4) == 0 && ((uintptr_t)v % 16) == 0 && ((uintptr_t)g % 16) == 0 && ((uintptr_t)r % 16) == 0;
+    if (cudaLaunchKernelEx(&cfg, ntt_conv_kernel, v, g, r, (int)L, (int)D, (int)gpb, vec) != cudaSuccess) {
+        cudaGetLastError();
+        return 5;  // CC_ERR_CUDA
+    }
+    return 0;  // CC_OK
 }
 
 }  // namespace ccv

@@ -85,7 +85,10 @@ def test_no_kernel_wait_ran_out():
     assert ssm.fault_flags() == 0
 
 
-INT_SHAPES = [(1, 1, 1), (1, 2, 3), (2, 33, 5), (2, 1000, 37), (1, 4097, 3), (1, 8192, 2)]
+# clusters of 4 adjacent channels: partial groups, and whole groups with
+# 16-byte accesses (D = 8, 12)
+INT_SHAPES = [(1, 1, 1), (1, 2, 3), (2, 33, 5), (2, 1000, 37), (1, 4097, 3), (1, 8192, 2), (2, 1000, 8),
+              (1, 8192, 12), (3, 500, 6)]
 
 
 @pytest.mark.parametrize("shape", INT_SHAPES, ids=lambda s: "x".join(map(str, s)))
