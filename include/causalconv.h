@@ -206,6 +206,23 @@ CC_API int causal_conv_from_host(int dtype, const void *v_host, const void *g_ho
                           int64_t B, int64_t L, int64_t D,
                           void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * causal_conv_fast_workspace_bytes -- optional workspace for rows longer than
+ * one CTA holds (4096 < L <= 65536, float paths).  Such a row is transformed
+ * by a cluster of 8 CTAs; read straight from a channel-last [B, L, D] tensor
+ * its time steps are D elements apart.  When causal_fftconv_f32/bf16 and the
+ * backward entry points receive a workspace of at least this many bytes they
+ * take a two-pass path instead: v and g are transposed to [B, D, L] in the
+ * workspace (rows contiguous), the rows are transformed from there, and r is
+ * transposed back (three [B, L, D] arrays, each 256-byte aligned).  The result
+ * is the same convolution computed in the same order; the workspace must not
+ * overlap any tensor of the call (CC_ERR_ALIAS).  A smaller workspace (or
+ * none) selects the single-pass path.  Returns 0 when no such path applies
+ * (L <= 4096, the NTT path, B > 65535) and for invalid arguments.  The pages
+ * have no counterpart; it is a layout choice of this library.
+ */
+CC_API size_t causal_conv_fast_workspace_bytes(int dtype, int64_t B, int64_t L, int64_t D);
+
 /* Device workspace bytes the conv entry points need for this problem (0 when
  * no scratch is needed).  Returns (size_t)-1 for an invalid dtype/shape. */
 CC_API size_t causal_conv_workspace_bytes(int dtype, int64_t B, int64_t L, int64_t D);

@@ -23,7 +23,8 @@ from ._lib import (CC_DTYPE_BF16, CC_DTYPE_F32, CC_DTYPE_I32, CausalConvError, l
 __all__ = [
     "causal_fftconv_f32", "causal_fftconv_bf16", "causal_ntt_conv_i32", "causal_conv", "causal_conv_bwd",
     "causal_conv_decode", "decode_workspace_bytes",
-    "causal_conv_from_host", "workspace_bytes", "max_len", "ntt_params", "strerror", "fault_flags",
+    "causal_conv_from_host", "workspace_bytes", "fast_workspace_bytes", "max_len", "ntt_params", "strerror",
+    "fault_flags",
     "CausalConvError", "CC_DTYPE_F32", "CC_DTYPE_BF16", "CC_DTYPE_I32",
 ]
 
@@ -50,6 +51,25 @@ def _stream_ptr(stream) -> int:
     return int(stream.cuda_stream)
 
 
+def fast_workspace_bytes(dtype: torch.dtype, B: int, L: int, D: int) -> int:
+    """Bytes of the optional workspace that lets long rows (4096 < L <= 65536)
+    take the two-pass path with contiguous rows; 0 where it does not apply."""
+    return int(load().causal_conv_fast_workspace_bytes(_DT[dtype], B, L, D))
+
+
+def _workspace(workspace, dtype_code: int, B: int, L: int, D: int, device):
+    """(pointer, bytes) of the caller's workspace; with none given, one of the
+    optional two-pass size is taken from the torch allocator when that path
+    applies.  A tensor of 0 bytes selects the single-pass path."""
+    if workspace is None:
+        n = int(load().causal_conv_fast_workspace_bytes(dtype_code, B, L, D))
+        if n == 0:
+            return None, 0
+        workspace = torch.empty(n, dtype=torch.uint8, device=device)
+    nbytes = workspace.numel() * workspace.element_size()
+    return (workspace.data_ptr() if nbytes else None), nbytes
+
+
 def _run(dtype_code: int, v: torch.Tensor, g: torch.Tensor, out, workspace, stream):
     dtype = v.dtype
     _check(v, "v", dtype)
@@ -60,9 +80,7 @@ def _run(dtype_code: int, v: torch.Tensor, g: torch.Tensor, out, workspace, stre
     if out is None:
         out = torch.empty_like(v)
     _check(out, "out", dtype, v.shape)
-    ws_ptr, ws_bytes = None, 0
-    if workspace is not None:
-        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    ws_ptr, ws_bytes = _workspace(workspace, dtype_code, B, L, D, v.device)
     with torch.cuda.device(v.device):
         st = getattr(load(), _FN[dtype_code])(v.data_ptr(), g.data_ptr(), out.data_ptr(), B, L, D, ws_ptr, ws_bytes,
                                               _stream_ptr(stream))
@@ -113,9 +131,7 @@ def causal_conv_bwd(dr: torch.Tensor, v: torch.Tensor, g: torch.Tensor, dv=None,
     _check(dv, "dv", dtype, v.shape)
     _check(dg, "dg", dtype, v.shape)
     B, L, D = v.shape
-    ws_ptr, ws_bytes = None, 0
-    if workspace is not None:
-        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    ws_ptr, ws_bytes = _workspace(workspace, _DT[dtype], B, L, D, v.device)
     fn = "causal_fftconv_bwd_f32" if dtype == torch.float32 else "causal_fftconv_bwd_bf16"
     with torch.cuda.device(v.device):
         st = getattr(load(), fn)(dr.data_ptr(), v.data_ptr(), g.data_ptr(), dv.data_ptr(), dg.data_ptr(), B, L, D,
@@ -169,9 +185,7 @@ def causal_conv_from_host(v_host: torch.Tensor, g_host: torch.Tensor, r_host: to
     if v_host.is_cuda or g_host.is_cuda or r_host.is_cuda:
         raise ValueError("*_host tensors must live in host memory")
     B, L, D = v_host.shape
-    ws_ptr, ws_bytes = None, 0
-    if workspace is not None:
-        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    ws_ptr, ws_bytes = _workspace(workspace, _DT[dtype], B, L, D, v_dev.device)
     with torch.cuda.device(v_dev.device):
         st = load().causal_conv_from_host(_DT[dtype], v_host.data_ptr(), g_host.data_ptr(), r_host.data_ptr(),
                                           v_dev.data_ptr(), g_dev.data_ptr(), r_dev.data_ptr(), B, L, D, ws_ptr,

@@ -31,6 +31,7 @@ SIGNATURES = {
     "causal_conv_decode_f32_noalloc": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _I64, _P]),
     "causal_conv_from_host": (ctypes.c_int, [ctypes.c_int, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "causal_conv_workspace_bytes": (_SZ, [ctypes.c_int, _I64, _I64, _I64]),
+    "causal_conv_fast_workspace_bytes": (_SZ, [ctypes.c_int, _I64, _I64, _I64]),
     "causal_conv_max_len": (_I64, [ctypes.c_int]),
     "causal_conv_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "causal_ntt_params": (ctypes.c_int, [_I64, ctypes.POINTER(ctypes.c_uint32)]),

@@ -13,6 +13,7 @@
 #include <algorithm>
 #include <initializer_list>
 #include <mutex>
+#include <type_traits>
 #include <vector>
 
 #include "causalconv.h"
@@ -20,6 +21,7 @@
 #include "bigconv.cuh"
 #include "ntt.cuh"
 #include "decode.cuh"
+#include "transpose.cuh"
 
 namespace ccv {
 
@@ -308,7 +310,7 @@ static int launch_fused(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, i
 
 template <class Cfg, int MINB, typename IO>
 static int launch_big(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, const float2 *tw,
-                      cudaStream_t s, int rev) {
+                      cudaStream_t s, int rev, int row_major) {
     const int64_t rows = B * D;
     if (rows * Cfg::CL > INT32_MAX) return CC_ERR_UNSUPPORTED;
     auto kern = bigconv_kernel<Cfg::R0, Cfg::RA, Cfg::RB, Cfg::RC, Cfg::CL, Cfg::T, MINB, IO>;
@@ -324,12 +326,38 @@ static int launch_big(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, v, g, r, (int)L, (int)D, rev, tw);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, v, g, r, (int)L, (int)D, rev, row_major, tw);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return CC_ERR_CUDA;
     }
     return CC_OK;
+}
+
+// Workspace that enables the two-pass path of rows longer than one CTA holds
+// (three [B, L, D] arrays: v and g with rows made contiguous, and r before
+// its transpose back); 0 when that path does not apply.
+static size_t fast_ws_bytes(int dtype, int64_t B, int64_t L, int64_t D) {
+    if (dtype != CC_DTYPE_F32 && dtype != CC_DTYPE_BF16) return 0;
+    if (B < 1 || D < 1 || L <= BigL<float>::LMAX || L > BigX<float>::LMAX) return 0;
+    if (B > 65535 || (L + kTrTile - 1) / kTrTile > 65535 || (D + kTrTile - 1) / kTrTile > 65535) return 0;
+    const int64_t es = dtype == CC_DTYPE_F32 ? 4 : 2;
+    if (D > INT64_MAX / (16 * L * es) / B) return 0;
+    const size_t one = ((size_t)(B * L * D * es) + 255) / 256 * 256;
+    return 3 * one;
+}
+
+// A workspace large enough for the two-pass path is used by it: it must be
+// device memory of the current device and overlap none of the tensors.
+static int check_fast_ws(int dtype, int64_t B, int64_t L, int64_t D, const void *ws, size_t ws_bytes,
+                         std::initializer_list<const void *> tensors) {
+    const size_t fast = fast_ws_bytes(dtype, B, L, D);
+    if (!ws || fast == 0 || ws_bytes < fast) return CC_OK;
+    const size_t bytes = (size_t)(B * L * D) * dtype_size(dtype);
+    for (const void *t : tensors)
+        if (ranges_overlap(ws, fast, t, bytes)) return CC_ERR_ALIAS;
+    int dev;
+    return check_device({ws}, &dev);
 }
 
 // Rows that fit one CTA, kGroup adjacent channels per cluster.
@@ -365,8 +393,8 @@ static int launch_group(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, i
 }
 
 template <typename IO>
-static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, cudaStream_t s,
-                            int dev, int rev = 0) {
+static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, void *ws,
+                            size_t ws_bytes, cudaStream_t s, int dev, int rev = 0) {
     void *tw = nullptr;
     if (L <= CfgS<IO>::LMAX) {
         if (cudaGetSymbolAddress(&tw, g_tw_s) != cudaSuccess) return CC_ERR_CUDA;
@@ -382,7 +410,21 @@ static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t 
     }
     if (L <= BigX<IO>::LMAX) {
         if (cudaGetSymbolAddress(&tw, g_tw_bx) != cudaSuccess) return CC_ERR_CUDA;
-        return launch_big<BigX<IO>, kMinbBigX>(v, g, r, B, L, D, (const float2 *)tw, s, rev);
+        const size_t fast = fast_ws_bytes(sizeof(IO) == 4 ? CC_DTYPE_F32 : CC_DTYPE_BF16, B, L, D);
+        if (ws == nullptr || fast == 0 || ws_bytes < fast)
+            return launch_big<BigX<IO>, kMinbBigX>(v, g, r, B, L, D, (const float2 *)tw, s, rev, 0);
+        // two-pass path: rows made contiguous in the workspace, transformed, transposed back
+        typedef typename std::conditional<sizeof(IO) == 4, uint32_t, uint16_t>::type W;
+        const size_t one = fast / 3;
+        IO *vt = reinterpret_cast<IO *>(ws);
+        IO *gt = reinterpret_cast<IO *>(reinterpret_cast<char *>(ws) + one);
+        IO *rt = reinterpret_cast<IO *>(reinterpret_cast<char *>(ws) + 2 * one);
+        int st;
+        if ((st = transpose_last2<W>((const W *)v, (W *)vt, B, L, D, s)) != CC_OK) return st;
+        if ((st = transpose_last2<W>((const W *)g, (W *)gt, B, L, D, s)) != CC_OK) return st;
+        if ((st = launch_big<BigX<IO>, kMinbBigX>(vt, gt, rt, B, L, D, (const float2 *)tw, s, rev, 1)) != CC_OK)
+            return st;
+        return transpose_last2<W>((const W *)rt, (W *)r, B, D, L, s);
     }
     return CC_ERR_UNSUPPORTED;
 }
@@ -390,10 +432,10 @@ static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t 
 // Backward: dv = rev(conv(rev(dr), g)), dg = rev(conv(rev(dr), v)).
 template <typename IO>
 static int fftconv_bwd(const IO *dr, const IO *v, const IO *g, IO *dv, IO *dg, int64_t B, int64_t L, int64_t D,
-                       cudaStream_t s, int dev) {
-    int st = fftconv_dispatch<IO>(dr, g, dv, B, L, D, s, dev, 3);
+                       void *ws, size_t ws_bytes, cudaStream_t s, int dev) {
+    int st = fftconv_dispatch<IO>(dr, g, dv, B, L, D, ws, ws_bytes, s, dev, 3);
     if (st != CC_OK) return st;
-    return fftconv_dispatch<IO>(dr, v, dg, B, L, D, s, dev, 3);
+    return fftconv_dispatch<IO>(dr, v, dg, B, L, D, ws, ws_bytes, s, dev, 3);
 }
 
 static int check_bwd(int dtype, const void *dr, const void *v, const void *g, const void *dv, const void *dg,
@@ -494,23 +536,23 @@ const char *causal_conv_strerror(int status) {
 
 int causal_fftconv_f32(const float *v, const float *g, float *r, int64_t B, int64_t L, int64_t D, void *workspace,
                        size_t workspace_bytes, void *stream) {
-    (void)workspace;
     int dev;
     int st = check_common(CC_DTYPE_F32, v, g, r, B, L, D, workspace_bytes, &dev);
     if (st != CC_OK) return st;
+    if ((st = check_fast_ws(CC_DTYPE_F32, B, L, D, workspace, workspace_bytes, {v, g, r})) != CC_OK) return st;
     if (ensure_init(dev) != cudaSuccess) return CC_ERR_CUDA;
-    return fftconv_dispatch<float>(v, g, r, B, L, D, (cudaStream_t)stream, dev);
+    return fftconv_dispatch<float>(v, g, r, B, L, D, workspace, workspace_bytes, (cudaStream_t)stream, dev);
 }
 
 int causal_fftconv_bf16(const uint16_t *v, const uint16_t *g, uint16_t *r, int64_t B, int64_t L, int64_t D,
                         void *workspace, size_t workspace_bytes, void *stream) {
-    (void)workspace;
     int dev;
     int st = check_common(CC_DTYPE_BF16, v, g, r, B, L, D, workspace_bytes, &dev);
     if (st != CC_OK) return st;
+    if ((st = check_fast_ws(CC_DTYPE_BF16, B, L, D, workspace, workspace_bytes, {v, g, r})) != CC_OK) return st;
     if (ensure_init(dev) != cudaSuccess) return CC_ERR_CUDA;
     return fftconv_dispatch<__nv_bfloat16>((const __nv_bfloat16 *)v, (const __nv_bfloat16 *)g, (__nv_bfloat16 *)r, B,
-                                           L, D, (cudaStream_t)stream, dev);
+                                           L, D, workspace, workspace_bytes, (cudaStream_t)stream, dev);
 }
 
 int causal_ntt_conv_i32(const int32_t *v, const int32_t *g, int32_t *r, int64_t B, int64_t L, int64_t D,
@@ -525,24 +567,30 @@ int causal_ntt_conv_i32(const int32_t *v, const int32_t *g, int32_t *r, int64_t 
 
 int causal_fftconv_bwd_f32(const float *dr, const float *v, const float *g, float *dv, float *dg, int64_t B,
                            int64_t L, int64_t D, void *workspace, size_t workspace_bytes, void *stream) {
-    (void)workspace;
     int dev;
     int st = check_bwd(CC_DTYPE_F32, dr, v, g, dv, dg, B, L, D, workspace_bytes, &dev);
     if (st != CC_OK) return st;
+    if ((st = check_fast_ws(CC_DTYPE_F32, B, L, D, workspace, workspace_bytes, {dr, v, g, dv, dg})) != CC_OK)
+        return st;
     if (ensure_init(dev) != cudaSuccess) return CC_ERR_CUDA;
-    return fftconv_bwd<float>(dr, v, g, dv, dg, B, L, D, (cudaStream_t)stream, dev);
+    return fftconv_bwd<float>(dr, v, g, dv, dg, B, L, D, workspace, workspace_bytes, (cudaStream_t)stream, dev);
 }
 
 int causal_fftconv_bwd_bf16(const uint16_t *dr, const uint16_t *v, const uint16_t *g, uint16_t *dv, uint16_t *dg,
                             int64_t B, int64_t L, int64_t D, void *workspace, size_t workspace_bytes, void *stream) {
-    (void)workspace;
     int dev;
     int st = check_bwd(CC_DTYPE_BF16, dr, v, g, dv, dg, B, L, D, workspace_bytes, &dev);
     if (st != CC_OK) return st;
+    if ((st = check_fast_ws(CC_DTYPE_BF16, B, L, D, workspace, workspace_bytes, {dr, v, g, dv, dg})) != CC_OK)
+        return st;
     if (ensure_init(dev) != cudaSuccess) return CC_ERR_CUDA;
     typedef __nv_bfloat16 bf;
-    return fftconv_bwd<bf>((const bf *)dr, (const bf *)v, (const bf *)g, (bf *)dv, (bf *)dg, B, L, D,
-                           (cudaStream_t)stream, dev);
+    return fftconv_bwd<bf>((const bf *)dr, (const bf *)v, (const bf *)g, (bf *)dv, (bf *)dg, B, L, D, workspace,
+                           workspace_bytes, (cudaStream_t)stream, dev);
+}
+
+size_t causal_conv_fast_workspace_bytes(int dtype, int64_t B, int64_t L, int64_t D) {
+    return fast_ws_bytes(dtype, B, L, D);
 }
 
 size_t causal_conv_decode_workspace_bytes(int dtype, int64_t B, int64_t D, int64_t t) {

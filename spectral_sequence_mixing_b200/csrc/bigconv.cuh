@@ -149,8 +149,10 @@ __device__ __forceinline__ void bc_local_pass(float2 *xs, const float2 *__restri
 template <int R0, int RA, int RB, int RC, int CL, int T, int MINB, typename IO>
 __global__ void __launch_bounds__(T, MINB)
     bigconv_kernel(const IO *__restrict__ v, const IO *__restrict__ g, IO *__restrict__ r, int L, int D, int rev,
-                   const float2 *__restrict__ tw) {
-    // rev bit 0: read v reversed in time; bit 1: write r reversed
+                   int row_major, const float2 *__restrict__ tw) {
+    // rev bit 0: read v reversed in time; bit 1: write r reversed.
+    // row_major: v, g, r are [B, D, L] (each row contiguous) instead of
+    // channel-last [B, L, D].
     using C = BigCfg<R0, RA, RB, RC, CL, T, IO>;
     constexpr int S = C::S, SL = C::SL, SC = C::SC, HEAD = C::HEAD;
     constexpr int LOG_R0 = ilog2(R0);
@@ -162,7 +164,9 @@ __global__ void __launch_bounds__(T, MINB)
     if constexpr (CL > 1) rank = (int)cg::this_cluster().block_rank();
     const int row = blockIdx.x / CL;
     const int b = row / D, d = row - b * D;
-    const int64_t base = (int64_t)b * L * D + d;
+    // element (row, t) sits at base + t * tstep
+    const int64_t base = row_major ? (int64_t)row * L : (int64_t)b * L * D + d;
+    const int64_t tstep = row_major ? 1 : D;
 
     auto cluster_sync = [&]() {
         if constexpr (CL > 1)
@@ -212,8 +216,8 @@ __global__ void __launch_bounds__(T, MINB)
         for (int n0 = 0; n0 < R0 / 2; ++n0) {
             const int t = n0 * SL + n;
             float2 z = make_float2(0.f, 0.f);
-            if (t < L) z = make_float2(IO_t<IO>::cvt(IO_t<IO>::ld(v + base + (int64_t)((rev & 1) ? L - 1 - t : t) * D)),
-                                       IO_t<IO>::cvt(IO_t<IO>::ld(g + base + (int64_t)t * D)));
+            if (t < L) z = make_float2(IO_t<IO>::cvt(IO_t<IO>::ld(v + base + (int64_t)((rev & 1) ? L - 1 - t : t) * tstep)),
+                                       IO_t<IO>::cvt(IO_t<IO>::ld(g + base + (int64_t)t * tstep)));
             if (t < HEAD) head[t] = z;
             zin[p][n0] = z;
             nv = fmaf(z.x, z.x, nv);
@@ -334,7 +338,7 @@ __global__ void __launch_bounds__(T, MINB)
                     for (int j = 0; j <= t; ++j) a = fmaf(head[j].x, head[t - j].y, a);
                     out = a;
                 }
-                IO_t<IO>::st(r + base + (int64_t)((rev & 2) ? L - 1 - t : t) * D, out);
+                IO_t<IO>::st(r + base + (int64_t)((rev & 2) ? L - 1 - t : t) * tstep, out);
             }
         }
     }

@@ -161,3 +161,15 @@ def test_fault_flags_host_checks(lib):
     assert lib.causal_conv_fault_flags(0, None, 0) == 1                      # NULL flags
     out = ctypes.c_uint(7)
     assert lib.causal_conv_fault_flags(-1, ctypes.byref(out), 0) == 1       # bad device
+
+
+def test_fast_workspace_bytes(lib):
+    f = lib.causal_conv_fast_workspace_bytes
+    assert f(0, 1, 4096, 8) == 0                       # rows of one CTA: no two-pass path
+    one = (4097 * 8 * 4 + 255) // 256 * 256
+    assert f(0, 1, 4097, 8) == 3 * one                  # fp32: three [B, L, D] arrays, 256-byte aligned
+    assert f(1, 2, 65536, 16) == 3 * (2 * 65536 * 16 * 2)
+    assert f(2, 1, 5000, 8) == 0                       # NTT path
+    assert f(0, 1, 65537, 8) == 0                      # beyond the longest row
+    assert f(0, 70000, 5000, 8) == 0                   # B beyond the transpose grid
+    assert f(0, 1, 5000, 0) == 0 and f(7, 1, 5000, 8) == 0

@@ -77,6 +77,21 @@ def test_unaligned_base_pointers(dtype, shape):
     assert n_bad == 0, f"{n_bad} elements beyond the bound, worst ratio {worst:.3g}"
 
 
+def test_fast_workspace_must_not_overlap_tensors():
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    from spectral_sequence_mixing_b200._lib import CausalConvError
+    B, L, D = 1, 5000, 4
+    v = torch.randn(B, L, D, device="cuda")
+    g = torch.randn(B, L, D, device="cuda")
+    n = ssm.fast_workspace_bytes(torch.float32, B, L, D)
+    big = torch.empty(n + v.numel() * 4, dtype=torch.uint8, device="cuda")
+    out = big[:v.numel() * 4].view(torch.float32).view(B, L, D)  # r inside the workspace
+    with pytest.raises(CausalConvError) as e:
+        ssm.causal_conv(v, g, out=out, workspace=big)
+    assert e.value.status == 3
+
+
 def test_no_kernel_wait_ran_out():
     """Every bounded wait in the kernels completed during the tests so far."""
     import spectral_sequence_mixing_b200 as ssm
@@ -155,16 +170,26 @@ def test_big_rows_full_oracle(shape, dtype):
     assert n_bad == 0, f"{n_bad} violations, worst ratio {worst:.3g}"
 
 
-CLUSTER_SHAPES = [(1, 4097, 3), (2, 20000, 2), (1, 65536, 2)]
+CLUSTER_SHAPES = [(1, 4097, 3), (2, 20000, 2), (1, 65536, 2), (2, 5000, 33)]
 
 
+@pytest.mark.parametrize("two_pass", [True, False], ids=["two_pass", "single_pass"])
 @pytest.mark.parametrize("shape", CLUSTER_SHAPES, ids=lambda s: "x".join(map(str, s)))
-def test_cluster_rows_sampled_oracle(shape):
+def test_cluster_rows_sampled_oracle(shape, two_pass):
+    """Rows beyond one CTA: with the optional workspace (transposed rows) and
+    without it (rows read straight from the channel-last tensors)."""
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
     B, L, D = shape
     rng = np.random.Generator(np.random.PCG64(sum(shape)))
     v = rng.standard_normal(shape).astype(np.float32)
     g = (rng.standard_normal(shape) * (1.0 + np.arange(L).reshape(1, L, 1)) ** -0.75).astype(np.float32)
-    r = run_gpu(v, g, "f32")
+    n_ws = ssm.fast_workspace_bytes(torch.float32, B, L, D) if two_pass else 0
+    assert (n_ws > 0) == two_pass
+    ws = torch.empty(n_ws, dtype=torch.uint8, device="cuda")
+    r = ssm.causal_conv(to_dev(v, "f32"), to_dev(g, "f32"), workspace=ws)
+    torch.cuda.synchronize()
+    r = from_dev(r, "f32")
     pts = workloads.sample_points(B, L, D, 1024, seed=7)
     r_ref, den = oracle.causal_conv_points(v, g, pts)
     n_bad, worst = float_violations(r[pts[:, 0], pts[:, 1], pts[:, 2]], r_ref, den, F32_TOL)
