@@ -37,7 +37,7 @@ import workloads  # noqa: E402
 
 METRIC = "causal FFT-conv GB/s and (B*D*L)/s at 1 B200; % of HBM roofline"
 L2_BYTES = 126 * 2 ** 20
-KERNEL_SOURCES = ["fftconv_fused.cuh", "fft_reg.cuh", "bigconv.cuh", "ntt.cuh", "api.cu"]
+KERNEL_SOURCES = ["fftconv_fused.cuh", "fft_reg.cuh", "tma.cuh", "bigconv.cuh", "ntt.cuh", "transpose.cuh", "api.cu"]
 
 
 def parse_args():
@@ -356,7 +356,14 @@ def run_ours(args, rank, world, local):
     _, e2e_gbs = throughput(w.units, world, e2e_steps, ems, 3 * w.elem_bytes)
 
     peak, peak_src = measured_peaks()
-    kernel = "ntt_conv_kernel" if w.dtype == "i32" else ("fftconv_fused_kernel" if w.L <= 1024 else "bigconv_kernel")
+    if w.dtype == "i32":
+        kernel = "ntt_conv_kernel"
+    elif w.L <= 1024:
+        kernel = "fftconv_fused_kernel"
+    elif w.L <= 4096:
+        kernel = "bigrow_group_kernel"
+    else:
+        kernel = "bigconv_kernel"
     if args.path == "decode":
         kernel = "decode_partial_kernel"
     if n_ws and args.path != "decode":

@@ -12,8 +12,9 @@
 //
 // Layout: caches [B, Lcap, D] channel-last; output [B, D].  Work is split
 // over j into `splits` ranges so the whole GPU streams the caches: kernel 1
-// writes fp64 partial sums part[split][b][d] (caller's workspace), kernel 2
-// adds them in a fixed order and rounds once.  Accumulating in fp64 keeps the
+// (each thread four adjacent channels, one 16-byte fp32 or 8-byte bf16
+// access per cache row) writes fp64 partial sums part[split][b][d] (caller's
+// workspace), kernel 2 adds them in a fixed order and rounds once.  Accumulating in fp64 keeps the
 // result within one fp32 rounding of the exact sum and makes it
 // deterministic.
 #pragma once
@@ -24,56 +25,88 @@
 
 namespace ccv {
 
-constexpr int kDecodeThreads = 256;
-constexpr int kDecodeUnroll = 4;
+constexpr int kDecodeThreads = 64;   // partial kernel: 64 threads x 4 channels per CTA
+constexpr int kDecodeVec = 4;        // channels per thread (one 16-byte fp32 / 8-byte bf16 access)
+constexpr int kReduceThreads = 256;
+constexpr int kDecodeUnroll = 8;
 
-// Number of j-ranges for a decode call: aim at ~1024 CTAs of 256 channels,
-// at least 64 positions per range, at most 64 ranges.  Depends only on the
-// problem (so the workspace size is host-computable).
+// Number of j-ranges for a decode call: aim at ~1184 CTAs (8 per SM of a
+// 148-SM part) of 256 channels, at least 16 positions per range, at most 128
+// ranges.  Depends only on the problem (so the workspace size is
+// host-computable).
 static inline int decode_splits(int64_t B, int64_t D, int64_t t) {
-    const int64_t ctas = B * ((D + kDecodeThreads - 1) / kDecodeThreads);
-    int64_t s = (1024 + ctas - 1) / ctas;
-    const int64_t max_by_len = (t + 1 + 63) / 64;
+    const int64_t ctas = B * ((D + kDecodeThreads * kDecodeVec - 1) / (kDecodeThreads * kDecodeVec));
+    int64_t s = (1184 + ctas - 1) / ctas;
+    const int64_t max_by_len = (t + 1 + 15) / 16;
     if (s > max_by_len) s = max_by_len;
-    if (s > 64) s = 64;
+    if (s > 128) s = 128;
     if (s < 1) s = 1;
     return (int)s;
 }
 
+// kDecodeVec consecutive channels starting at p (aligned for one access).
+__device__ __forceinline__ void decode_ld4(const float *p, float (&o)[kDecodeVec]) {
+    const float4 x = __ldg(reinterpret_cast<const float4 *>(p));
+    o[0] = x.x;
+    o[1] = x.y;
+    o[2] = x.z;
+    o[3] = x.w;
+}
+__device__ __forceinline__ void decode_ld4(const __nv_bfloat16 *p, float (&o)[kDecodeVec]) {
+    const uint2 x = __ldg(reinterpret_cast<const uint2 *>(p));
+    o[0] = __uint_as_float(x.x << 16);
+    o[1] = __uint_as_float(x.x & 0xffff0000u);
+    o[2] = __uint_as_float(x.y << 16);
+    o[3] = __uint_as_float(x.y & 0xffff0000u);
+}
+
+// part[split][b][d] = sum over the split's j of v[b, j, d] g[b, t-j, d], in
+// fp64, j ascending.  vec: D is a multiple of kDecodeVec and the caches are
+// aligned for one access per kDecodeVec channels.
 template <typename IO>
 __global__ void __launch_bounds__(kDecodeThreads)
     decode_partial_kernel(const IO *__restrict__ v, const IO *__restrict__ g, double *__restrict__ part, int B,
-                          int Lcap, int D, int t, int chunk) {
-    const int d = blockIdx.x * kDecodeThreads + threadIdx.x;
+                          int Lcap, int D, int t, int chunk, int vec) {
+    const int d0 = (blockIdx.x * kDecodeThreads + threadIdx.x) * kDecodeVec;
     const int sp = blockIdx.y, b = blockIdx.z;
-    if (d >= D) return;
+    if (d0 >= D) return;
     const int j0 = sp * chunk;
     const int j1 = min(t + 1, j0 + chunk);
     const int64_t row = (int64_t)b * Lcap;
-    const IO *vb = v + row * D + d;
-    const IO *gb = g + row * D + d;
-    double acc[kDecodeUnroll] = {0.0, 0.0, 0.0, 0.0};
-    int j = j0;
-    for (; j + kDecodeUnroll <= j1; j += kDecodeUnroll) {
+    const IO *vb = v + row * D + d0;
+    const IO *gb = g + row * D + d0;
+    double acc[kDecodeVec] = {0.0, 0.0, 0.0, 0.0};
+    if (vec) {
+#pragma unroll kDecodeUnroll
+        for (int j = j0; j < j1; ++j) {
+            float a[kDecodeVec], c[kDecodeVec];
+            decode_ld4(vb + (int64_t)j * D, a);
+            decode_ld4(gb + (int64_t)(t - j) * D, c);
 #pragma unroll
-        for (int u = 0; u < kDecodeUnroll; ++u) {
-            const float a = IO_t<IO>::cvt(IO_t<IO>::ld(vb + (int64_t)(j + u) * D));
-            const float c = IO_t<IO>::cvt(IO_t<IO>::ld(gb + (int64_t)(t - j - u) * D));
-            acc[u] = fma((double)a, (double)c, acc[u]);
+            for (int q = 0; q < kDecodeVec; ++q) acc[q] = fma((double)a[q], (double)c[q], acc[q]);
+        }
+    } else {
+        const int nc = min(kDecodeVec, D - d0);
+        for (int j = j0; j < j1; ++j) {
+#pragma unroll
+            for (int q = 0; q < kDecodeVec; ++q)
+                if (q < nc) {
+                    const float a = IO_t<IO>::cvt(IO_t<IO>::ld(vb + (int64_t)j * D + q));
+                    const float c = IO_t<IO>::cvt(IO_t<IO>::ld(gb + (int64_t)(t - j) * D + q));
+                    acc[q] = fma((double)a, (double)c, acc[q]);
+                }
         }
     }
-    for (; j < j1; ++j) {
-        const float a = IO_t<IO>::cvt(IO_t<IO>::ld(vb + (int64_t)j * D));
-        const float c = IO_t<IO>::cvt(IO_t<IO>::ld(gb + (int64_t)(t - j) * D));
-        acc[0] = fma((double)a, (double)c, acc[0]);
-    }
-    part[((int64_t)sp * B + b) * D + d] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    double *pp = part + ((int64_t)sp * B + b) * D + d0;
+#pragma unroll
+    for (int q = 0; q < kDecodeVec; ++q)
+        if (d0 + q < D) pp[q] = acc[q];
 }
 
 template <typename IO>
-__global__ void __launch_bounds__(kDecodeThreads)
+__global__ void __launch_bounds__(kReduceThreads)
     decode_reduce_kernel(const double *__restrict__ part, IO *__restrict__ r, int64_t BD, int splits) {
-    const int64_t i = (int64_t)blockIdx.x * kDecodeThreads + threadIdx.x;
+    const int64_t i = (int64_t)blockIdx.x * kReduceThreads + threadIdx.x;
     if (i >= BD) return;
     double s = 0.0;
     for (int k = 0; k < splits; ++k) s += part[(int64_t)k * BD + i];
@@ -85,11 +118,15 @@ static int decode_launch(const IO *v, const IO *g, IO *r, int64_t B, int64_t Lca
                          double *part, cudaStream_t s) {
     const int splits = decode_splits(B, D, t);
     const int chunk = (int)((t + 1 + splits - 1) / splits);
-    const dim3 grid((unsigned)((D + kDecodeThreads - 1) / kDecodeThreads), (unsigned)splits, (unsigned)B);
-    decode_partial_kernel<IO><<<grid, kDecodeThreads, 0, s>>>(v, g, part, (int)B, (int)Lcap, (int)D, (int)t, chunk);
+    const int per_cta = kDecodeThreads * kDecodeVec;
+    const dim3 grid((unsigned)((D + per_cta - 1) / per_cta), (unsigned)splits, (unsigned)B);
+    const size_t align = kDecodeVec * sizeof(IO);
+    const int vec = (D % kDecodeVec) == 0 && ((uintptr_t)v % align) == 0 && ((uintptr_t)g % align) == 0;
+    decode_partial_kernel<IO><<<grid, kDecodeThreads, 0, s>>>(v, g, part, (int)B, (int)Lcap, (int)D, (int)t, chunk,
+                                                              vec);
     if (cudaGetLastError() != cudaSuccess) return 5;  // CC_ERR_CUDA
     const int64_t BD = B * D;
-    decode_reduce_kernel<IO><<<(unsigned)((BD + kDecodeThreads - 1) / kDecodeThreads), kDecodeThreads, 0, s>>>(
+    decode_reduce_kernel<IO><<<(unsigned)((BD + kReduceThreads - 1) / kReduceThreads), kReduceThreads, 0, s>>>(
         part, r, BD, splits);
     return cudaGetLastError() == cudaSuccess ? 0 : 5;
 }

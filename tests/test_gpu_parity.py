@@ -366,7 +366,8 @@ def test_bwd_consistent_with_forward_adjoint():
 # ---------------------------------------------------------------- decode step
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("case", [(2, 64, 5, 0), (2, 64, 5, 1), (3, 300, 37, 63), (3, 300, 37, 64),
-                                  (1, 5000, 19, 4999), (8, 1024, 768, 1023), (8, 1024, 768, 500)],
+                                  (1, 5000, 19, 4999), (8, 1024, 768, 1023), (8, 1024, 768, 500),
+                                  (2, 3000, 260, 2999), (1, 40, 12, 15)],
                          ids=lambda c: "x".join(map(str, c)))
 def test_decode_step_matches_oracle(case, dtype):
     """One decode step equals the causal sum at position t, bit-identically
