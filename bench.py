@@ -103,19 +103,21 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def recorded_traffic(workload: str, kernel: str):
-    """DRAM bytes (read + write) per launch of `kernel` on the full-size
-    `workload`, from profiles/dram_traffic.txt (lines: workload kernel
-    source_hash bytes), if it was taken on the current kernel sources; else
-    None."""
-    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+def recorded_counters(workload: str, kernel: str):
+    """(DRAM bytes read + write, FP32 lane operations) per launch of `kernel`
+    on the full-size `workload`, from profiles/kernel_counters.txt (lines:
+    workload kernel source_hash dram_bytes fp32_lane_ops), if they were taken
+    on the current kernel sources; else (None, None)."""
+    p = os.path.join(ROOT, "profiles", "kernel_counters.txt")
     if not os.path.exists(p):
-        return None
+        return None, None
     for line in open(p):
         f = line.split()
-        if len(f) == 4 and not line.startswith("#") and f[0] == workload and f[1] == kernel:
-            return float(f[3]) if f[2] == kernel_source_hash() else None
-    return None
+        if len(f) == 5 and not line.startswith("#") and f[0] == workload and f[1] == kernel:
+            if f[2] != kernel_source_hash():
+                return None, None
+            return float(f[3]), float(f[4])
+    return None, None
 
 
 class ClockSampler:
@@ -370,6 +372,8 @@ def run_ours(args, rank, world, local):
         kernel = "bigconv_kernel (two-pass step: 2 transposes in, 1 out)"
     per_launch_bytes = bytes_per_step // 2 if args.path == "bwd" else bytes_per_step
     achieved = bytes_per_step / (ms_per_step * 1e-3) / 1e9
+    traffic, fp32_ops = (None, None) if (args.shape or args.path != "fwd") else recorded_counters(w.name, kernel)
+    clocks = clk.report()
     line = {
         "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -382,14 +386,23 @@ def run_ours(args, rank, world, local):
         "hbm_frac": gbs / world / peak,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
-                     "kernel": kernel, "algorithmic_bytes_per_launch": per_launch_bytes,
-                     "traffic": None if (args.shape or args.path != "fwd") else recorded_traffic(w.name, kernel)},
+                     "kernel": kernel, "algorithmic_bytes_per_launch": per_launch_bytes, "traffic": traffic},
         "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": 2 * w.units * w.elem_bytes,
                 "d2h_bytes_per_step": w.units * w.elem_bytes, "steps": e2e_steps,
                 "path": "causal_conv_from_host (pinned host buffers)"},
         "gpu_launches": args.steps * launches_per_step,
-        "clocks": clk.report(),
+        "clocks": clocks,
     }
+    if fp32_ops and launches_per_step == 1:
+        # the transform kernels are bound by FP32 issue, not by HBM: executed
+        # FP32 lane operations (ncu, same sources) per launch against
+        # 148 SMs x 128 FP32 lanes x the SM clock sampled during the run
+        sm_hz = clocks["sm_mhz"] * 1e6 if clocks and clocks.get("sm_mhz") else 1.965e9
+        alu_peak = 148 * 128 * sm_hz / 1e9
+        alu_achieved = fp32_ops / (ms_per_step * 1e-3) / 1e9
+        line["alu_roofline"] = {"bound": "alu", "achieved": alu_achieved, "peak": alu_peak, "unit": "G FP32 lane-op/s",
+                                "frac": alu_achieved / alu_peak, "fp32_lane_ops_per_launch": fp32_ops,
+                                "peak_source": "148 SMs x 128 FP32 lanes/clk x sampled SM clock"}
     if args.path != "fwd":  # the host-buffer leg and CPU baseline describe the forward line only
         line.pop("e2e")
         args.no_cpu_baseline = True
