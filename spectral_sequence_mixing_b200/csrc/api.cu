@@ -108,7 +108,10 @@ static int g_num_sms[128];
 
 template <class Cfg, typename IO, int MINB>
 static cudaError_t set_smem_attr() {
-    return cudaFuncSetAttribute(fftconv_fused_kernel<Cfg::N2, Cfg::ROWS, MINB, IO>,
+    const cudaError_t e = cudaFuncSetAttribute(fftconv_fused_kernel<Cfg::N2, Cfg::ROWS, MINB, IO, false>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(fftconv_fused_kernel<Cfg::N2, Cfg::ROWS, MINB, IO, true>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_BYTES);
 }
 
@@ -286,7 +289,9 @@ static int launch_fused(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, i
     const int64_t groups = (D + Cfg::ROWS - 1) / Cfg::ROWS;
     const int64_t tiles = B * groups;
     if (tiles > INT32_MAX) return CC_ERR_UNSUPPORTED;
-    auto kern = fftconv_fused_kernel<Cfg::N2, Cfg::ROWS, MINB, IO>;
+    // v read reversed in time (backward pass): the kernel instance that reverses on its shared-memory reads
+    auto kern = (rev & 1) ? fftconv_fused_kernel<Cfg::N2, Cfg::ROWS, MINB, IO, true>
+                          : fftconv_fused_kernel<Cfg::N2, Cfg::ROWS, MINB, IO, false>;
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cfg::THREADS, Cfg::SMEM_BYTES) != cudaSuccess ||
         per_sm < 1) {
@@ -296,11 +301,11 @@ static int launch_fused(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, i
     const int64_t grid = std::min<int64_t>(tiles, (int64_t)per_sm * g_num_sms[dev]);
     // whole-chunk async copies need full, aligned channel groups
     const bool vec = (D % Cfg::ROWS) == 0 && ((uintptr_t)v % Cfg::CHUNK) == 0 && ((uintptr_t)g % Cfg::CHUNK) == 0;
-    // TMA boxes when a tile row is whole 16-byte units and v is read forward in time
+    // TMA boxes when a tile row is whole 16-byte units
     CUtensorMap tmv, tmg;
     memset(&tmv, 0, sizeof(tmv));
     memset(&tmg, 0, sizeof(tmg));
-    const bool tma = Cfg::TMA_OK && (rev & 1) == 0 &&
+    const bool tma = Cfg::TMA_OK &&
                      encode_btd_map<IO>(&tmv, v, B, L, D, Cfg::ROWS, Cfg::BOXT) &&
                      encode_btd_map<IO>(&tmg, g, B, L, D, Cfg::ROWS, Cfg::BOXT);
     kern<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(v, g, r, (int)L, (int)D, (int)groups, (int)tiles,

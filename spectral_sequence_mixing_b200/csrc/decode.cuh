@@ -30,13 +30,13 @@ constexpr int kDecodeVec = 4;        // channels per thread (one 16-byte fp32 / 
 constexpr int kReduceThreads = 256;
 constexpr int kDecodeUnroll = 8;
 
-// Number of j-ranges for a decode call: aim at ~1184 CTAs (8 per SM of a
+// Number of j-ranges for a decode call: aim at ~2368 CTAs (16 per SM of a
 // 148-SM part) of 256 channels, at least 16 positions per range, at most 128
 // ranges.  Depends only on the problem (so the workspace size is
 // host-computable).
 static inline int decode_splits(int64_t B, int64_t D, int64_t t) {
     const int64_t ctas = B * ((D + kDecodeThreads * kDecodeVec - 1) / (kDecodeThreads * kDecodeVec));
-    int64_t s = (1184 + ctas - 1) / ctas;
+    int64_t s = (2368 + ctas - 1) / ctas;
     const int64_t max_by_len = (t + 1 + 15) / 16;
     if (s > max_by_len) s = max_by_len;
     if (s > 128) s = 128;

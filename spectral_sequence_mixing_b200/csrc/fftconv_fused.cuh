@@ -183,7 +183,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // plain loads (2-byte elements) are used.
 template <class C, typename IO>
 __device__ __forceinline__ void stage_tile(const IO *__restrict__ v, const IO *__restrict__ g, IO *sv, IO *sg,
-                                           int64_t boff, int d0, int L, int D, bool vec, bool rev_a) {
+                                           int64_t boff, int d0, int L, int D, bool vec) {
     constexpr int ROWS = C::ROWS;
     const int tid = threadIdx.x;
     const IO *vb = v + boff + d0;
@@ -193,17 +193,16 @@ __device__ __forceinline__ void stage_tile(const IO *__restrict__ v, const IO *_
         for (int e = tid; e < L * C::NCHUNK; e += C::THREADS) {
             const int t = e / C::NCHUNK, q = e - t * C::NCHUNK;
             const int64_t o = (int64_t)t * D + q * EPC;
-            const int64_t ov = (int64_t)(rev_a ? L - 1 - t : t) * D + q * EPC;
             IO *dv = sv + t * ROWS + q * EPC;
             IO *dg = sg + t * ROWS + q * EPC;
             if (C::CHUNK == 16) {
-                cp_async16(dv, vb + ov);
+                cp_async16(dv, vb + o);
                 cp_async16(dg, gb + o);
             } else if (C::CHUNK == 8) {
-                cp_async8(dv, vb + ov);
+                cp_async8(dv, vb + o);
                 cp_async8(dg, gb + o);
             } else {
-                cp_async4(dv, vb + ov);
+                cp_async4(dv, vb + o);
                 cp_async4(dg, gb + o);
             }
         }
@@ -213,12 +212,11 @@ __device__ __forceinline__ void stage_tile(const IO *__restrict__ v, const IO *_
             const int t = e / ROWS, c = e - t * ROWS;
             if (c < nc) {
                 const int64_t o = (int64_t)t * D + c;
-                const int64_t ov = (int64_t)(rev_a ? L - 1 - t : t) * D + c;
                 if (sizeof(IO) == 4) {
-                    cp_async4(sv + e, vb + ov);
+                    cp_async4(sv + e, vb + o);
                     cp_async4(sg + e, gb + o);
                 } else {
-                    sv[e] = IO_t<IO>::ld(vb + ov);
+                    sv[e] = IO_t<IO>::ld(vb + o);
                     sg[e] = IO_t<IO>::ld(gb + o);
                 }
             }
@@ -236,18 +234,20 @@ __device__ __forceinline__ void bar_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
 }
 
-template <int N2, int ROWS, int MINB, typename IO>
+template <int N2, int ROWS, int MINB, typename IO, bool REVA>
 __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
     fftconv_fused_kernel(const IO *__restrict__ v, const IO *__restrict__ g, IO *__restrict__ r, int L, int D,
                          int groups_per_batch, int num_tiles, int vec_ok, int rev, const float2 *__restrict__ tw,
                          const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmg,
                          int use_tma) {
-    // rev bit 0: read v reversed in time (v_t -> v_{L-1-t}); bit 1: write r reversed
+    // REVA: v is read reversed in time (v_t -> v_{L-1-t}); the staging keeps v
+    // in natural order and the reversal happens on the shared-memory reads.
+    // rev bit 1: write r reversed.
     // use_tma: stage tiles with TMA boxes from tmv / tmg (3-D maps over {D, L, B}),
     // otherwise with cp.async from the pointers
     using C = FusedCfg<N2, ROWS, IO>;
     constexpr int N1 = C::N1, N = C::N, M2 = C::M2, H = C::H, MH = C::MH;
-    const bool rev_a = rev & 1, rev_out = (rev >> 1) & 1;
+    const bool rev_out = (rev >> 1) & 1;
     constexpr int SC = C::SC, SF_N = C::SF_N, SI_M = C::SI_M, HEAD = C::HEAD, LMAX = C::LMAX;
     constexpr int THREADS = C::THREADS;
     extern __shared__ float4 smem_raw[];
@@ -260,6 +260,16 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
     float2 *rot = reinterpret_cast<float2 *>(alpha_row + 2 * ROWS);       // [2h+s][H+1]
     uint64_t *bar = reinterpret_cast<uint64_t *>(rot + 4 * (H + 1));      // staging-complete barrier
     const int tid = threadIdx.x;
+    // v at time t (0 <= t < LMAX) of row c from the staging: v_t, or v_{L-1-t} (0 for t >= L)
+    auto v_at = [&](int t, int c) -> float {
+        if constexpr (REVA) {
+            const int tr = L - 1 - t;
+            const float x = IO_t<IO>::cvt(sv[max(tr, 0) * ROWS + c]);
+            return tr >= 0 ? x : 0.f;
+        } else {
+            return IO_t<IO>::cvt(sv[t * ROWS + c]);
+        }
+    };
     const bool tma = C::TMA_OK && use_tma && (smem_u32(sv) & 127) == 0;
     unsigned phase = 0;
     // stage tile `t` (v and g, t < LMAX, zero-filled past L and D) into sv / sg
@@ -276,7 +286,7 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
                 }
             }
         } else {
-            stage_tile<C, IO>(v, g, sv, sg, (int64_t)b * L * D, d0, L, D, vec_ok && d0 + ROWS <= D, rev_a);
+            stage_tile<C, IO>(v, g, sv, sg, (int64_t)b * L * D, d0, L, D, vec_ok && d0 + ROWS <= D);
         }
     };
 
@@ -333,7 +343,7 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
 #pragma unroll
             for (int n1 = 0; n1 < N2; ++n1) {
                 const int t = n2 + N2 * n1;
-                const float2 zv = make_float2(IO_t<IO>::cvt(sv[t * ROWS + c]), IO_t<IO>::cvt(sg[t * ROWS + c]));
+                const float2 zv = make_float2(v_at(t, c), IO_t<IO>::cvt(sg[t * ROWS + c]));
                 zr[n1] = zv;
                 nv = fmaf(zv.x, zv.x, nv);
                 ng = fmaf(zv.y, zv.y, ng);
@@ -343,7 +353,7 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
             {
                 constexpr int HP = C::HP, JP = HEAD / HP;
                 const int w = tid >> 5, hc = w % ROWS, hp = w / ROWS, lt = tid & 31;
-                const float vt = IO_t<IO>::cvt(sv[lt * ROWS + hc]);
+                const float vt = v_at(lt, hc);
                 const float gt = IO_t<IO>::cvt(sg[lt * ROWS + hc]);
                 float acc = 0.f;
 #pragma unroll
