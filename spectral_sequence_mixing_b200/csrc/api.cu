@@ -11,6 +11,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <initializer_list>
 #include <mutex>
 #include <type_traits>
@@ -105,6 +106,8 @@ constexpr int kMinbM = 2;
 
 // Per device: SM count and, per kernel instantiation, resident CTAs per SM.
 static int g_num_sms[128];
+// Per device: device addresses of the twiddle tables (small, mid, one-CTA rows, cluster rows).
+static void *g_tw_addr[128][4];
 
 template <class Cfg, typename IO, int MINB>
 static cudaError_t set_smem_attr() {
@@ -158,6 +161,10 @@ static cudaError_t ensure_init(int dev) {
     if ((e = set_smem_attr<CfgM<float>, float, kMinbM>()) != cudaSuccess) return e;
     if ((e = set_smem_attr<CfgM<__nv_bfloat16>, __nv_bfloat16, kMinbM>()) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaGetSymbolAddress(&g_tw_addr[dev][0], g_tw_s)) != cudaSuccess) return e;
+    if ((e = cudaGetSymbolAddress(&g_tw_addr[dev][1], g_tw_m)) != cudaSuccess) return e;
+    if ((e = cudaGetSymbolAddress(&g_tw_addr[dev][2], g_tw_bl)) != cudaSuccess) return e;
+    if ((e = cudaGetSymbolAddress(&g_tw_addr[dev][3], g_tw_bx)) != cudaSuccess) return e;
     g_init_done[dev] = true;
     return cudaSuccess;
 }
@@ -292,11 +299,17 @@ static int launch_fused(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, i
     // v read reversed in time (backward pass): the kernel instance that reverses on its shared-memory reads
     auto kern = (rev & 1) ? fftconv_fused_kernel<Cfg::N2, Cfg::ROWS, MINB, IO, true>
                           : fftconv_fused_kernel<Cfg::N2, Cfg::ROWS, MINB, IO, false>;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cfg::THREADS, Cfg::SMEM_BYTES) != cudaSuccess ||
-        per_sm < 1) {
-        cudaGetLastError();
-        return CC_ERR_CUDA;
+    // resident CTAs per SM, queried once per device and kernel instance
+    static std::atomic<int> resident[2][128];
+    int per_sm = resident[rev & 1][dev].load(std::memory_order_relaxed);
+    if (per_sm == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cfg::THREADS, Cfg::SMEM_BYTES) !=
+                cudaSuccess ||
+            per_sm < 1) {
+            cudaGetLastError();
+            return CC_ERR_CUDA;
+        }
+        resident[rev & 1][dev].store(per_sm, std::memory_order_relaxed);
     }
     const int64_t grid = std::min<int64_t>(tiles, (int64_t)per_sm * g_num_sms[dev]);
     // whole-chunk async copies need full, aligned channel groups
@@ -400,21 +413,15 @@ static int launch_group(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, i
 template <typename IO>
 static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, void *ws,
                             size_t ws_bytes, cudaStream_t s, int dev, int rev = 0) {
-    void *tw = nullptr;
-    if (L <= CfgS<IO>::LMAX) {
-        if (cudaGetSymbolAddress(&tw, g_tw_s) != cudaSuccess) return CC_ERR_CUDA;
-        return launch_fused<CfgS<IO>, kMinbS>(v, g, r, B, L, D, (const float2 *)tw, s, dev, rev);
-    }
-    if (L <= CfgM<IO>::LMAX) {
-        if (cudaGetSymbolAddress(&tw, g_tw_m) != cudaSuccess) return CC_ERR_CUDA;
-        return launch_fused<CfgM<IO>, kMinbM>(v, g, r, B, L, D, (const float2 *)tw, s, dev, rev);
-    }
-    if (L <= BigL<IO>::LMAX) {
-        if (cudaGetSymbolAddress(&tw, g_tw_bl) != cudaSuccess) return CC_ERR_CUDA;
-        return launch_group<BigL<IO>, kMinbBigL>(v, g, r, B, L, D, (const float2 *)tw, s, rev);
-    }
+    void *const *tws = g_tw_addr[dev];  // filled by ensure_init
+    if (L <= CfgS<IO>::LMAX)
+        return launch_fused<CfgS<IO>, kMinbS>(v, g, r, B, L, D, (const float2 *)tws[0], s, dev, rev);
+    if (L <= CfgM<IO>::LMAX)
+        return launch_fused<CfgM<IO>, kMinbM>(v, g, r, B, L, D, (const float2 *)tws[1], s, dev, rev);
+    if (L <= BigL<IO>::LMAX)
+        return launch_group<BigL<IO>, kMinbBigL>(v, g, r, B, L, D, (const float2 *)tws[2], s, rev);
     if (L <= BigX<IO>::LMAX) {
-        if (cudaGetSymbolAddress(&tw, g_tw_bx) != cudaSuccess) return CC_ERR_CUDA;
+        const void *tw = tws[3];
         const size_t fast = fast_ws_bytes(sizeof(IO) == 4 ? CC_DTYPE_F32 : CC_DTYPE_BF16, B, L, D);
         if (ws == nullptr || fast == 0 || ws_bytes < fast)
             return launch_big<BigX<IO>, kMinbBigX>(v, g, r, B, L, D, (const float2 *)tw, s, rev, 0);
