@@ -70,7 +70,11 @@ typedef enum {
  *   (device), must not overlap v or g.  B, L, D >= 1.
  *   workspace / workspace_bytes: device scratch of at least
  *   causal_conv_workspace_bytes(CC_DTYPE_F32, B, L, D) bytes (0 for every
- *   supported L today; pass NULL, 0).
+ *   supported L: NULL, 0 is valid).  A workspace of at least
+ *   causal_conv_fast_workspace_bytes(...) bytes (nonzero for 4096 < L) makes
+ *   long rows take the two-pass path (rows transposed to be contiguous); it
+ *   must then not overlap v, g or r (CC_ERR_ALIAS).  Caller-owned; its
+ *   contents are scratch, undefined after the call.
  *
  * Accuracy: |r - r_exact| <= 1e-5 * sum_j |v_j g_{t-j}| per element on the
  * tested workloads; outputs with t < 32 are summed directly (no transform),
