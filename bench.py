@@ -196,7 +196,19 @@ def cpu_oracle_rate(w: workloads.Workload, v, g, budget_s: float):
         if spent >= budget_s / 3 or k == w.D or dt * 2 > budget_s - spent:
             break
         k *= 2
-    desc = f"oracle on channels [0,{k}) of {w.name}: {w.B}x{w.L}x{k} = {units} outputs (whole rows)"
+    reps = 1
+    if k == w.D and secs < budget_s / 3:
+        # the whole workload is cheap: repeat it to time about budget_s of work
+        reps = max(1, min(64, int(budget_s / max(secs, 1e-3))))
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            if w.dtype == "i32":
+                oracle.causal_conv_int(sv, sg)
+            else:
+                oracle.causal_conv(sv, sg)
+        units, secs = w.B * w.L * k * reps, time.perf_counter() - t0
+    desc = (f"oracle on channels [0,{k}) of {w.name}: {w.B}x{w.L}x{k} outputs (whole rows)"
+            + (f", {reps} passes" if reps > 1 else ""))
     return units / secs, oracle.num_threads(), desc, secs
 
 

@@ -57,11 +57,16 @@ def fast_workspace_bytes(dtype: torch.dtype, B: int, L: int, D: int) -> int:
     return int(load().causal_conv_fast_workspace_bytes(_DT[dtype], B, L, D))
 
 
+_ONE_CTA_ROW = 4096  # rows up to this length never use the optional workspace
+
+
 def _workspace(workspace, dtype_code: int, B: int, L: int, D: int, device):
     """(pointer, bytes) of the caller's workspace; with none given, one of the
     optional two-pass size is taken from the torch allocator when that path
     applies.  A tensor of 0 bytes selects the single-pass path."""
     if workspace is None:
+        if L <= _ONE_CTA_ROW or dtype_code == CC_DTYPE_I32:
+            return None, 0
         n = int(load().causal_conv_fast_workspace_bytes(dtype_code, B, L, D))
         if n == 0:
             return None, 0
@@ -81,9 +86,12 @@ def _run(dtype_code: int, v: torch.Tensor, g: torch.Tensor, out, workspace, stre
         out = torch.empty_like(v)
     _check(out, "out", dtype, v.shape)
     ws_ptr, ws_bytes = _workspace(workspace, dtype_code, B, L, D, v.device)
-    with torch.cuda.device(v.device):
-        st = getattr(load(), _FN[dtype_code])(v.data_ptr(), g.data_ptr(), out.data_ptr(), B, L, D, ws_ptr, ws_bytes,
-                                              _stream_ptr(stream))
+    fn = getattr(load(), _FN[dtype_code])
+    if v.device.index == torch.cuda.current_device():
+        st = fn(v.data_ptr(), g.data_ptr(), out.data_ptr(), B, L, D, ws_ptr, ws_bytes, _stream_ptr(stream))
+    else:  # the library works on the current device: switch to the tensors' one (and its stream)
+        with torch.cuda.device(v.device):
+            st = fn(v.data_ptr(), g.data_ptr(), out.data_ptr(), B, L, D, ws_ptr, ws_bytes, _stream_ptr(stream))
     if st != 0:
         raise CausalConvError(st, _FN[dtype_code])
     return out
