@@ -44,14 +44,19 @@ MUTANTS = {
 }
 
 
+MUTANT_DIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_build", "mutants")  # git-ignored
+
+
 @pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_mutant_is_caught(name, tmp_path):
+def test_mutant_is_caught(name):
     old, new = MUTANTS[name]
     src = open(oracle._SRC).read()
     assert src.count(old) >= 1, f"mutation site for {name} not found"
-    mut = tmp_path / f"mut_{name}.c"
-    mut.write_text(src.replace(old, new))
-    so = tmp_path / f"libmut_{name}.so"
+    os.makedirs(MUTANT_DIR, exist_ok=True)
+    mut = os.path.join(MUTANT_DIR, f"mut_{name}.c")
+    with open(mut, "w") as f:
+        f.write(src.replace(old, new))
+    so = os.path.join(MUTANT_DIR, f"libmut_{name}.so")
     oracle.build(str(mut), str(so), force=True)
     lib = oracle.load(str(so))
     failed = oracle_pins.run_all(lib)
