@@ -197,13 +197,19 @@ CC_API int causal_conv_decode_f32_noalloc(const float *v, const float *g, float 
 CC_API size_t causal_conv_decode_workspace_bytes(int dtype, int64_t B, int64_t D, int64_t t);
 
 /*
- * causal_conv_from_host -- the same convolution for HOST buffers: enqueues on
- * `stream` the copy of v_host and g_host into the caller's device buffers
- * v_dev and g_dev, the convolution into r_dev, and the copy of r_dev back
- * into r_host, then returns (asynchronous; pass pinned host memory for
- * overlap, and synchronise `stream` before reading r_host).
+ * causal_conv_from_host -- the same convolution for HOST buffers: the copy of
+ * v_host and g_host into the caller's device buffers v_dev and g_dev, the
+ * convolution into r_dev, and the copy of r_dev back into r_host, ordered
+ * after the work already on `stream`; `stream` waits for the last copy back
+ * (asynchronous: synchronise `stream` before reading r_host; pass pinned host
+ * memory, or the copies are synchronous).  With B >= 2 the batches go in up
+ * to 4 pieces on two library-owned streams of the device, so the upload and
+ * transform of one piece overlap the download of the previous one (copies in
+ * both directions at once); concurrent calls on one device are serialised
+ * while they enqueue.
  *   dtype: a cc_dtype.  All six buffers hold B*L*D elements of that type.
- * Errors as for the device entry points; nothing is enqueued on failure.
+ * Errors as for the device entry points; nothing is enqueued on an argument
+ * error (a CUDA error part-way may leave earlier pieces enqueued).
  */
 CC_API int causal_conv_from_host(int dtype, const void *v_host, const void *g_host, void *r_host,
                           void *v_dev, void *g_dev, void *r_dev,

@@ -23,21 +23,15 @@
 #include "ntt.cuh"
 #include "decode.cuh"
 #include "transpose.cuh"
+#include "configs.cuh"
 
 namespace ccv {
 
 // ------------------------------------------------------------------ tables
-// Transform geometry per size class (the twiddle tables depend only on N1, N2).
-template <typename IO> using CfgS = FusedCfg<16, 8, IO>;  // N = 512,  L <= 256
-template <typename IO> using CfgM = FusedCfg<32, 4, IO>;  // N = 2048, L <= 1024
-
+// Twiddle tables per size class (configs.cuh; they depend only on the geometry).
 __device__ float2 g_tw_s[CfgS<float>::TW_SIZE];
 __device__ float2 g_tw_m[CfgM<float>::TW_SIZE];
 
-// Long rows: one row per CTA (N = 8192) or per 8-CTA cluster (N = 131072).
-template <typename IO> using BigL = BigCfg<32, 16, 16, 1, 1, 256, IO>;   // N = 8192,   L <= 4096
-template <typename IO> using BigX = BigCfg<8, 32, 32, 16, 8, 512, IO>;   // N = 131072, L <= 65536
-constexpr int kMinbBigL = 2, kMinbBigX = 1;
 __device__ float2 g_tw_bl[BigL<float>::TW_SIZE];
 __device__ float2 g_tw_bx[BigX<float>::TW_SIZE];
 
@@ -101,8 +95,6 @@ static cudaError_t set_big_attr() {
 static std::mutex g_init_mu;
 static bool g_init_done[128];
 
-constexpr int kMinbS = 4;
-constexpr int kMinbM = 2;
 
 // Per device: SM count and, per kernel instantiation, resident CTAs per SM.
 static int g_num_sms[128];
@@ -521,6 +513,72 @@ static int noalloc_scratch(int dev, double **out) {
 
 using namespace ccv;
 
+// ------------------------------------------------------------------ host buffers
+constexpr int64_t kHostChunks = 4;
+
+// Per device: the two streams and events of the pipelined host-buffer path.
+struct HostPipe {
+    cudaStream_t up = nullptr, down = nullptr;
+    cudaEvent_t start = nullptr, handoff = nullptr, done = nullptr;
+    std::mutex mu;
+};
+
+static HostPipe *host_pipe(int dev) {
+    static HostPipe pipes[128];
+    static std::once_flag once[128];
+    static bool ok[128];
+    std::call_once(once[dev], [dev] {
+        HostPipe &p = pipes[dev];
+        ok[dev] = cudaStreamCreateWithFlags(&p.up, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&p.down, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&p.start, cudaEventDisableTiming) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&p.handoff, cudaEventDisableTiming) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&p.done, cudaEventDisableTiming) == cudaSuccess;
+        cudaGetLastError();
+    });
+    return ok[dev] ? &pipes[dev] : nullptr;
+}
+
+// Batches [b0, b0 + nb) of a host-buffer call: upload v, g on `up`, transform
+// on `up`, download r on `down` after `up` (through `handoff` when the streams differ).
+static int from_host_chunk(int dtype, const void *v_host, const void *g_host, void *r_host, void *v_dev, void *g_dev,
+                           void *r_dev, int64_t b0, int64_t nb, int64_t L, int64_t D, void *ws, size_t ws_bytes,
+                           cudaStream_t up, cudaStream_t down, cudaEvent_t handoff = nullptr) {
+    const size_t es = dtype_size(dtype);
+    const size_t off = (size_t)(b0 * L * D) * es, bytes = (size_t)(nb * L * D) * es;
+    const char *hv = (const char *)v_host + off, *hg = (const char *)g_host + off;
+    char *hr = (char *)r_host + off, *dv = (char *)v_dev + off, *dg = (char *)g_dev + off, *dr = (char *)r_dev + off;
+    if (cudaMemcpyAsync(dv, hv, bytes, cudaMemcpyHostToDevice, up) != cudaSuccess ||
+        cudaMemcpyAsync(dg, hg, bytes, cudaMemcpyHostToDevice, up) != cudaSuccess) {
+        cudaGetLastError();
+        return CC_ERR_CUDA;
+    }
+    int st;
+    switch (dtype) {
+        case CC_DTYPE_F32:
+            st = causal_fftconv_f32((const float *)dv, (const float *)dg, (float *)dr, nb, L, D, ws, ws_bytes, up);
+            break;
+        case CC_DTYPE_BF16:
+            st = causal_fftconv_bf16((const uint16_t *)dv, (const uint16_t *)dg, (uint16_t *)dr, nb, L, D, ws, ws_bytes,
+                                     up);
+            break;
+        default:
+            st = causal_ntt_conv_i32((const int32_t *)dv, (const int32_t *)dg, (int32_t *)dr, nb, L, D, ws, ws_bytes,
+                                     up);
+            break;
+    }
+    if (st != CC_OK) return st;
+    if (up != down && (cudaEventRecord(handoff, up) != cudaSuccess || cudaStreamWaitEvent(down, handoff, 0) != cudaSuccess)) {
+        cudaGetLastError();
+        return CC_ERR_CUDA;
+    }
+    if (cudaMemcpyAsync(hr, dr, bytes, cudaMemcpyDeviceToHost, down) != cudaSuccess) {
+        cudaGetLastError();
+        return CC_ERR_CUDA;
+    }
+    return CC_OK;
+}
+
 extern "C" {
 
 size_t causal_conv_workspace_bytes(int dtype, int64_t B, int64_t L, int64_t D) {
@@ -651,28 +709,28 @@ int causal_conv_from_host(int dtype, const void *v_host, const void *g_host, voi
     if (st != CC_OK) return st;
     const size_t bytes = (size_t)(B * L * D) * dtype_size(dtype);
     if (ranges_overlap(v_dev, g_dev, bytes)) return CC_ERR_ALIAS;
+    if (ensure_init(dev) != cudaSuccess) return CC_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
-    if (cudaMemcpyAsync(v_dev, v_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(g_dev, g_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+    const int64_t chunks = std::min<int64_t>(B, kHostChunks);
+    HostPipe *pipe = chunks > 1 ? host_pipe(dev) : nullptr;
+    if (!pipe) return from_host_chunk(dtype, v_host, g_host, r_host, v_dev, g_dev, r_dev, 0, B, L, D, workspace,
+                                      workspace_bytes, s, s);
+    // batches in kHostChunks pieces: the upload and transform of piece c+1 (stream
+    // up) overlap the download of piece c (stream down); the caller's stream
+    // waits for the last download
+    std::lock_guard<std::mutex> lk(pipe->mu);
+    if (cudaEventRecord(pipe->start, s) != cudaSuccess || cudaStreamWaitEvent(pipe->up, pipe->start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(pipe->down, pipe->start, 0) != cudaSuccess) {
         cudaGetLastError();
         return CC_ERR_CUDA;
     }
-    switch (dtype) {
-        case CC_DTYPE_F32:
-            st = causal_fftconv_f32((const float *)v_dev, (const float *)g_dev, (float *)r_dev, B, L, D, workspace,
-                                    workspace_bytes, stream);
-            break;
-        case CC_DTYPE_BF16:
-            st = causal_fftconv_bf16((const uint16_t *)v_dev, (const uint16_t *)g_dev, (uint16_t *)r_dev, B, L, D,
-                                     workspace, workspace_bytes, stream);
-            break;
-        default:
-            st = causal_ntt_conv_i32((const int32_t *)v_dev, (const int32_t *)g_dev, (int32_t *)r_dev, B, L, D,
-                                     workspace, workspace_bytes, stream);
-            break;
+    for (int64_t c = 0; c < chunks; ++c) {
+        const int64_t b0 = c * B / chunks, b1 = (c + 1) * B / chunks;
+        st = from_host_chunk(dtype, v_host, g_host, r_host, v_dev, g_dev, r_dev, b0, b1 - b0, L, D, workspace,
+                             workspace_bytes, pipe->up, pipe->down, pipe->handoff);
+        if (st != CC_OK) return st;
     }
-    if (st != CC_OK) return st;
-    if (cudaMemcpyAsync(r_host, r_dev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+    if (cudaEventRecord(pipe->done, pipe->down) != cudaSuccess || cudaStreamWaitEvent(s, pipe->done, 0) != cudaSuccess) {
         cudaGetLastError();
         return CC_ERR_CUDA;
     }

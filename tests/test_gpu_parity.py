@@ -270,11 +270,16 @@ def test_leakage_f32_measured():
 
 
 def test_from_host_matches_device_path():
+    """Host buffers in and out (batches pipelined in pieces over two streams
+    when B >= 2; B = 5 splits unevenly, B = 1 takes the single-stream path)."""
     import torch
     import spectral_sequence_mixing_b200 as ssm
+    rng = np.random.Generator(np.random.PCG64(2))
     for dtype, (v, g) in (("f32", _rand_float((2, 1000, 12), 1)),
-                          ("i32", tuple(np.random.Generator(np.random.PCG64(2)).integers(-128, 128, (2, 700, 8))
-                                        .astype(np.int32) for _ in range(2)))):
+                          ("f32", _rand_float((5, 300, 8), 3)),
+                          ("f32", _rand_float((1, 5000, 4), 4)),
+                          ("i32", tuple(rng.integers(-128, 128, (2, 700, 8)).astype(np.int32) for _ in range(2))),
+                          ("i32", tuple(rng.integers(-128, 128, (7, 100, 4)).astype(np.int32) for _ in range(2)))):
         tv, tg = to_dev(v, dtype), to_dev(g, dtype)
         ref = from_dev(ssm.causal_conv(tv, tg), dtype)
         hv = torch.from_numpy(v).pin_memory()
