@@ -37,8 +37,14 @@ import workloads  # noqa: E402
 
 METRIC = "causal FFT-conv GB/s and (B*D*L)/s at 1 B200; % of HBM roofline"
 L2_BYTES = 126 * 2 ** 20
-# the device code of the kernels (api.cu holds host code and table storage)
-KERNEL_SOURCES = ["fftconv_fused.cuh", "fft_reg.cuh", "tma.cuh", "bigconv.cuh", "ntt.cuh", "transpose.cuh", "configs.cuh"]
+# the device code each kernel is built from (api.cu holds host code and table storage)
+_FUSED_SOURCES = ["fftconv_fused.cuh", "fft_reg.cuh", "tma.cuh", "configs.cuh"]
+KERNEL_SOURCES = {
+    "fftconv_fused_kernel": _FUSED_SOURCES,
+    "bigrow_group_kernel": ["bigconv.cuh"] + _FUSED_SOURCES,
+    "bigconv_kernel": ["bigconv.cuh", "transpose.cuh"] + _FUSED_SOURCES,
+    "ntt_conv_kernel": ["ntt.cuh"],
+}
 
 
 def parse_args():
@@ -87,9 +93,10 @@ def throughput(units_per_rank: int, world: int, steps: int, ms: float, bytes_per
     return units / (ms * 1e-3), units * bytes_per_unit / (ms * 1e-3) / 1e9
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str) -> str:
+    """sha256 (16 hex digits) of the device sources `kernel` is built from."""
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_SOURCES.get(kernel, []):
         p = os.path.join(ROOT, "spectral_sequence_mixing_b200", "csrc", f)
         if os.path.exists(p):
             h.update(open(p, "rb").read())
@@ -115,7 +122,7 @@ def recorded_counters(workload: str, kernel: str):
     for line in open(p):
         f = line.split()
         if len(f) == 5 and not line.startswith("#") and f[0] == workload and f[1] == kernel:
-            if f[2] != kernel_source_hash():
+            if f[2] != kernel_source_hash(kernel):
                 return None, None
             return float(f[3]), float(f[4])
     return None, None

@@ -41,7 +41,7 @@ constexpr int64_t kNttMaxL = kNttN / 2;
 constexpr int kNttThreads = 512;
 constexpr int kNttWordsPerArray = kNttN + kNttN / 32;
 constexpr int kNttGroup = 4;  // channels per cluster (4 x 4 bytes per time step)
-constexpr size_t kNttSmemBytes = 2u * kNttWordsPerArray * 4u;
+constexpr size_t kNttSmemBytes = 2u * kNttWordsPerArray * 4u + 2u * 32 * 32 * 8;
 
 struct NttParams {
     uint32_t p, w, winv, ninv, pinv, r2;
@@ -178,7 +178,13 @@ __global__ void __launch_bounds__(kNttThreads, 1)
     extern __shared__ uint32_t nsm[];
     uint32_t *sv = nsm;
     uint32_t *sg = nsm + kNttWordsPerArray;
+    uint2 *stf2 = reinterpret_cast<uint2 *>(nsm + 2 * kNttWordsPerArray);  // pass-2 twiddles, forward
+    uint2 *sti2 = stf2 + 32 * 32;                                            // and inverse
     const int tid = threadIdx.x;
+    for (int i = tid; i < 32 * 32; i += kNttThreads) {
+        stf2[i] = g_ntf2[i];
+        sti2[i] = g_nti2[i];
+    }
     cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int grp = blockIdx.x / kNttGroup;
@@ -267,7 +273,7 @@ __global__ void __launch_bounds__(kNttThreads, 1)
             ntt_dif<32, 32>(x);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const uint2 w = g_ntf2[i * 32 + nC];
+                const uint2 w = stf2[i * 32 + nC];
                 s[pad_idx(a * 1024 + i * 32 + nC)] = i == 0 ? x[i] : n_mul_shoup(x[i], w.x, w.y);
             }
         }
@@ -301,7 +307,7 @@ __global__ void __launch_bounds__(kNttThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const uint32_t val = sv[pad_idx(a * 1024 + i * 32 + nC)];
-            const uint2 w = g_nti2[i * 32 + nC];
+            const uint2 w = sti2[i * 32 + nC];
             x[i] = i == 0 ? val : n_mul_shoup(val, w.x, w.y);
         }
         ntt_dit_inv<32, 32>(x);
