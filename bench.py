@@ -112,20 +112,21 @@ def measured_peaks():
 
 
 def recorded_counters(workload: str, kernel: str):
-    """(DRAM bytes read + write, FP32 lane operations) per launch of `kernel`
-    on the full-size `workload`, from profiles/kernel_counters.txt (lines:
-    workload kernel source_hash dram_bytes fp32_lane_ops), if they were taken
-    on the current kernel sources; else (None, None)."""
+    """(DRAM bytes read + write, ALU lane operations, their pipe "fp32" or
+    "imad") per launch of `kernel` on the full-size `workload`, from
+    profiles/kernel_counters.txt (lines: workload kernel source_hash
+    dram_bytes alu_lane_ops pipe), if they were taken on the current kernel
+    sources; else (None, None, None)."""
     p = os.path.join(ROOT, "profiles", "kernel_counters.txt")
     if not os.path.exists(p):
-        return None, None
+        return None, None, None
     for line in open(p):
         f = line.split()
-        if len(f) == 5 and not line.startswith("#") and f[0] == workload and f[1] == kernel:
+        if len(f) == 6 and not line.startswith("#") and f[0] == workload and f[1] == kernel:
             if f[2] != kernel_source_hash(kernel):
-                return None, None
-            return float(f[3]), float(f[4])
-    return None, None
+                return None, None, None
+            return float(f[3]), float(f[4]), f[5]
+    return None, None, None
 
 
 class ClockSampler:
@@ -392,7 +393,8 @@ def run_ours(args, rank, world, local):
         kernel = "bigconv_kernel (two-pass step: 2 transposes in, 1 out)"
     per_launch_bytes = bytes_per_step // 2 if args.path == "bwd" else bytes_per_step
     achieved = bytes_per_step / (ms_per_step * 1e-3) / 1e9
-    traffic, fp32_ops = (None, None) if (args.shape or args.path != "fwd") else recorded_counters(w.name, kernel)
+    traffic, alu_ops, alu_pipe = ((None, None, None) if (args.shape or args.path != "fwd")
+                                  else recorded_counters(w.name, kernel))
     clocks = clk.report()
     line = {
         "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -413,16 +415,19 @@ def run_ours(args, rank, world, local):
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clocks,
     }
-    if fp32_ops and launches_per_step == 1:
-        # the transform kernels are bound by FP32 issue, not by HBM: executed
-        # FP32 lane operations (ncu, same sources) per launch against
-        # 148 SMs x 128 FP32 lanes x the SM clock sampled during the run
+    if alu_ops and launches_per_step == 1:
+        # the transform kernels are bound by ALU issue, not by HBM: executed
+        # lane operations of their busiest pipe (ncu, same sources) per launch
+        # against 148 SMs x lanes/clk of that pipe (FP32 128, IMAD 64) x the
+        # SM clock sampled during the run
+        lanes = {"fp32": 128, "imad": 64}[alu_pipe]
         sm_hz = clocks["sm_mhz"] * 1e6 if clocks and clocks.get("sm_mhz") else 1.965e9
-        alu_peak = 148 * 128 * sm_hz / 1e9
-        alu_achieved = fp32_ops / (ms_per_step * 1e-3) / 1e9
-        line["alu_roofline"] = {"bound": "alu", "achieved": alu_achieved, "peak": alu_peak, "unit": "G FP32 lane-op/s",
-                                "frac": alu_achieved / alu_peak, "fp32_lane_ops_per_launch": fp32_ops,
-                                "peak_source": "148 SMs x 128 FP32 lanes/clk x sampled SM clock"}
+        alu_peak = 148 * lanes * sm_hz / 1e9
+        alu_achieved = alu_ops / (ms_per_step * 1e-3) / 1e9
+        line["alu_roofline"] = {"bound": "alu", "pipe": alu_pipe, "achieved": alu_achieved, "peak": alu_peak,
+                                "unit": f"G {alu_pipe.upper()} lane-op/s", "frac": alu_achieved / alu_peak,
+                                "lane_ops_per_launch": alu_ops,
+                                "peak_source": f"148 SMs x {lanes} lanes/clk x sampled SM clock"}
     if args.path != "fwd":  # the host-buffer leg and CPU baseline describe the forward line only
         line.pop("e2e")
         args.no_cpu_baseline = True
