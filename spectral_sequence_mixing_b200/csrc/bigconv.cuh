@@ -225,6 +225,7 @@ __global__ void __launch_bounds__(T, MINB)
         }
     }
     float alpha;
+    bool live;  // false: v or g is all zero, the row is exactly zero
     {
         float2 *red = head + HEAD;  // [T/32] warp partials, then [T/32] = CTA total
 #pragma unroll
@@ -253,6 +254,7 @@ __global__ void __launch_bounds__(T, MINB)
             }
         }
         alpha = balance_scale(tot.x, tot.y);
+        live = tot.x > 0.f && tot.y > 0.f;
     }
 
     // ---- forward pass 0: odd-frequency R0-point DFT over n0 of z = v + i alpha g
@@ -316,7 +318,7 @@ __global__ void __launch_bounds__(T, MINB)
 
     // ---- inverse pass 0: twiddle, inverse R0-point DFT (outputs n0 < R0/2), untwist, store t < L
     {
-        const float s = 1.f / (4.f * (float)S * alpha);
+        const float s = live ? 1.f / (4.f * (float)S * alpha) : 0.f;
 #pragma unroll 1
         for (int c = tid; c < C::COLS0; c += T) {
             const int n = rank * C::COLS0 + c;
@@ -472,6 +474,7 @@ __global__ void __launch_bounds__(T, MINB)
         }
     }
     float alpha;
+    bool live;  // false: v or g is all zero, the row is exactly zero
     {
         float2 *red = head + HEAD;
 #pragma unroll
@@ -488,6 +491,7 @@ __global__ void __launch_bounds__(T, MINB)
             tot.y += red[w].y;
         }
         alpha = balance_scale(tot.x, tot.y);
+        live = tot.x > 0.f && tot.y > 0.f;
     }
     auto tw0 = [&](int k0, int n) -> float2 {
         const float2 a = __ldg(tw + C::T0A + k0 * C::Q0 + (n % C::Q0));
@@ -544,7 +548,7 @@ __global__ void __launch_bounds__(T, MINB)
     // ---- inverse pass 0: twiddle, inverse R0-point DFT (outputs n0 < R0/2),
     // untwist; r_t (t < L) is left in slot t of the same column
     {
-        const float sc = 1.f / (4.f * (float)S * alpha);
+        const float sc = live ? 1.f / (4.f * (float)S * alpha) : 0.f;
 #pragma unroll 1
         for (int n = tid; n < SL; n += T) {
             float2 x[R0];

@@ -256,7 +256,8 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
     IO *sv = reinterpret_cast<IO *>(reinterpret_cast<char *>(smem_raw) + C::SOFF);
     IO *sg = sv + LMAX * ROWS;
     float2 *red = reinterpret_cast<float2 *>(sg + LMAX * ROWS);  // [NWARPS][ROWS] partial norms
-    float *alpha_row = reinterpret_cast<float *>(red + C::NWARPS * ROWS);  // [ROWS] balance scale
+    // [ROWS] output scale 1/(4 N alpha), 0 for a row whose v or g is all zero; [ROWS] unused
+    float *alpha_row = reinterpret_cast<float *>(red + C::NWARPS * ROWS);
     float2 *rot = reinterpret_cast<float2 *>(alpha_row + 2 * ROWS);       // [2h+s][H+1]
     uint64_t *bar = reinterpret_cast<uint64_t *>(rot + 4 * (H + 1));      // staging-complete barrier
     const int tid = threadIdx.x;
@@ -379,7 +380,9 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
                 tot.y += red[w * ROWS + c].y;
             }
             const float alpha = balance_scale(tot.x, tot.y);
-            if (tid < ROWS) alpha_row[c] = alpha;
+            // a stream that is all zero makes the row exactly zero (the transform
+            // would otherwise spread the other stream's rounding over it)
+            if (tid < ROWS) alpha_row[c] = (tot.x > 0.f && tot.y > 0.f) ? 1.f / (4.f * (float)N * alpha) : 0.f;
 
             // x[n1] = z[n2 + N2 n1] * omega_2N1^((2e+1) n1), in bit-reversed slots.
             // e is warp-uniform: the twist comes from a constant table at a
@@ -505,7 +508,7 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
             // combine the two parities h: lane h keeps m in [h H/2, (h+1) H/2)
             const int d = d0 + c;
             const bool dok = d < D;
-            const float sc = 1.f / (4.f * (float)N * alpha_row[c]);
+            const float sc = alpha_row[c];
             const int t0 = 2 * m2 + N2 * (H * s + (H / 2) * h);
             const int64_t dir = rev_out ? -1 : 1;  // output time direction
             IO *rp = r + boff + d + (int64_t)(rev_out ? L - 1 - t0 : t0) * D;

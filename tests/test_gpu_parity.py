@@ -250,6 +250,48 @@ def _leak(dtype, v, g, t_c, scale, seed):
     return float(np.abs(r1[:, : t_c + 1, :].astype(np.float64) - r0[:, : t_c + 1, :]).max())
 
 
+# one representative shape per kernel: fused, channel groups, cluster rows (the
+# binding takes the two-pass path), and the NTT
+DEGENERATE_CASES = [("f32", (2, 1000, 5)), ("bf16", (1, 700, 8)), ("f32", (1, 3000, 9)), ("bf16", (2, 4096, 8)),
+                    ("f32", (1, 5000, 3)), ("i32", (2, 3000, 5))]
+
+
+@pytest.mark.parametrize("dtype,shape", DEGENERATE_CASES, ids=lambda c: str(c))
+def test_degenerate_inputs(dtype, shape):
+    """Zero inputs give exactly zero; an impulse v = delta_0 returns g (and
+    g = delta_0 returns v): exactly for the NTT, within 1e-5 (fp32) or 2e-2
+    (bf16) of max|g| for the float paths (the float error is spread over the
+    row, so a per-element bound cannot hold where |g_t| is tiny)."""
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    B, L, D = shape
+    rng = np.random.Generator(np.random.PCG64(L + D))
+    if dtype == "i32":
+        x = rng.integers(-128, 128, shape).astype(np.int32)
+    else:
+        x = rng.standard_normal(shape).astype(np.float32)
+        if dtype == "bf16":
+            x = workloads.bf16_round(x)
+    zero = np.zeros_like(x)
+    delta = np.zeros_like(x)
+    delta[:, 0, :] = 1 if dtype != "bf16" else workloads.bf16_round(np.ones((B, D), np.float32))
+
+    def conv(a, b):
+        r = ssm.causal_conv(to_dev(a, dtype), to_dev(b, dtype))
+        torch.cuda.synchronize()
+        return as_f32(from_dev(r, dtype), dtype) if dtype != "i32" else from_dev(r, dtype)
+
+    assert not np.any(conv(zero, zero)) and not np.any(conv(zero, x)) and not np.any(conv(x, zero))
+    for a, b in ((delta, x), (x, delta)):
+        r = conv(a, b)
+        if dtype == "i32":
+            assert np.array_equal(r, x)
+        else:
+            xf = as_f32(x, dtype)
+            tol = (F32_TOL if dtype == "f32" else BF16_TOL) * np.abs(xf).max()
+            assert np.abs(r - xf).max() <= tol
+
+
 def test_leakage_ntt_is_exactly_zero():
     rng = np.random.Generator(np.random.PCG64(5))
     v = rng.integers(-128, 128, (2, 8192, 8)).astype(np.int32)
