@@ -147,11 +147,23 @@ class ClockSampler:
             import pynvml
             pynvml.nvmlInit()
             self._nv = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self._h = self._handle(pynvml, index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
         except Exception:
             self._nv = None
         self._t = threading.Thread(target=self._run, daemon=True)
+
+    @staticmethod
+    def _handle(pynvml, index: int):
+        """NVML handle of CUDA device `index`, found by PCI address (CUDA and
+        NVML may number devices differently); by index if that fails."""
+        try:
+            import torch
+            pr = torch.cuda.get_device_properties(index)
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(index)
 
     def _run(self):
         while not self._stop.is_set():
