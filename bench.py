@@ -38,11 +38,11 @@ import workloads  # noqa: E402
 METRIC = "causal FFT-conv GB/s and (B*D*L)/s at 1 B200; % of HBM roofline"
 L2_BYTES = 126 * 2 ** 20
 # the device code each kernel is built from (api.cu holds host code and table storage)
-_FUSED_SOURCES = ["fftconv_fused.cuh", "fft_reg.cuh", "tma.cuh", "configs.cuh"]
+_FUSED_SOURCES = ["fftconv_fused.cuh", "fft_reg.cuh", "tma.cuh", "configs_fused.cuh"]
 KERNEL_SOURCES = {
     "fftconv_fused_kernel": _FUSED_SOURCES,
-    "bigrow_group_kernel": ["bigconv.cuh"] + _FUSED_SOURCES,
-    "bigconv_kernel": ["bigconv.cuh", "transpose.cuh"] + _FUSED_SOURCES,
+    "bigrow_group_kernel": ["bigconv.cuh", "configs_rows.cuh"] + _FUSED_SOURCES,
+    "bigconv_kernel": ["bigconv.cuh", "configs_rows.cuh", "transpose.cuh"] + _FUSED_SOURCES,
     "ntt_conv_kernel": ["ntt.cuh"],
 }
 

@@ -32,6 +32,7 @@ namespace ccv {
 __device__ float2 g_tw_s[CfgS<float>::TW_SIZE];
 __device__ float2 g_tw_m[CfgM<float>::TW_SIZE];
 
+__device__ float2 g_tw_bm[BigM<float>::TW_SIZE];
 __device__ float2 g_tw_bl[BigL<float>::TW_SIZE];
 __device__ float2 g_tw_bx[BigX<float>::TW_SIZE];
 
@@ -98,8 +99,9 @@ static bool g_init_done[128];
 
 // Per device: SM count and, per kernel instantiation, resident CTAs per SM.
 static int g_num_sms[128];
-// Per device: device addresses of the twiddle tables (small, mid, one-CTA rows, cluster rows).
-static void *g_tw_addr[128][4];
+// Per device: device addresses of the twiddle tables (fused N = 512, 2048; one-CTA
+// rows N = 8192; cluster rows; one-CTA rows N = 4096).
+static void *g_tw_addr[128][5];
 
 template <class Cfg, typename IO, int MINB>
 static cudaError_t set_smem_attr() {
@@ -136,6 +138,10 @@ static cudaError_t ensure_init(int dev) {
         if ((e = cudaMemcpyToSymbol(g_tw_m, t.data(), t.size() * sizeof(float2))) != cudaSuccess) return e;
     }
     {
+        auto t = big_twiddles<BigM<float>>();
+        if ((e = cudaMemcpyToSymbol(g_tw_bm, t.data(), t.size() * sizeof(float2))) != cudaSuccess) return e;
+    }
+    {
         auto t = big_twiddles<BigL<float>>();
         if ((e = cudaMemcpyToSymbol(g_tw_bl, t.data(), t.size() * sizeof(float2))) != cudaSuccess) return e;
     }
@@ -143,6 +149,8 @@ static cudaError_t ensure_init(int dev) {
         auto t = big_twiddles<BigX<float>>();
         if ((e = cudaMemcpyToSymbol(g_tw_bx, t.data(), t.size() * sizeof(float2))) != cudaSuccess) return e;
     }
+    if ((e = set_big_attr<BigM<float>, float, kMinbBigM>()) != cudaSuccess) return e;
+    if ((e = set_big_attr<BigM<__nv_bfloat16>, __nv_bfloat16, kMinbBigM>()) != cudaSuccess) return e;
     if ((e = set_big_attr<BigL<float>, float, kMinbBigL>()) != cudaSuccess) return e;
     if ((e = set_big_attr<BigL<__nv_bfloat16>, __nv_bfloat16, kMinbBigL>()) != cudaSuccess) return e;
     if ((e = set_big_attr<BigX<float>, float, kMinbBigX>()) != cudaSuccess) return e;
@@ -157,6 +165,7 @@ static cudaError_t ensure_init(int dev) {
     if ((e = cudaGetSymbolAddress(&g_tw_addr[dev][1], g_tw_m)) != cudaSuccess) return e;
     if ((e = cudaGetSymbolAddress(&g_tw_addr[dev][2], g_tw_bl)) != cudaSuccess) return e;
     if ((e = cudaGetSymbolAddress(&g_tw_addr[dev][3], g_tw_bx)) != cudaSuccess) return e;
+    if ((e = cudaGetSymbolAddress(&g_tw_addr[dev][4], g_tw_bm)) != cudaSuccess) return e;
     g_init_done[dev] = true;
     return cudaSuccess;
 }
@@ -410,6 +419,8 @@ static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t 
         return launch_fused<CfgS<IO>, kMinbS>(v, g, r, B, L, D, (const float2 *)tws[0], s, dev, rev);
     if (L <= CfgM<IO>::LMAX)
         return launch_fused<CfgM<IO>, kMinbM>(v, g, r, B, L, D, (const float2 *)tws[1], s, dev, rev);
+    if (L <= BigM<IO>::LMAX)
+        return launch_group<BigM<IO>, kMinbBigM>(v, g, r, B, L, D, (const float2 *)tws[4], s, rev);
     if (L <= BigL<IO>::LMAX)
         return launch_group<BigL<IO>, kMinbBigL>(v, g, r, B, L, D, (const float2 *)tws[2], s, rev);
     if (L <= BigX<IO>::LMAX) {
