@@ -320,8 +320,8 @@ static int launch_fused(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, i
     memset(&tmv, 0, sizeof(tmv));
     memset(&tmg, 0, sizeof(tmg));
     const bool tma = Cfg::TMA_OK &&
-                     encode_btd_map<IO>(&tmv, v, B, L, D, Cfg::ROWS, Cfg::BOXT) &&
-                     encode_btd_map<IO>(&tmg, g, B, L, D, Cfg::ROWS, Cfg::BOXT);
+                     encode_btd_map<IO>(&tmv, v, B, L, D, Cfg::SW, Cfg::BOXT) &&
+                     encode_btd_map<IO>(&tmg, g, B, L, D, Cfg::SW, Cfg::BOXT);
     kern<<<(unsigned)grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(v, g, r, (int)L, (int)D, (int)groups, (int)tiles,
                                                               vec ? 1 : 0, rev, tw, tmv, tmg, tma ? 1 : 0);
     return cudaGetLastError() == cudaSuccess ? CC_OK : CC_ERR_CUDA;

@@ -106,7 +106,11 @@ struct FusedCfg {
     static constexpr size_t XBYTES = (size_t)ROWS * SC * 8;
     static constexpr size_t HBYTES = ((size_t)ROWS * HP * HEAD * 4 + 15) / 16 * 16;  // [ROWS][HP][HEAD] partial sums
     // staging: [LMAX][ROWS] elements of IO for v, then for g
-    static constexpr size_t SBYTES = (size_t)2 * LMAX * ROWS * sizeof(IO);
+    // staged channels per time step: the tile's ROWS, widened to a whole
+    // 16-byte TMA box row (bf16 tiles of 4 channels stage 8; the tile's
+    // channels sit at offset d0 % SW of the row)
+    static constexpr int SW = ROWS * (int)sizeof(IO) >= 16 ? ROWS : 16 / (int)sizeof(IO);
+    static constexpr size_t SBYTES = (size_t)2 * LMAX * SW * sizeof(IO);
     // norm partials [NWARPS][ROWS] float2, per-row scale [ROWS] float (padded),
     // rotations [(2h+s)][H+1] float2 (padded so the four (h, s) lane groups hit distinct banks)
     static constexpr size_t RBYTES = (size_t)(NWARPS * ROWS) * 8 + (size_t)ROWS * 8 + (size_t)4 * (N2 / 2 + 1) * 8;
@@ -114,8 +118,8 @@ struct FusedCfg {
     static constexpr size_t SOFF = (XBYTES + HBYTES + 127) / 128 * 128;
     // + one mbarrier (8 bytes, padded)
     static constexpr size_t SMEM_BYTES = SOFF + SBYTES + RBYTES + 16;
-    // TMA staging: boxes of [BOXT t][ROWS d]; a box row must be a multiple of 16 bytes
-    static constexpr bool TMA_OK = (ROWS * sizeof(IO)) % 16 == 0;
+    // TMA staging: boxes of [BOXT t][SW d]; a box row must be a multiple of 16 bytes
+    static constexpr bool TMA_OK = (SW * sizeof(IO)) % 16 == 0;
     static constexpr int BOXT = LMAX < 256 ? LMAX : 256;
     static constexpr int NBOX = LMAX / BOXT;
     static constexpr unsigned STAGE_BYTES = (unsigned)SBYTES;
@@ -137,7 +141,8 @@ struct FusedCfg {
     static constexpr int CHUNK = CH < 16 ? CH : 16;
     static constexpr int NCHUNK = CH / CHUNK;
     static_assert(CH % CHUNK == 0 && (CHUNK == 4 || CHUNK == 8 || CHUNK == 16), "staging chunking");
-    static_assert((LMAX * CH) % 128 == 0 && LMAX % BOXT == 0, "staging boxes must stay 128-byte aligned");
+    static_assert(SW % ROWS == 0 && (LMAX * SW * sizeof(IO)) % 128 == 0 && LMAX % BOXT == 0,
+                  "staging boxes must stay 128-byte aligned");
 };
 
 // X' = -i (Zk + conj Zm)(Zk - conj Zm) = 4 V_k G_k for z = v + i g, Zm = mirror bin.
@@ -184,7 +189,8 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 template <class C, typename IO>
 __device__ __forceinline__ void stage_tile(const IO *__restrict__ v, const IO *__restrict__ g, IO *sv, IO *sg,
                                            int64_t boff, int d0, int L, int D, bool vec) {
-    constexpr int ROWS = C::ROWS;
+    constexpr int ROWS = C::ROWS, SW = C::SW;
+    const int coff = d0 % SW;  // the tile's channels within a staged row
     const int tid = threadIdx.x;
     const IO *vb = v + boff + d0;
     const IO *gb = g + boff + d0;
@@ -193,8 +199,8 @@ __device__ __forceinline__ void stage_tile(const IO *__restrict__ v, const IO *_
         for (int e = tid; e < L * C::NCHUNK; e += C::THREADS) {
             const int t = e / C::NCHUNK, q = e - t * C::NCHUNK;
             const int64_t o = (int64_t)t * D + q * EPC;
-            IO *dv = sv + t * ROWS + q * EPC;
-            IO *dg = sg + t * ROWS + q * EPC;
+            IO *dv = sv + t * SW + coff + q * EPC;
+            IO *dg = sg + t * SW + coff + q * EPC;
             if (C::CHUNK == 16) {
                 cp_async16(dv, vb + o);
                 cp_async16(dg, gb + o);
@@ -213,11 +219,11 @@ __device__ __forceinline__ void stage_tile(const IO *__restrict__ v, const IO *_
             if (c < nc) {
                 const int64_t o = (int64_t)t * D + c;
                 if (sizeof(IO) == 4) {
-                    cp_async4(sv + e, vb + o);
-                    cp_async4(sg + e, gb + o);
+                    cp_async4(sv + t * SW + coff + c, vb + o);
+                    cp_async4(sg + t * SW + coff + c, gb + o);
                 } else {
-                    sv[e] = IO_t<IO>::ld(vb + o);
-                    sg[e] = IO_t<IO>::ld(gb + o);
+                    sv[t * SW + coff + c] = IO_t<IO>::ld(vb + o);
+                    sg[t * SW + coff + c] = IO_t<IO>::ld(gb + o);
                 }
             }
         }
@@ -254,21 +260,23 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
     float2 *xs = reinterpret_cast<float2 *>(smem_raw);
     float *hres = reinterpret_cast<float *>(xs + ROWS * SC);  // [ROWS][HP][HEAD]: partial direct sums, t < HEAD
     IO *sv = reinterpret_cast<IO *>(reinterpret_cast<char *>(smem_raw) + C::SOFF);
-    IO *sg = sv + LMAX * ROWS;
-    float2 *red = reinterpret_cast<float2 *>(sg + LMAX * ROWS);  // [NWARPS][ROWS] partial norms
+    constexpr int SW = C::SW;
+    IO *sg = sv + LMAX * SW;
+    float2 *red = reinterpret_cast<float2 *>(sg + LMAX * SW);  // [NWARPS][ROWS] partial norms
     // [ROWS] output scale 1/(4 N alpha), 0 for a row whose v or g is all zero; [ROWS] unused
     float *alpha_row = reinterpret_cast<float *>(red + C::NWARPS * ROWS);
     float2 *rot = reinterpret_cast<float2 *>(alpha_row + 2 * ROWS);       // [2h+s][H+1]
     uint64_t *bar = reinterpret_cast<uint64_t *>(rot + 4 * (H + 1));      // staging-complete barrier
     const int tid = threadIdx.x;
-    // v at time t (0 <= t < LMAX) of row c from the staging: v_t, or v_{L-1-t} (0 for t >= L)
-    auto v_at = [&](int t, int c) -> float {
+    // v at time t (0 <= t < LMAX) of staged channel cc (tile row + offset in
+    // the staged row): v_t, or v_{L-1-t} (0 for t >= L)
+    auto v_at = [&](int t, int cc) -> float {
         if constexpr (REVA) {
             const int tr = L - 1 - t;
-            const float x = IO_t<IO>::cvt(sv[max(tr, 0) * ROWS + c]);
+            const float x = IO_t<IO>::cvt(sv[max(tr, 0) * SW + cc]);
             return tr >= 0 ? x : 0.f;
         } else {
-            return IO_t<IO>::cvt(sv[t * ROWS + c]);
+            return IO_t<IO>::cvt(sv[t * SW + cc]);
         }
     };
     const bool tma = C::TMA_OK && use_tma && (smem_u32(sv) & 127) == 0;
@@ -282,8 +290,8 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
                 mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
 #pragma unroll
                 for (int k = 0; k < C::NBOX; ++k) {
-                    tma_load_3d(sv + k * C::BOXT * ROWS, &tmv, d0, k * C::BOXT, b, bar);
-                    tma_load_3d(sg + k * C::BOXT * ROWS, &tmg, d0, k * C::BOXT, b, bar);
+                    tma_load_3d(sv + k * C::BOXT * SW, &tmv, d0 - d0 % SW, k * C::BOXT, b, bar);
+                    tma_load_3d(sg + k * C::BOXT * SW, &tmg, d0 - d0 % SW, k * C::BOXT, b, bar);
                 }
             }
         } else {
@@ -301,7 +309,7 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
         if (tid == 0) mbar_init(bar, 1);
     } else {
         // staging beyond L is never written by the copies: zero it once so loads need no bounds test
-        for (int i = L * ROWS + tid; i < LMAX * ROWS; i += THREADS) {
+        for (int i = L * SW + tid; i < LMAX * SW; i += THREADS) {
             sv[i] = IO(0.f);
             sg[i] = IO(0.f);
         }
@@ -339,12 +347,13 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
         {
             const int e = tid / (ROWS * N2);  // warp-uniform
             const int c = tid % ROWS, n2 = (tid / ROWS) % N2;
+            const int coff = d0 % SW;  // the tile's channels within a staged row
             float2 zr[N2];
             float nv = 0.f, ng = 0.f;
 #pragma unroll
             for (int n1 = 0; n1 < N2; ++n1) {
                 const int t = n2 + N2 * n1;
-                const float2 zv = make_float2(v_at(t, c), IO_t<IO>::cvt(sg[t * ROWS + c]));
+                const float2 zv = make_float2(v_at(t, coff + c), IO_t<IO>::cvt(sg[t * SW + coff + c]));
                 zr[n1] = zv;
                 nv = fmaf(zv.x, zv.x, nv);
                 ng = fmaf(zv.y, zv.y, ng);
@@ -354,8 +363,8 @@ __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)
             {
                 constexpr int HP = C::HP, JP = HEAD / HP;
                 const int w = tid >> 5, hc = w % ROWS, hp = w / ROWS, lt = tid & 31;
-                const float vt = v_at(lt, hc);
-                const float gt = IO_t<IO>::cvt(sg[lt * ROWS + hc]);
+                const float vt = v_at(lt, coff + hc);
+                const float gt = IO_t<IO>::cvt(sg[lt * SW + coff + hc]);
                 float acc = 0.f;
 #pragma unroll
                 for (int jj = 0; jj < JP; ++jj) {

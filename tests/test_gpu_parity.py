@@ -27,10 +27,11 @@ def _rand_float(shape, seed, scale_g=1.0):
 # shapes spanning several tiles with ragged tails in L (vs N/2) and D (vs the channel tile)
 # (D * element size a multiple of 16 bytes selects the TMA staging: (3, 200, 36)
 # and (2, 130, 24) end in a partial channel group the copy engine zero-fills,
-# (1, 513, 4) and (2, 700, 20) have many zero-filled time steps past L)
+# (1, 513, 4) and (2, 700, 20) have many zero-filled time steps past L; in
+# bf16, (2, 1000, 16) and (1, 513, 8) stage 8-channel rows for 4-channel tiles)
 FLOAT_SHAPES = [(1, 1, 1), (1, 2, 3), (1, 3, 2), (2, 31, 5), (1, 32, 4), (1, 33, 7), (3, 200, 19), (1, 256, 8),
                 (2, 257, 9), (2, 513, 5), (2, 1000, 37), (1, 1024, 12), (3, 200, 36), (2, 130, 24), (1, 513, 4),
-                (2, 700, 20)]
+                (2, 700, 20), (2, 1000, 16), (1, 513, 8)]
 
 
 @pytest.mark.parametrize("shape", FLOAT_SHAPES, ids=lambda s: "x".join(map(str, s)))
