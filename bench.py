@@ -93,13 +93,23 @@ def throughput(units_per_rank: int, world: int, steps: int, ms: float, bytes_per
     return units / (ms * 1e-3), units * bytes_per_unit / (ms * 1e-3) / 1e9
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments and whitespace (edits to comments do not
+    change the code a kernel is compiled from)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return re.sub(r"\s+", "", text)
+
+
 def kernel_source_hash(kernel: str) -> str:
-    """sha256 (16 hex digits) of the device sources `kernel` is built from."""
+    """sha256 (16 hex digits) of the device code `kernel` is built from: its
+    sources with comments and whitespace removed."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES.get(kernel, []):
         p = os.path.join(ROOT, "spectral_sequence_mixing_b200", "csrc", f)
         if os.path.exists(p):
-            h.update(open(p, "rb").read())
+            h.update(_code_only(open(p).read()).encode())
     return h.hexdigest()[:16]
 
 

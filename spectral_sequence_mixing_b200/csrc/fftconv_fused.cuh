@@ -42,9 +42,12 @@
 // Pipeline: each CTA loops over tiles; the next tile's v and g are copied
 // into a staging buffer while the current tile runs F3 and I3.  The copy is a
 // handful of TMA boxes issued by one thread (completion counted on an
-// mbarrier; the copy engine zero-fills t >= L and d >= D) whenever a tile row
-// is a multiple of 16 bytes and the tensors allow a tensor map; otherwise the
-// threads issue cp.async pieces.
+// mbarrier; the copy engine zero-fills t >= L and d >= D) whenever the tensors
+// allow a tensor map (16-byte aligned base and row pitch); a staged row is
+// widened to 16 bytes where the tile's is narrower (bf16 tiles of 4 channels
+// stage 8 and read their half).  Otherwise the threads issue cp.async pieces.
+// The backward pass reads v reversed in time: the staging keeps natural
+// order and the reversal happens on the shared-memory reads.
 #pragma once
 
 #include <cuda_bf16.h>
