@@ -475,3 +475,12 @@ def test_decode_step_matches_oracle(case, dtype):
     assert n_bad == 0, f"{n_bad} violations, worst ratio {worst:.3g}"
     if dtype == "f32":  # fp64 accumulation, one rounding to float at the end
         assert np.all(np.abs(got.reshape(-1) - ref) <= 6.0e-8 * np.abs(ref) + 1e-12 * den)
+
+
+def test_accuracy_report_runs():
+    """The accuracy / leakage report (tests/accuracy_report.py) on the small
+    workloads: no bound violation, the directly summed head does not leak."""
+    import accuracy_report
+    for line in accuracy_report.main(["--workloads", "tiny_f32,small_f32"]):
+        assert line["accuracy"]["violations"] == 0
+        assert line["leakage"]["31"]["max_abs"] == 0.0
