@@ -20,6 +20,10 @@ in Convolutional Sequence Modeling", abstract) is exact, so its oracle is the
 same sum in int64; ``centered_mod`` gives what an exact mod-p transform returns
 when the true sum does not fit in (-p/2, p/2).
 
+The submodule ``oracle.mhf_gate`` adds the gate stream of the same block
+(sigmoid and the head-grouped causal Conv1d_G2, float64 numpy) and composes it
+with this sum; its pins are in tests/test_oracle_mhf_pins.py.
+
 Pins (tests/test_oracle_pins.py): hand-computed fixtures in tests/golden/,
 delta inputs, closed-form sums, numpy.convolve on single rows, an fp64 FFT
 convolution (independent algorithm), commutativity, bilinearity, shift
