@@ -44,7 +44,9 @@ KERNEL_SOURCES = {
     "bigrow_group_kernel": ["bigconv.cuh", "configs_rows.cuh"] + _FUSED_SOURCES,
     "bigconv_kernel": ["bigconv.cuh", "configs_rows.cuh", "transpose.cuh"] + _FUSED_SOURCES,
     "ntt_conv_kernel": ["ntt.cuh"],
+    "mhf_gate_kernel": ["mhf_gate.cuh", "tcgen05.cuh", "tma.cuh"],
 }
+GATE_METRIC = "MHF gate stream + causal FFT-conv GB/s (v, a in, r out) at 1 B200; % of HBM roofline"
 
 
 def parse_args():
@@ -53,7 +55,9 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="small_f32", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="small_f32",
+                    choices=sorted(workloads.WORKLOADS) + sorted(workloads.GATE_WORKLOADS),
+                    help="a convolution workload, or a gate workload (MHF gate stream + convolution)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--path", choices=["fwd", "bwd", "decode"], default="fwd",
@@ -464,15 +468,229 @@ def run_ours(args, rank, world, local):
         pg.destroy_process_group()
 
 
+def gate_oracle_rate(gw, v, a, w, bias, budget_s: float):
+    """Time the oracle (gate, then convolution) on whole heads of batch 0,
+    repeated to about budget_s.  Returns (units/s, threads, description, seconds)."""
+    import oracle
+    import oracle.mhf_gate as mhf
+    C = gw.D // gw.H
+    sv, sa = np.ascontiguousarray(v[:1, :, :C]), np.ascontiguousarray(a[:1, :, :C])
+    sw, sb = np.ascontiguousarray(w[:C]), np.ascontiguousarray(bias[:C])
+    reps, secs = 0, 0.0
+    t0 = time.perf_counter()
+    while secs < budget_s and reps < 1000:
+        mhf.mhf_gated_conv(sv, sa, sw, sb, 1)
+        reps += 1
+        secs = time.perf_counter() - t0
+    units = gw.L * C * reps
+    desc = f"oracle (gate + direct sum) on head 0 of batch 0 of {gw.name}: 1x{gw.L}x{C} outputs, {reps} passes"
+    return units / secs, oracle.num_threads(), desc, secs
+
+
+def run_gated(args, rank, world, local):
+    """The MHF gate stream + convolution on a gate workload: one step = one
+    call of mhf_gated_conv (the tcgen05 gate kernel, then the convolution)."""
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    gw = workloads.GATE_WORKLOADS[args.workload]
+    v, a, w, bias = workloads.generate_gate(gw.B, gw.L, gw.D, gw.H, gw.K, gw.dtype, gw.seed + 1000 * rank)
+    tdt = {"f32": torch.float32, "bf16": torch.bfloat16}[gw.dtype]
+    es = 4 if gw.dtype == "f32" else 2
+
+    def to_t(x):
+        return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16) if gw.dtype == "bf16" else torch.from_numpy(x)
+
+    hv, ha = to_t(v), to_t(a)
+    tw, tb = torch.from_numpy(w).to(dev), torch.from_numpy(bias).to(dev)
+    units = gw.units
+    set_bytes = 4 * units * es  # v, a, gate workspace, r
+    n_sets = max(2, math.ceil(2.2 * L2_BYTES / set_bytes))
+    v0, a0 = hv.to(dev), ha.to(dev)
+    ws_bytes = ssm.mhf_gated_conv_workspace_bytes(tdt, gw.B, gw.L, gw.D)
+    sets = [(v0 if i == 0 else v0.clone(), a0 if i == 0 else a0.clone(),
+             torch.empty(ws_bytes, dtype=torch.uint8, device=dev), torch.empty_like(v0)) for i in range(n_sets)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        sv, sa, sws, sr = sets[i % n_sets]
+        ssm.mhf_gated_conv(sv, sa, tw, tb, gw.H, out=sr, workspace=sws, stream=stream)
+
+    def timed(fn, steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for i in range(steps):
+            fn(i)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1), pg, dev)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        ms = timed(step, args.steps)
+    clocks = clk.report()
+    ms_per_step = ms / args.steps
+    alg_bytes = 3 * units * es  # v and a in, r out: the gate stream need never leave the chip
+    gbs = alg_bytes * world * args.steps / (ms * 1e-3) / 1e9
+
+    # each kernel alone, same rotation (the gate's output goes to the set's workspace)
+    gviews = [s[2].view(tdt).view(gw.B, gw.L, gw.D) for s in sets]
+
+    def gate_only(i):
+        ssm.mhf_gate(sets[i % n_sets][1], tw, tb, gw.H, out=gviews[i % n_sets], stream=stream)
+
+    def conv_only(i):
+        ssm.causal_conv(sets[i % n_sets][0], gviews[i % n_sets], out=sets[i % n_sets][3], stream=stream)
+
+    k_steps = max(10, min(args.steps, 500))
+    for i in range(3):
+        gate_only(i)
+        conv_only(i)
+    gate_us = timed(gate_only, k_steps) / k_steps * 1e3
+    conv_us = timed(conv_only, k_steps) / k_steps * 1e3
+
+    # end to end: pinned host v, a -> device, gated conv, r -> pinned host, every step
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    phv, pha = hv.pin_memory(), ha.pin_memory()
+    phr = torch.empty_like(phv).pin_memory()
+    dv_, da_, dws_, dr_ = sets[0]
+
+    def e2e_step(_i):
+        dv_.copy_(phv, non_blocking=True)
+        da_.copy_(pha, non_blocking=True)
+        ssm.mhf_gated_conv(dv_, da_, tw, tb, gw.H, out=dr_, workspace=dws_, stream=stream)
+        phr.copy_(dr_, non_blocking=True)
+
+    for i in range(2):
+        e2e_step(i)
+    ems = timed(e2e_step, e2e_steps)
+    e2e_gbs = alg_bytes * world * e2e_steps / (ems * 1e-3) / 1e9
+
+    peak, peak_src = measured_peaks()
+    C = gw.D // gw.H
+    conv_bytes, gate_bytes = 3 * units * es, 2 * units * es + gw.D * C * gw.K * 4 + gw.D * 4
+    gate_flops = 2 * units * C * gw.K * 3  # three tf32 products per term (hi*hi, hi*lo, lo*hi)
+    kernel = "fftconv_fused_kernel" if gw.L <= 1024 else ("bigrow_group_kernel" if gw.L <= 4096 else "bigconv_kernel")
+    dominant = (kernel, conv_bytes, conv_us) if conv_us >= gate_us else ("mhf_gate_kernel", gate_bytes, gate_us)
+    traffic, _, _ = recorded_counters(gw.name, "mhf_gate_kernel")
+    bf16_peak = None
+    pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pp):
+        bf16_peak = json.load(open(pp)).get("bf16_tflops")
+    tf32_peak = (bf16_peak or 1590.0) * (1.1 / 2.25)
+    line = {
+        "metric": GATE_METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": gw.name, "path": "gated", "B": gw.B, "L": gw.L, "D": gw.D, "heads": gw.H,
+                   "taps": gw.K, "io_dtype": gw.dtype,
+                   "l2": f"inputs larger than L2: {n_sets} rotating (v,a,g,r) sets of {set_bytes / 2 ** 20:.0f} MiB",
+                   "parallelism": f"dp{world} (independent batches, no collective)"},
+        "outputs_per_s": units * world * args.steps / (ms * 1e-3),
+        "hbm_frac": gbs / world / peak,
+        "roofline": {"bound": "hbm", "achieved": dominant[1] / (dominant[2] * 1e-6) / 1e9, "peak": peak,
+                     "unit": "GB/s", "frac": dominant[1] / (dominant[2] * 1e-6) / 1e9 / peak,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)", "kernel": dominant[0],
+                     "algorithmic_bytes_per_launch": dominant[1], "launch_us": dominant[2],
+                     "traffic": None},
+        "gate_kernel": {"kernel": "mhf_gate_kernel (tcgen05 kind::tf32, 3 split products)", "launch_us": gate_us,
+                        "hbm": {"achieved": gate_bytes / (gate_us * 1e-6) / 1e9, "peak": peak, "unit": "GB/s",
+                                "frac": gate_bytes / (gate_us * 1e-6) / 1e9 / peak,
+                                "algorithmic_bytes_per_launch": gate_bytes, "traffic": traffic},
+                        "tensor": {"achieved": gate_flops / (gate_us * 1e-6) / 1e12, "peak": tf32_peak,
+                                   "unit": "TFLOP/s", "frac": gate_flops / (gate_us * 1e-6) / 1e12 / tf32_peak,
+                                   "flops_per_launch": gate_flops,
+                                   "peak_source": "MEASURED_PEAKS.json bf16_tflops x 1.1/2.25 (nominal tf32/bf16)"}},
+        "conv_kernel_us": conv_us,
+        "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": 2 * units * es,
+                "d2h_bytes_per_step": units * es, "steps": e2e_steps,
+                "path": "pinned host v, a -> device; mhf_gated_conv; r -> pinned host"},
+        "gpu_launches": args.steps * 2,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu_ups, cores, desc, secs = gate_oracle_rate(gw, v if gw.dtype == "f32" else workloads.bf16_to_f32(v),
+                                                      a if gw.dtype == "f32" else workloads.bf16_to_f32(a), w, bias,
+                                                      budget_s=15.0)
+        line["cpu_baseline"] = {"value": cpu_ups * 3 * es / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                "sample": desc, "seconds": secs}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def run_gated_reference(args, rank, world):
+    """The oracle (gate + direct sum) on the host cores, same metric."""
+    if rank != 0:
+        return
+    gw = workloads.GATE_WORKLOADS[args.workload]
+    v, a, w, bias = workloads.generate_gate(gw.B, gw.L, gw.D, gw.H, gw.K, "f32", gw.seed)
+    per_step = max(0.05, 120.0 / max(1, args.steps + args.warmup))
+    import oracle
+    import oracle.mhf_gate as mhf
+    C = gw.D // gw.H
+    sv, sa = np.ascontiguousarray(v[:1, :, :C]), np.ascontiguousarray(a[:1, :, :C])
+    sw, sb = np.ascontiguousarray(w[:C]), np.ascontiguousarray(bias[:C])
+    t0 = time.perf_counter()
+    mhf.mhf_gated_conv(sv, sa, sw, sb, 1)
+    reps = max(1, int(per_step / max(time.perf_counter() - t0, 1e-4)))
+    for _ in range(args.warmup):
+        mhf.mhf_gated_conv(sv, sa, sw, sb, 1)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for _ in range(reps):
+            mhf.mhf_gated_conv(sv, sa, sw, sb, 1)
+    el = time.perf_counter() - t0
+    es = 4 if gw.dtype == "f32" else 2
+    units = gw.L * C * reps * args.steps
+    gbs = units * 3 * es / el / 1e9
+    sample = f"oracle (gate + direct sum) on head 0 of batch 0 of {gw.name}, {reps} passes per step"
+    print(json.dumps({
+        "impl": "reference", "metric": GATE_METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": gw.name, "path": "gated", "B": gw.B, "L": gw.L, "D": gw.D, "heads": gw.H,
+                   "taps": gw.K, "io_dtype": gw.dtype},
+        "outputs_per_s": units / el,
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def main():
     args = parse_args()
     rank, world, local = dist_env()
     if world != args.gpus and "RANK" in os.environ:
         print(f"warning: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
+    gated = args.workload in workloads.GATE_WORKLOADS
     if args.impl == "reference":
-        run_reference(args, rank, world)
+        (run_gated_reference if gated else run_reference)(args, rank, world)
     else:
-        run_ours(args, rank, world, local)
+        if gated:
+            run_gated(args, rank, world, local)
+        else:
+            run_ours(args, rank, world, local)
 
 
 if __name__ == "__main__":

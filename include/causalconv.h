@@ -256,12 +256,68 @@ CC_API const char *causal_conv_strerror(int status);
 CC_API int causal_ntt_params(int64_t N, uint32_t out[6]);
 
 /*
+ * causal_mhf_gate_f32 / _bf16 -- the gate stream of the Multi-Head Fourier
+ * block (Caracal: Causal Architecture via Spectral Mixing, "Key design 1":
+ * x_g = Conv1d_G2(sigma(Linear_G1(x_norm))), a 1-D convolution grouped by
+ * head), starting from a = Linear_G1(x_norm):
+ *
+ *   g[b,t,hC+n] = bias[hC+n]
+ *               + sum_{k<K} sum_{c<C} w[hC+n][c][k] * sigmoid(a[b, t-(K-1)+k, hC+c])
+ *
+ * with C = D / H channels a head and terms with t-(K-1)+k < 0 left out (a
+ * causal convolution: K-1 zeros on the left).  sigma is the logistic
+ * function.  Readings where the page is silent: causal padding (a centred
+ * kernel would let g_t see future tokens), kernel size K a parameter, bias
+ * as in a default Conv1d.
+ *   a     [B, L, D] device array, channel-last (bf16: uint16 bit patterns);
+ *   w     [D, C, K] float32 device array (the grouped Conv1d weight layout:
+ *         output channel, input channel within the head, tap);
+ *   bias  [D] float32 device array, or NULL for no bias;
+ *   g     [B, L, D] device output, same dtype as a (bf16: rounded to nearest
+ *         even); must not overlap a, w or bias (CC_ERR_ALIAS);
+ *   H     number of heads, D % H == 0 (else CC_ERR_INVALID_ARG); the head
+ *         width C = D / H must be 16, 32 or 64 and 1 <= K <= 4, else
+ *         CC_ERR_UNSUPPORTED; L is limited as for causal_fftconv_f32.
+ * The contraction runs on the tensor cores (tf32 with each operand split
+ * into two tf32 parts, fp32 accumulation), so g carries fp32-level error:
+ * |g - g_exact| stays far below 1e-6 * (|bias| + sum |w| sigmoid(a)).
+ * Stream-ordered and asynchronous on `stream`; allocates nothing.  Returns
+ * CC_OK or an error status before launching anything.
+ */
+CC_API int causal_mhf_gate_f32(const float *a, const float *w, const float *bias, float *g, int64_t B, int64_t L,
+                               int64_t D, int64_t H, int64_t K, void *stream);
+CC_API int causal_mhf_gate_bf16(const uint16_t *a, const float *w, const float *bias, uint16_t *g, int64_t B,
+                                int64_t L, int64_t D, int64_t H, int64_t K, void *stream);
+
+/*
+ * causal_mhf_gated_conv_f32 / _bf16 -- the gate stream followed by the
+ * causal convolution: r = causal_fftconv(v, causal_mhf_gate(a, w, bias)).
+ * v, a, r are [B, L, D] device arrays of the entry's dtype; w, bias as for
+ * causal_mhf_gate_f32.  The gate is written once into the caller's
+ * workspace (at least causal_mhf_gated_conv_workspace_bytes() bytes of
+ * device memory, overlapping none of the arrays: CC_ERR_WORKSPACE /
+ * CC_ERR_ALIAS), then the convolution reads it.  r must overlap no input.
+ * Two launches on `stream`; allocates nothing.
+ */
+CC_API int causal_mhf_gated_conv_f32(const float *v, const float *a, const float *w, const float *bias, float *r,
+                                     int64_t B, int64_t L, int64_t D, int64_t H, int64_t K, void *workspace,
+                                     size_t workspace_bytes, void *stream);
+CC_API int causal_mhf_gated_conv_bf16(const uint16_t *v, const uint16_t *a, const float *w, const float *bias,
+                                      uint16_t *r, int64_t B, int64_t L, int64_t D, int64_t H, int64_t K,
+                                      void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace of the gated convolution: B*L*D elements of the dtype (the gate
+ * stream), or (size_t)-1 for invalid sizes or dtype (only F32 and BF16). */
+CC_API size_t causal_mhf_gated_conv_workspace_bytes(int dtype, int64_t B, int64_t L, int64_t D);
+
+/*
  * causal_conv_fault_flags -- the library's per-device fault word.  The pages
  * have no counterpart: it reports waits inside the kernels that ran out of
  * time.  Every wait in the kernels (on an asynchronous copy, an mbarrier) is
  * bounded to about two seconds; a wait that runs out sets a bit here and its
  * kernel returns early, leaving its outputs incomplete, instead of hanging the
- * device.  Bit 0: a TMA staging copy did not complete.
+ * device.  Bit 0: a TMA staging copy did not complete.  Bit 1: the
+ * tensor-core MMAs of the gate stream did not signal completion.
  *   device  CUDA device ordinal;
  *   flags   host pointer, receives the word;
  *   clear   non-zero: reset the word to 0 after reading it.

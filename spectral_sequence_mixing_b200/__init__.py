@@ -4,7 +4,8 @@
 
 computed as in Caracal: Causal Architecture via Spectral Mixing (Multi-Head
 Fourier module: zero-pad to 2L, FFT, pointwise product, inverse FFT,
-truncate to L), plus the exact number-theoretic variant of "Catastrophic
+truncate to L), the gate stream of the same block (sigmoid and the head-grouped causal
+Conv1d_G2, on the tensor cores), plus the exact number-theoretic variant of "Catastrophic
 Token Leakage in Convolutional Sequence Modeling and How to Mitigate It".
 
 This module is argument marshalling only: every step of the computation runs
@@ -24,7 +25,7 @@ __all__ = [
     "causal_fftconv_f32", "causal_fftconv_bf16", "causal_ntt_conv_i32", "causal_conv", "causal_conv_bwd",
     "causal_conv_decode", "decode_workspace_bytes",
     "causal_conv_from_host", "workspace_bytes", "fast_workspace_bytes", "max_len", "ntt_params", "strerror",
-    "fault_flags",
+    "fault_flags", "mhf_gate", "mhf_gated_conv", "mhf_gated_conv_workspace_bytes",
     "CausalConvError", "CC_DTYPE_F32", "CC_DTYPE_BF16", "CC_DTYPE_I32",
 ]
 
@@ -227,3 +228,81 @@ def fault_flags(device: int | None = None, clear: bool = False) -> int:
     if st != 0:
         raise CausalConvError(st, "causal_conv_fault_flags")
     return int(out.value)
+
+
+# ------------------------------------------------------------------ MHF gate stream
+_GATE_FN = {torch.float32: "causal_mhf_gate_f32", torch.bfloat16: "causal_mhf_gate_bf16"}
+_GATED_FN = {torch.float32: "causal_mhf_gated_conv_f32", torch.bfloat16: "causal_mhf_gated_conv_bf16"}
+
+
+def _check_gate_params(w: torch.Tensor, bias, D: int, n_head: int, device):
+    if not isinstance(w, torch.Tensor) or w.dtype != torch.float32 or w.dim() != 3:
+        raise TypeError("w must be a float32 tensor [D, D/n_head, K]")
+    if n_head < 1 or D % n_head or tuple(w.shape[:2]) != (D, D // n_head):
+        raise ValueError(f"w shape {tuple(w.shape)} does not fit D={D}, n_head={n_head}")
+    if not w.is_contiguous() or w.device != device:
+        raise ValueError("w must be contiguous and on the device of a")
+    if bias is not None:
+        if not isinstance(bias, torch.Tensor) or bias.dtype != torch.float32 or tuple(bias.shape) != (D,):
+            raise TypeError("bias must be a float32 tensor [D] or None")
+        if not bias.is_contiguous() or bias.device != device:
+            raise ValueError("bias must be contiguous and on the device of a")
+    return int(w.shape[2])
+
+
+def mhf_gate(a: torch.Tensor, w: torch.Tensor, bias: torch.Tensor | None, n_head: int, out=None,
+             stream=None) -> torch.Tensor:
+    """g = Conv1d_G2(sigmoid(a)): the head-grouped causal convolution of the
+    gate stream (w: [D, D/n_head, K] float32, bias: [D] float32 or None);
+    a and the result are [B, L, D] float32 or bfloat16."""
+    if a.dtype not in _GATE_FN:
+        raise TypeError(f"unsupported dtype {a.dtype}")
+    _check(a, "a", a.dtype)
+    if not a.is_cuda:
+        raise ValueError("a must be a CUDA tensor")
+    B, L, D = a.shape
+    K = _check_gate_params(w, bias, D, n_head, a.device)
+    if out is None:
+        out = torch.empty_like(a)
+    _check(out, "out", a.dtype, a.shape)
+    fn = getattr(load(), _GATE_FN[a.dtype])
+    with torch.cuda.device(a.device):
+        st = fn(a.data_ptr(), w.data_ptr(), bias.data_ptr() if bias is not None else None, out.data_ptr(), B, L, D,
+                n_head, K, _stream_ptr(stream))
+    if st != 0:
+        raise CausalConvError(st, _GATE_FN[a.dtype])
+    return out
+
+
+def mhf_gated_conv_workspace_bytes(dtype: torch.dtype, B: int, L: int, D: int) -> int:
+    return int(load().causal_mhf_gated_conv_workspace_bytes(_DT[dtype], B, L, D))
+
+
+def mhf_gated_conv(v: torch.Tensor, a: torch.Tensor, w: torch.Tensor, bias: torch.Tensor | None, n_head: int,
+                   out=None, workspace=None, stream=None) -> torch.Tensor:
+    """r = causal_conv(v, mhf_gate(a, w, bias, n_head)); the gate goes through
+    ``workspace`` (a device tensor of at least mhf_gated_conv_workspace_bytes
+    bytes; taken from the torch allocator when None)."""
+    if v.dtype not in _GATED_FN:
+        raise TypeError(f"unsupported dtype {v.dtype}")
+    _check(v, "v", v.dtype)
+    _check(a, "a", v.dtype, v.shape)
+    if not v.is_cuda or v.device != a.device:
+        raise ValueError("v and a must be CUDA tensors on the same device")
+    B, L, D = v.shape
+    K = _check_gate_params(w, bias, D, n_head, v.device)
+    if out is None:
+        out = torch.empty_like(v)
+    _check(out, "out", v.dtype, v.shape)
+    if workspace is None:
+        workspace = torch.empty(mhf_gated_conv_workspace_bytes(v.dtype, B, L, D), dtype=torch.uint8,
+                                device=v.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    fn = getattr(load(), _GATED_FN[v.dtype])
+    with torch.cuda.device(v.device):
+        st = fn(v.data_ptr(), a.data_ptr(), w.data_ptr(), bias.data_ptr() if bias is not None else None,
+                out.data_ptr(), B, L, D, n_head, K, workspace.data_ptr() if nbytes else None, nbytes,
+                _stream_ptr(stream))
+    if st != 0:
+        raise CausalConvError(st, _GATED_FN[v.dtype])
+    return out

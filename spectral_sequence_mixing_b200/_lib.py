@@ -36,6 +36,11 @@ SIGNATURES = {
     "causal_conv_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "causal_ntt_params": (ctypes.c_int, [_I64, ctypes.POINTER(ctypes.c_uint32)]),
     "causal_conv_fault_flags": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_uint), ctypes.c_int]),
+    "causal_mhf_gate_f32": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P]),
+    "causal_mhf_gate_bf16": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P]),
+    "causal_mhf_gated_conv_f32": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
+    "causal_mhf_gated_conv_bf16": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
+    "causal_mhf_gated_conv_workspace_bytes": (_SZ, [ctypes.c_int, _I64, _I64, _I64]),
 }
 
 _lib = None

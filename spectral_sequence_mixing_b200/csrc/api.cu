@@ -23,6 +23,7 @@
 #include "ntt.cuh"
 #include "decode.cuh"
 #include "transpose.cuh"
+#include "mhf_gate.cuh"
 #include "configs.cuh"
 
 namespace ccv {
@@ -590,6 +591,118 @@ static int from_host_chunk(int dtype, const void *v_host, const void *g_host, vo
     return CC_OK;
 }
 
+// ------------------------------------------------------------------ MHF gate
+template <int C, int KT, typename IO>
+static int launch_gate_ck(const IO *a, const float *w, const float *bias, IO *g, int64_t B, int64_t L, int64_t D,
+                          int64_t H, cudaStream_t s, int dev) {
+    using Cfg = GateCfg<C, KT>;
+    static std::atomic<bool> attr_set[128];
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(mhf_gate_kernel<C, KT, IO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)Cfg::SMEM_BYTES) != cudaSuccess)
+            return CC_ERR_CUDA;
+        attr_set[dev].store(true, std::memory_order_release);
+    }
+    const int64_t per_row = (L + kGateM - 1) / kGateM;
+    const int64_t tiles = B * per_row;  // tiles of one head
+    if (tiles > INT32_MAX || H > INT32_MAX / 2) return CC_ERR_UNSUPPORTED;
+    // persistent CTAs: as many as fit on the SMs at once, split evenly over the heads
+    static std::atomic<int> resident[128];
+    int cps = resident[dev].load(std::memory_order_relaxed);
+    if (cps == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&cps, mhf_gate_kernel<C, KT, IO>, kGateThreads,
+                                                          Cfg::SMEM_BYTES) != cudaSuccess)
+            return CC_ERR_CUDA;
+        cps = std::max(1, cps);
+        resident[dev].store(cps, std::memory_order_relaxed);
+    }
+    const int64_t groups = std::max<int64_t>(1, std::min<int64_t>(tiles, (int64_t)g_num_sms[dev] * cps / H));
+    const int64_t grid = H * groups;
+    if (grid > INT32_MAX) return CC_ERR_UNSUPPORTED;
+    const int vec_in = ((uintptr_t)a % (sizeof(IO) == 4 ? 16 : 8)) == 0;
+    const int vec_out = ((uintptr_t)g % 16) == 0;
+    const int vec_w = ((uintptr_t)w % 16) == 0;
+    mhf_gate_kernel<C, KT, IO><<<(unsigned)grid, kGateThreads, Cfg::SMEM_BYTES, s>>>(
+        a, w, bias, g, (int)L, (int)D, (int)H, (int)groups, (int)per_row, (int)tiles, vec_in, vec_out, vec_w);
+    return cudaGetLastError() == cudaSuccess ? CC_OK : CC_ERR_CUDA;
+}
+
+template <int C, typename IO>
+static int launch_gate_c(const IO *a, const float *w, const float *bias, IO *g, int64_t B, int64_t L, int64_t D,
+                         int64_t H, int64_t K, cudaStream_t s, int dev) {
+    switch (K) {
+        case 1: return launch_gate_ck<C, 1, IO>(a, w, bias, g, B, L, D, H, s, dev);
+        case 2: return launch_gate_ck<C, 2, IO>(a, w, bias, g, B, L, D, H, s, dev);
+        case 3: return launch_gate_ck<C, 3, IO>(a, w, bias, g, B, L, D, H, s, dev);
+        case 4: return launch_gate_ck<C, 4, IO>(a, w, bias, g, B, L, D, H, s, dev);
+        default: return CC_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename IO>
+static int launch_gate(const IO *a, const float *w, const float *bias, IO *g, int64_t B, int64_t L, int64_t D,
+                       int64_t H, int64_t K, cudaStream_t s, int dev) {
+    switch (D / H) {
+        case 16: return launch_gate_c<16, IO>(a, w, bias, g, B, L, D, H, K, s, dev);
+        case 32: return launch_gate_c<32, IO>(a, w, bias, g, B, L, D, H, K, s, dev);
+        case 64: return launch_gate_c<64, IO>(a, w, bias, g, B, L, D, H, K, s, dev);
+        default: return CC_ERR_UNSUPPORTED;
+    }
+}
+
+// Shapes, head width, taps and aliasing of a gate call (no CUDA call).
+static int check_gate_host(int dtype, const void *a, const float *w, const float *bias, const void *g, int64_t B,
+                           int64_t L, int64_t D, int64_t H, int64_t K, size_t *bytes) {
+    if (dtype != CC_DTYPE_F32 && dtype != CC_DTYPE_BF16) return CC_ERR_INVALID_ARG;
+    if (!a || !w || !g) return CC_ERR_INVALID_ARG;
+    int st = check_shape(dtype, B, L, D, bytes);
+    if (st != CC_OK) return st;
+    if (H < 1 || K < 1 || D % H != 0) return CC_ERR_INVALID_ARG;
+    const int64_t C = D / H;
+    if ((C != 16 && C != 32 && C != 64) || K > kGateMaxTaps) return CC_ERR_UNSUPPORTED;
+    const size_t wb = (size_t)D * (size_t)C * (size_t)K * sizeof(float);
+    if (ranges_overlap(g, *bytes, a, *bytes) || ranges_overlap(g, *bytes, w, wb) ||
+        (bias && ranges_overlap(g, *bytes, bias, (size_t)D * sizeof(float))))
+        return CC_ERR_ALIAS;
+    return CC_OK;
+}
+
+template <typename IO>
+static int gate_entry(int dtype, const IO *a, const float *w, const float *bias, IO *g, int64_t B, int64_t L,
+                      int64_t D, int64_t H, int64_t K, cudaStream_t s) {
+    size_t bytes = 0;
+    int st = check_gate_host(dtype, a, w, bias, g, B, L, D, H, K, &bytes);
+    if (st != CC_OK) return st;
+    int dev;
+    if ((st = check_device({a, w, g}, &dev)) != CC_OK) return st;
+    if (bias && (st = check_device_ptr(bias, dev)) != CC_OK) return st;
+    if (ensure_init(dev) != cudaSuccess) return CC_ERR_CUDA;
+    return launch_gate<IO>(a, w, bias, g, B, L, D, H, K, s, dev);
+}
+
+template <typename IO>
+static int gated_conv_entry(int dtype, const IO *v, const IO *a, const float *w, const float *bias, IO *r, int64_t B,
+                            int64_t L, int64_t D, int64_t H, int64_t K, void *ws, size_t ws_bytes, cudaStream_t s) {
+    if (!v || !r || !ws) return CC_ERR_INVALID_ARG;
+    size_t bytes = 0;
+    int st = check_gate_host(dtype, a, w, bias, ws, B, L, D, H, K, &bytes);
+    if (st != CC_OK) return st;
+    if (ws_bytes < bytes) return CC_ERR_WORKSPACE;
+    const int64_t C = D / H;
+    const size_t wb = (size_t)D * (size_t)C * (size_t)K * sizeof(float);
+    if (ranges_overlap(r, bytes, v, bytes) || ranges_overlap(r, bytes, a, bytes) || ranges_overlap(r, bytes, w, wb) ||
+        ranges_overlap(r, bytes, ws, bytes) || ranges_overlap(ws, bytes, v, bytes) ||
+        (bias && ranges_overlap(r, bytes, bias, (size_t)D * sizeof(float))))
+        return CC_ERR_ALIAS;
+    int dev;
+    if ((st = check_device({v, a, w, r, ws}, &dev)) != CC_OK) return st;
+    if (bias && (st = check_device_ptr(bias, dev)) != CC_OK) return st;
+    if (ensure_init(dev) != cudaSuccess) return CC_ERR_CUDA;
+    IO *gbuf = reinterpret_cast<IO *>(ws);
+    if ((st = launch_gate<IO>(a, w, bias, gbuf, B, L, D, H, K, s, dev)) != CC_OK) return st;
+    return fftconv_dispatch<IO>(v, gbuf, r, B, L, D, nullptr, 0, s, dev);
+}
+
 extern "C" {
 
 size_t causal_conv_workspace_bytes(int dtype, int64_t B, int64_t L, int64_t D) {
@@ -759,6 +872,39 @@ int causal_ntt_params(int64_t N, uint32_t out[6]) {
     out[4] = p.pinv;
     out[5] = p.r2;
     return CC_OK;
+}
+
+int causal_mhf_gate_f32(const float *a, const float *w, const float *bias, float *g, int64_t B, int64_t L,
+                        int64_t D, int64_t H, int64_t K, void *stream) {
+    return gate_entry<float>(CC_DTYPE_F32, a, w, bias, g, B, L, D, H, K, (cudaStream_t)stream);
+}
+
+int causal_mhf_gate_bf16(const uint16_t *a, const float *w, const float *bias, uint16_t *g, int64_t B, int64_t L,
+                         int64_t D, int64_t H, int64_t K, void *stream) {
+    return gate_entry<__nv_bfloat16>(CC_DTYPE_BF16, (const __nv_bfloat16 *)a, w, bias, (__nv_bfloat16 *)g, B, L, D, H,
+                                     K, (cudaStream_t)stream);
+}
+
+size_t causal_mhf_gated_conv_workspace_bytes(int dtype, int64_t B, int64_t L, int64_t D) {
+    size_t bytes = 0;
+    if ((dtype != CC_DTYPE_F32 && dtype != CC_DTYPE_BF16) || check_shape(dtype, B, L, D, &bytes) != CC_OK)
+        return (size_t)-1;
+    return bytes;
+}
+
+int causal_mhf_gated_conv_f32(const float *v, const float *a, const float *w, const float *bias, float *r, int64_t B,
+                              int64_t L, int64_t D, int64_t H, int64_t K, void *workspace, size_t workspace_bytes,
+                              void *stream) {
+    return gated_conv_entry<float>(CC_DTYPE_F32, v, a, w, bias, r, B, L, D, H, K, workspace, workspace_bytes,
+                                   (cudaStream_t)stream);
+}
+
+int causal_mhf_gated_conv_bf16(const uint16_t *v, const uint16_t *a, const float *w, const float *bias, uint16_t *r,
+                               int64_t B, int64_t L, int64_t D, int64_t H, int64_t K, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+    return gated_conv_entry<__nv_bfloat16>(CC_DTYPE_BF16, (const __nv_bfloat16 *)v, (const __nv_bfloat16 *)a, w, bias,
+                                           (__nv_bfloat16 *)r, B, L, D, H, K, workspace, workspace_bytes,
+                                           (cudaStream_t)stream);
 }
 
 int causal_conv_fault_flags(int device, unsigned int *flags, int clear) {

@@ -1,0 +1,345 @@
+// mhf_gate.cuh -- gate stream of the Multi-Head Fourier block on the tensor cores.
+//
+// Caracal: Causal Architecture via Spectral Mixing, "Key design 1": the gate
+// stream is x_g = Conv1d_G2(sigma(Linear_G1(x_norm))), a 1-D convolution
+// grouped by head.  Starting from a = Linear_G1(x_norm) ([B, L, D],
+// channel-last, C = D / H channels a head, K taps, causal):
+//
+//   g[b, t, h C + n] = bias[h C + n]
+//                    + sum_{k<K} sum_{c<C} w[h C + n][c][k] * sigmoid(a[b, t-(K-1)+k, h C + c])
+//
+// For one head and one batch this is a dense contraction over (k, c):
+// [128 time steps x C] times [C x C] per tap, so it runs as tcgen05 MMAs:
+// M = 128 time steps, N = C output channels, K = C input channels per tap,
+// accumulated over the taps in TMEM.  The taps need no extra copies: the
+// staged sigmoid tile holds time steps t0-(K-1) .. t0+127, and tap k's
+// operand is the same tile started k rows later (16 bytes in the K-major
+// no-swizzle layout).
+//
+// fp32 accuracy from tf32 tensor cores: every operand x is split into
+// hi = x with its 13 low mantissa bits cleared (exact in tf32) and
+// lo = x - hi (exact in fp32, |lo| <= 2^-10 |x|), and the product is
+// hi*W_hi + hi*W_lo + lo*W_hi.  The dropped lo*W_lo term and the tf32 view of
+// the lo parts are below 2^-20 of |x W|, so g carries fp32-level error.
+//
+// Schedule: a persistent CTA per (head, group of tiles); the head's weights
+// are split and staged in shared memory once; per 128-step tile the CTA
+// stores sigmoid(a) (hi, lo) to shared memory, one thread issues
+// 3 K C/8 MMAs and commits them to an mbarrier, the next tile's a is loaded
+// into registers while the tensor core works, and the eight warps read the
+// accumulator back (warp w: TMEM lanes 32 (w % 4) .. +31 = time steps, half
+// of the columns each), add the bias and store g.  Every wait is bounded; no
+// load uses cluster multicast.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "tcgen05.cuh"
+#include "tma.cuh"
+
+namespace ccv {
+
+constexpr unsigned kFaultMmaWait = 2u;  // fault bit: an MMA completion wait ran out
+constexpr int kGateM = 128;             // time steps per tile (MMA M)
+constexpr int kGateThreads = 256;       // eight warps: two per TMEM lane quarter, each half of the columns
+constexpr int kGateMaxTaps = 4;
+
+template <int C, int KT>
+struct GateCfg {
+    static_assert(C == 16 || C == 32 || C == 64, "head width");
+    static_assert(KT >= 1 && KT <= kGateMaxTaps, "taps");
+    static constexpr int ROWS = kGateM + KT - 1;          // staged time steps
+    static constexpr int R = ROWS | 1;                     // odd row count: conflict-free 16-byte stores
+    static constexpr int KC = C / 4;                       // 16-byte chunks along the contraction axis
+    static constexpr unsigned LBO_A = R * 16u;             // chunk pitch of the sigmoid tile
+    static constexpr unsigned A_BYTES = KC * LBO_A;
+    static constexpr unsigned LBO_W = C * 16u;             // chunk pitch of one tap's weights
+    static constexpr unsigned W_TAP = KC * LBO_W;          // = C * C * 4
+    static constexpr unsigned W_BYTES = KT * W_TAP;
+    static constexpr unsigned OFF_AHI = 0, OFF_ALO = A_BYTES;
+    static constexpr unsigned OFF_WHI = 2 * A_BYTES, OFF_WLO = OFF_WHI + W_BYTES;
+    static constexpr unsigned OFF_BIAS = OFF_WLO + W_BYTES;
+    static constexpr unsigned OFF_BAR = (OFF_BIAS + C * 4u + 15u) & ~15u;
+    static constexpr unsigned SMEM_BYTES = OFF_BAR + 16u + 128u;  // + alignment slack
+    static constexpr unsigned TMEM_COLS = C < 32 ? 32u : (unsigned)C;
+    static constexpr int NLOAD = (ROWS * KC + kGateThreads - 1) / kGateThreads;  // 4-vectors per thread
+    static constexpr int NMMA = 3 * KT * (C / 8);
+};
+
+__device__ __forceinline__ void split_tf32(float x, float &hi, float &lo) {
+    hi = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
+    lo = x - hi;
+}
+
+// Logistic function from the fast exponential and reciprocal (both within a
+// few ulp; the bound on g is 1e-5 of |w| sigmoid(a)).  Saturates cleanly: a
+// large negative x gives exp = inf and 1/inf = 0.
+__device__ __forceinline__ float logistic(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+
+// Four consecutive channels of a, as loaded (fp32: one 16-byte load; bf16: 8 bytes).
+template <typename IO>
+struct Raw4;
+template <>
+struct Raw4<float> {
+    float4 x;
+    __device__ __forceinline__ void load(const float *p, bool vec) {
+        x = vec ? __ldg(reinterpret_cast<const float4 *>(p)) : make_float4(p[0], p[1], p[2], p[3]);
+    }
+    __device__ __forceinline__ void zero() { x = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ float4 f32() const { return x; }
+};
+template <>
+struct Raw4<__nv_bfloat16> {
+    uint2 x;
+    __device__ __forceinline__ void load(const __nv_bfloat16 *p, bool vec) {
+        if (vec) {
+            x = __ldg(reinterpret_cast<const uint2 *>(p));
+        } else {
+            const uint16_t *q = reinterpret_cast<const uint16_t *>(p);
+            x = make_uint2((unsigned)q[0] | ((unsigned)q[1] << 16), (unsigned)q[2] | ((unsigned)q[3] << 16));
+        }
+    }
+    __device__ __forceinline__ void zero() { x = make_uint2(0u, 0u); }
+    __device__ __forceinline__ float4 f32() const {
+        return make_float4(__uint_as_float(x.x << 16), __uint_as_float(x.x & 0xFFFF0000u),
+                           __uint_as_float(x.y << 16), __uint_as_float(x.y & 0xFFFF0000u));
+    }
+};
+
+// Store 16 consecutive output channels of one time step.
+__device__ __forceinline__ void store16(float *p, const float (&v)[16], bool vec) {
+    if (vec) {
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) reinterpret_cast<float4 *>(p)[i / 4] = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) p[i] = v[i];
+    }
+}
+__device__ __forceinline__ void store16(__nv_bfloat16 *p, const float (&v)[16], bool vec) {
+    unsigned u[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        u[i] = *reinterpret_cast<const unsigned *>(&h);
+    }
+    if (vec) {
+        reinterpret_cast<uint4 *>(p)[0] = make_uint4(u[0], u[1], u[2], u[3]);
+        reinterpret_cast<uint4 *>(p)[1] = make_uint4(u[4], u[5], u[6], u[7]);
+    } else {
+        uint16_t *q = reinterpret_cast<uint16_t *>(p);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            q[2 * i] = (uint16_t)(u[i] & 0xFFFFu);
+            q[2 * i + 1] = (uint16_t)(u[i] >> 16);
+        }
+    }
+}
+
+__device__ __forceinline__ void store8(float *p, const float (&v)[8], bool vec) {
+    if (vec) {
+        reinterpret_cast<float4 *>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+        reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) p[i] = v[i];
+    }
+}
+__device__ __forceinline__ void store8(__nv_bfloat16 *p, const float (&v)[8], bool vec) {
+    unsigned u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        u[i] = *reinterpret_cast<const unsigned *>(&h);
+    }
+    if (vec) {
+        reinterpret_cast<uint4 *>(p)[0] = make_uint4(u[0], u[1], u[2], u[3]);
+    } else {
+        uint16_t *q = reinterpret_cast<uint16_t *>(p);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            q[2 * i] = (uint16_t)(u[i] & 0xFFFFu);
+            q[2 * i + 1] = (uint16_t)(u[i] >> 16);
+        }
+    }
+}
+
+// grid = H * groups CTAs; CTA (h = blockIdx.x % H, j = blockIdx.x / H) takes
+// the tiles j, j + groups, ... of head h, tile = b * tiles_per_row + t0 / 128.
+// vec_in: a's rows allow 4-channel vector loads; vec_out: g allows 16-byte
+// stores; vec_w: w is 16-byte aligned.
+template <int C, int KT, typename IO>
+__global__ void __launch_bounds__(kGateThreads, 1)
+    mhf_gate_kernel(const IO *__restrict__ a, const float *__restrict__ w, const float *__restrict__ bias,
+                    IO *__restrict__ g, int L, int D, int H, int groups, int tiles_per_row, int num_tiles,
+                    int vec_in, int vec_out, int vec_w) {
+    using Cfg = GateCfg<C, KT>;
+    extern __shared__ unsigned char gate_smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(((uintptr_t)gate_smem_raw + 127) & ~(uintptr_t)127);
+    const unsigned sb = smem_u32(sm);
+    float *sbias = reinterpret_cast<float *>(sm + Cfg::OFF_BIAS);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + Cfg::OFF_BAR);
+    unsigned *tslot = reinterpret_cast<unsigned *>(sm + Cfg::OFF_BAR + 8);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.x % H;
+    const int64_t col0 = (int64_t)h * C;
+
+    if (warp == 0) tmem_alloc(tslot, Cfg::TMEM_COLS);
+    if (tid == 0) mbar_init(bar, 1);
+
+    // The head's weights, split into tf32 hi / lo, in the K-major layout:
+    // tap k, chunk c/4, output channel n, element c%4.  w is [D][C][K]; the
+    // head's block is C*C*K contiguous floats, read 4 at a time.
+    const float *wh = w + col0 * C * KT;
+    auto put_w = [&](int i, float x) {
+        const int k = i % KT, c = (i / KT) % C, n = i / (KT * C);
+        float hi, lo;
+        split_tf32(x, hi, lo);
+        const unsigned off = k * Cfg::W_TAP + (c >> 2) * Cfg::LBO_W + n * 16u + (c & 3) * 4u;
+        *reinterpret_cast<float *>(sm + Cfg::OFF_WHI + off) = hi;
+        *reinterpret_cast<float *>(sm + Cfg::OFF_WLO + off) = lo;
+    };
+    if (vec_w) {
+#pragma unroll 4
+        for (int i4 = tid; i4 < C * C * KT / 4; i4 += kGateThreads) {
+            const float4 x = __ldg(reinterpret_cast<const float4 *>(wh) + i4);
+            put_w(4 * i4, x.x);
+            put_w(4 * i4 + 1, x.y);
+            put_w(4 * i4 + 2, x.z);
+            put_w(4 * i4 + 3, x.w);
+        }
+    } else {
+#pragma unroll 4
+        for (int i = tid; i < C * C * KT; i += kGateThreads) put_w(i, __ldg(wh + i));
+    }
+    if (tid < C) sbias[tid] = bias ? __ldg(bias + col0 + tid) : 0.0f;
+
+    Raw4<IO> raw[Cfg::NLOAD];
+    auto load_tile = [&](int tile) {
+        const int b = tile / tiles_per_row;
+        const int t0 = (tile % tiles_per_row) * kGateM;
+        const IO *base = a + (int64_t)b * L * D + col0;
+#pragma unroll
+        for (int j = 0; j < Cfg::NLOAD; ++j) {
+            const int i = tid + j * kGateThreads;
+            const int r = i / Cfg::KC, kc = i % Cfg::KC;
+            const int t = t0 - (KT - 1) + r;
+            if (i < Cfg::ROWS * Cfg::KC && t >= 0 && t < L)
+                raw[j].load(base + (int64_t)t * D + kc * 4, vec_in != 0);
+            else
+                raw[j].zero();
+        }
+    };
+    auto stage_tile = [&](int tile) {
+        const int t0 = (tile % tiles_per_row) * kGateM;
+#pragma unroll
+        for (int j = 0; j < Cfg::NLOAD; ++j) {
+            const int i = tid + j * kGateThreads;
+            if (i >= Cfg::ROWS * Cfg::KC) break;
+            const int r = i / Cfg::KC, kc = i % Cfg::KC;
+            const int t = t0 - (KT - 1) + r;
+            float4 s = make_float4(0.f, 0.f, 0.f, 0.f);  // the convolution's zero padding
+            if (t >= 0 && t < L) {
+                const float4 x = raw[j].f32();
+                s = make_float4(logistic(x.x), logistic(x.y), logistic(x.z), logistic(x.w));
+            }
+            float4 hi, lo;
+            split_tf32(s.x, hi.x, lo.x);
+            split_tf32(s.y, hi.y, lo.y);
+            split_tf32(s.z, hi.z, lo.z);
+            split_tf32(s.w, hi.w, lo.w);
+            const unsigned off = kc * Cfg::LBO_A + r * 16u;
+            *reinterpret_cast<float4 *>(sm + Cfg::OFF_AHI + off) = hi;
+            *reinterpret_cast<float4 *>(sm + Cfg::OFF_ALO + off) = lo;
+        }
+    };
+
+    int tile = blockIdx.x / H;
+    if (tile < num_tiles) load_tile(tile);
+
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const unsigned tmem = *tslot;
+    constexpr uint32_t idesc = umma_idesc_tf32(kGateM, C);
+
+    unsigned parity = 0;
+    bool ok = true;
+    for (; tile < num_tiles; tile += groups) {
+        // sigmoid(a) of this tile -> shared memory (the previous tile's MMAs
+        // have completed, and its accumulator has been read by every warp)
+        stage_tile(tile);
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        __syncthreads();
+        tc_fence_after_sync();
+        if (tid == 0) {
+            int step = 0;
+#pragma unroll 1
+            for (int p = 0; p < 3; ++p) {  // hi*W_hi, hi*W_lo, lo*W_hi
+                const unsigned A = sb + (p < 2 ? Cfg::OFF_AHI : Cfg::OFF_ALO);
+                const unsigned W = sb + (p == 1 ? Cfg::OFF_WLO : Cfg::OFF_WHI);
+#pragma unroll 1
+                for (int k = 0; k < KT; ++k) {
+#pragma unroll
+                    for (int s = 0; s < C / 8; ++s) {
+                        const uint64_t ad = umma_smem_desc(A + k * 16u + 2u * s * Cfg::LBO_A, Cfg::LBO_A, 128u);
+                        const uint64_t bd = umma_smem_desc(W + k * Cfg::W_TAP + 2u * s * Cfg::LBO_W, Cfg::LBO_W, 128u);
+                        umma_tf32(tmem, ad, bd, idesc, step > 0);
+                        ++step;
+                    }
+                }
+            }
+            umma_commit(bar);
+        }
+        // the next tile's a streams into registers while the tensor core works
+        const int next = tile + groups;
+        if (next < num_tiles) load_tile(next);
+
+        const bool done = mbar_wait_bounded(bar, parity);
+        parity ^= 1u;
+        if (!__syncthreads_and(done)) {
+            ok = false;
+            break;
+        }
+        tc_fence_after_sync();
+
+        // accumulator row = time step t0 + 32 (warp % 4) + lane; warps 0-3
+        // take the first half of the C columns, warps 4-7 the second
+        const int b = tile / tiles_per_row;
+        const int q = warp & 3, cbase = (warp >> 2) * (C / 2);
+        const int t = (tile % tiles_per_row) * kGateM + q * 32 + lane;
+        IO *dst = g + ((int64_t)b * L + t) * D + col0 + cbase;
+        const unsigned trow = tmem + ((unsigned)(q * 32) << 16) + cbase;
+        if constexpr (C / 2 >= 16) {
+#pragma unroll
+            for (int c0 = 0; c0 < C / 2; c0 += 16) {
+                float v[16];
+                tmem_ld16(trow + c0, v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] += sbias[cbase + c0 + i];
+                if (t < L) store16(dst + c0, v, vec_out != 0);
+            }
+        } else {
+            float v[8];
+            tmem_ld8(trow, v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] += sbias[cbase + i];
+            if (t < L) store8(dst, v, vec_out != 0);
+        }
+    }
+    if (!ok) {
+        if (tid == 0) atomicOr(&g_cc_fault, kFaultMmaWait);
+        mbar_wait_bounded(bar, parity ^ 1u);  // give the MMAs in flight a last chance to finish
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, Cfg::TMEM_COLS);
+    }
+}
+
+}  // namespace ccv

@@ -57,3 +57,22 @@ def run_gpu_bwd(dr, v, g, dtype: str):
     dv, dg = ssm.causal_conv_bwd(to_dev(dr, dtype), to_dev(v, dtype), to_dev(g, dtype))
     torch.cuda.synchronize()
     return from_dev(dv, dtype), from_dev(dg, dtype)
+
+
+def run_gpu_gate(a: np.ndarray, w: np.ndarray, bias, n_head: int, dtype: str) -> np.ndarray:
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    tb = None if bias is None else torch.from_numpy(np.ascontiguousarray(bias, np.float32)).cuda()
+    g = ssm.mhf_gate(to_dev(a, dtype), torch.from_numpy(np.ascontiguousarray(w, np.float32)).cuda(), tb, n_head)
+    torch.cuda.synchronize()
+    return from_dev(g, dtype)
+
+
+def run_gpu_gated_conv(v: np.ndarray, a: np.ndarray, w: np.ndarray, bias, n_head: int, dtype: str) -> np.ndarray:
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    tb = None if bias is None else torch.from_numpy(np.ascontiguousarray(bias, np.float32)).cuda()
+    r = ssm.mhf_gated_conv(to_dev(v, dtype), to_dev(a, dtype),
+                           torch.from_numpy(np.ascontiguousarray(w, np.float32)).cuda(), tb, n_head)
+    torch.cuda.synchronize()
+    return from_dev(r, dtype)

@@ -173,3 +173,41 @@ def test_fast_workspace_bytes(lib):
     assert f(0, 1, 65537, 8) == 0                      # beyond the longest row
     assert f(0, 70000, 5000, 8) == 0                   # B beyond the transpose grid
     assert f(0, 1, 5000, 0) == 0 and f(7, 1, 5000, 8) == 0
+
+
+@pytest.mark.parametrize("fn", ["causal_mhf_gate_f32", "causal_mhf_gate_bf16"])
+def test_gate_host_side_argument_errors(lib, fn):
+    """Every check of the gate entry that needs no device (dummy pointers)."""
+    f = getattr(lib, fn)
+    W_, G_ = 0x40000000, 0x50000000
+    INVALID, UNSUP, ALIAS = 1, 2, 3
+    ok = (1, 16, 64, 2, 3)  # B, L, D, H, K: head width 32
+    assert f(None, W_, None, G_, *ok, None) == INVALID
+    assert f(A, None, None, G_, *ok, None) == INVALID
+    assert f(A, W_, None, None, *ok, None) == INVALID
+    for shape in [(0, 16, 64, 2, 3), (1, 0, 64, 2, 3), (1, 16, 0, 2, 3), (1, 16, 64, 0, 3), (1, 16, 64, 2, 0),
+                  (1, 16, 64, 3, 1), (1, 16, 64, -2, 1)]:
+        assert f(A, W_, None, G_, *shape, None) == INVALID, shape
+    for shape in [(1, 16, 96, 2, 1), (1, 16, 256, 2, 1), (1, 16, 8, 1, 1), (1, 16, 64, 2, 5)]:
+        assert f(A, W_, None, G_, *shape, None) == UNSUP, shape       # head width 48 / 128 / 8, 5 taps
+    assert f(A, W_, None, A + 8, *ok, None) == ALIAS                    # g overlaps a
+    assert f(A, W_, None, W_ - 8, *ok, None) == ALIAS                   # g overlaps w
+    assert f(A, W_, G_ + 16, G_, *ok, None) == ALIAS                    # g overlaps bias
+
+
+def test_gated_conv_host_side_checks(lib):
+    f = lib.causal_mhf_gated_conv_f32
+    V_, W_, R_, S_ = 0x40000000, 0x50000000, 0x60000000, 0x70000000
+    need = lib.causal_mhf_gated_conv_workspace_bytes(0, 1, 16, 64)
+    assert need == 16 * 64 * 4
+    assert lib.causal_mhf_gated_conv_workspace_bytes(1, 1, 16, 64) == 16 * 64 * 2
+    assert lib.causal_mhf_gated_conv_workspace_bytes(2, 1, 16, 64) == ctypes.c_size_t(-1).value
+    ok = (1, 16, 64, 2, 3)
+    assert f(None, A, W_, None, R_, *ok, S_, need, None) == 1           # null v
+    assert f(V_, A, W_, None, R_, *ok, None, need, None) == 1           # null workspace
+    assert f(V_, A, W_, None, R_, *ok, S_, need - 1, None) == 4         # workspace too small
+    assert f(V_, A, W_, None, V_ + 4, *ok, S_, need, None) == 3         # r overlaps v
+    assert f(V_, A, W_, None, R_, *ok, A + 64, need, None) == 3         # workspace overlaps a
+    assert f(V_, A, W_, None, R_, *ok, V_ + 64, need, None) == 3        # workspace overlaps v
+    assert f(V_, A, W_, None, R_, *ok, R_ - 64, need, None) == 3        # workspace overlaps r
+    assert f(V_, A, W_, None, R_, 1, 16, 96, 2, 1, S_, 16 * 96 * 4, None) == 2  # head width 48

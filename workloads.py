@@ -21,6 +21,14 @@ the order listed, then rounded to the I/O type):
   large_bf16    [4, 4096, 1536] bf16  v ~ N(0,1); g ~ N(0, 1/64)                  seed 2
   long_f32      [1, 65536, 1024] fp32 v ~ N(0,1); g = z*(1+t)^-0.75               seed 3
   ntt_i32       [4, 8192, 256]  int32 v, g uniform integers in [-128, 127]        seed 4
+
+The gate stream of the same block (x_g = Conv1d_G2(sigmoid(a)), grouped by
+head) takes a = Linear_G1(x_norm) and the Conv1d weights instead of g
+(``generate_gate``; v, then a, then w, then bias from one generator):
+
+  mhf_small_f32 [8, 1024, 768]  fp32  12 heads of 64, K = 3 taps               seed 5
+  v, a ~ N(0,1); w, bias ~ U(-1/sqrt(C K), 1/sqrt(C K)) (a default Conv1d's
+  initialisation range, fan-in C K), w float32 [D, C, K], bias float32 [D].
 """
 from __future__ import annotations
 
@@ -135,3 +143,41 @@ def sample_points(B: int, L: int, D: int, n: int, seed: int) -> np.ndarray:
     b = rng.integers(0, B, size=n)
     d = rng.integers(0, D, size=n)
     return np.stack([b, t, d], axis=1).astype(np.int64)
+
+
+@dataclass(frozen=True)
+class GateWorkload:
+    name: str
+    B: int
+    L: int
+    D: int
+    H: int
+    K: int
+    dtype: str  # "f32" | "bf16"
+    seed: int
+    description: str
+
+    @property
+    def units(self) -> int:
+        return self.B * self.L * self.D
+
+
+GATE_WORKLOADS = {
+    "mhf_small_f32": GateWorkload("mhf_small_f32", 8, 1024, 768, 12, 3, "f32", 5,
+                                  "Caracal-Small-shaped MHF gate + conv (12 heads x 64, 3 taps)"),
+}
+
+
+def generate_gate(B: int, L: int, D: int, H: int, K: int, dtype: str, seed: int):
+    """(v, a, w, bias): v, a [B, L, D] in the I/O type (float32, or bf16 bit
+    patterns as uint16); w float32 [D, D/H, K]; bias float32 [D]."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    C = D // H
+    v = rng.standard_normal((B, L, D)).astype(np.float32)
+    a = rng.standard_normal((B, L, D)).astype(np.float32)
+    bound = 1.0 / np.sqrt(C * K)
+    w = rng.uniform(-bound, bound, (D, C, K)).astype(np.float32)
+    bias = rng.uniform(-bound, bound, D).astype(np.float32)
+    if dtype == "bf16":
+        return bf16_round(v), bf16_round(a), w, bias
+    return v, a, w, bias
