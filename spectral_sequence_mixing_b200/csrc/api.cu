@@ -621,9 +621,8 @@ static int launch_gate_ck(const IO *a, const float *w, const float *bias, IO *g,
     if (grid > INT32_MAX) return CC_ERR_UNSUPPORTED;
     const int vec_in = ((uintptr_t)a % (sizeof(IO) == 4 ? 16 : 8)) == 0;
     const int vec_out = ((uintptr_t)g % 16) == 0;
-    const int vec_w = ((uintptr_t)w % 16) == 0;
     mhf_gate_kernel<C, KT, IO><<<(unsigned)grid, kGateThreads, Cfg::SMEM_BYTES, s>>>(
-        a, w, bias, g, (int)L, (int)D, (int)H, (int)groups, (int)per_row, (int)tiles, vec_in, vec_out, vec_w);
+        a, w, bias, g, (int)L, (int)D, (int)H, (int)groups, (int)per_row, (int)tiles, vec_in, vec_out);
     return cudaGetLastError() == cudaSuccess ? CC_OK : CC_ERR_CUDA;
 }
 

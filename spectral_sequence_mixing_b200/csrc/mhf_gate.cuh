@@ -23,12 +23,15 @@
 // the lo parts are below 2^-20 of |x W|, so g carries fp32-level error.
 //
 // Schedule: a persistent CTA per (head, group of tiles); the head's weights
-// are split and staged in shared memory once; per 128-step tile the CTA
-// stores sigmoid(a) (hi, lo) to shared memory, one thread issues
-// 3 K C/8 MMAs and commits them to an mbarrier, the next tile's a is loaded
-// into registers while the tensor core works, and the eight warps read the
-// accumulator back (warp w: TMEM lanes 32 (w % 4) .. +31 = time steps, half
-// of the columns each), add the bias and store g.  Every wait is bounded; no
+// are split and staged in shared memory once.  Per 128-step tile the CTA
+// stores sigmoid(a) (hi, lo) to shared memory, one thread issues 3 K C/8
+// MMAs and commits them to an mbarrier, and the sixteen warps read the
+// accumulator back (warp w: TMEM lanes 32 (w % 4) .. +31 = time steps, a
+// quarter of the columns each), add the bias and store g.  With two tile
+// buffers and two accumulators (every head width and tap count whose tiles
+// fit twice) the tensor core works on tile i+1 while the warps drain tile i
+// and stage tile i+2; the a of the tile after that streams into registers
+// meanwhile.  Every wait is bounded; no
 // load uses cluster multicast.
 #pragma once
 
@@ -42,7 +45,7 @@ namespace ccv {
 
 constexpr unsigned kFaultMmaWait = 2u;  // fault bit: an MMA completion wait ran out
 constexpr int kGateM = 128;             // time steps per tile (MMA M)
-constexpr int kGateThreads = 256;       // eight warps: two per TMEM lane quarter, each half of the columns
+constexpr int kGateThreads = 512;       // sixteen warps: four per TMEM lane quarter, a quarter of the columns each
 constexpr int kGateMaxTaps = 4;
 
 template <int C, int KT>
@@ -50,19 +53,30 @@ struct GateCfg {
     static_assert(C == 16 || C == 32 || C == 64, "head width");
     static_assert(KT >= 1 && KT <= kGateMaxTaps, "taps");
     static constexpr int ROWS = kGateM + KT - 1;          // staged time steps
-    static constexpr int R = ROWS | 1;                     // odd row count: conflict-free 16-byte stores
     static constexpr int KC = C / 4;                       // 16-byte chunks along the contraction axis
+    // Two sigmoid tiles (one being staged while the tensor core reads the
+    // other) when they fit next to the weights; an odd row count keeps the
+    // 16-byte stores conflict-free, an even one (2-way conflicts) is taken
+    // when only that fits.
+    static constexpr unsigned kMaxSmem = 232448;
+    static constexpr unsigned FIXED = 2u * KT * C * C * 4u + C * 4u + 48u + 128u;
+    static constexpr bool DB_ODD = 4u * KC * (ROWS | 1) * 16u + FIXED <= kMaxSmem;
+    static constexpr bool DB_EVEN = (ROWS % 2 == 0) && 4u * KC * ROWS * 16u + FIXED <= kMaxSmem;
+    static constexpr int NBUF = (DB_ODD || DB_EVEN) ? 2 : 1;
+    static constexpr int R = DB_ODD ? (ROWS | 1) : (DB_EVEN ? ROWS : (ROWS | 1));
     static constexpr unsigned LBO_A = R * 16u;             // chunk pitch of the sigmoid tile
     static constexpr unsigned A_BYTES = KC * LBO_A;
     static constexpr unsigned LBO_W = C * 16u;             // chunk pitch of one tap's weights
     static constexpr unsigned W_TAP = KC * LBO_W;          // = C * C * 4
     static constexpr unsigned W_BYTES = KT * W_TAP;
-    static constexpr unsigned OFF_AHI = 0, OFF_ALO = A_BYTES;
-    static constexpr unsigned OFF_WHI = 2 * A_BYTES, OFF_WLO = OFF_WHI + W_BYTES;
+    // buffer b: hi at OFF_A(b), lo at OFF_A(b) + A_BYTES
+    static constexpr unsigned OFF_WHI = NBUF * 2 * A_BYTES, OFF_WLO = OFF_WHI + W_BYTES;
     static constexpr unsigned OFF_BIAS = OFF_WLO + W_BYTES;
-    static constexpr unsigned OFF_BAR = (OFF_BIAS + C * 4u + 15u) & ~15u;
-    static constexpr unsigned SMEM_BYTES = OFF_BAR + 16u + 128u;  // + alignment slack
-    static constexpr unsigned TMEM_COLS = C < 32 ? 32u : (unsigned)C;
+    static constexpr unsigned OFF_BAR = (OFF_BIAS + C * 4u + 15u) & ~15u;  // NBUF mbarriers, then the TMEM slot
+    static constexpr unsigned SMEM_BYTES = OFF_BAR + 32u + 128u;           // + alignment slack
+    static_assert(SMEM_BYTES <= kMaxSmem, "shared memory");
+    // one fp32 accumulator of C columns per buffer, in a power-of-two allocation >= 32
+    static constexpr unsigned TMEM_COLS = NBUF * C <= 32 ? 32u : (NBUF * C <= 64 ? 64u : 128u);
     static constexpr int NLOAD = (ROWS * KC + kGateThreads - 1) / kGateThreads;  // 4-vectors per thread
     static constexpr int NMMA = 3 * KT * (C / 8);
 };
@@ -165,56 +179,51 @@ __device__ __forceinline__ void store8(__nv_bfloat16 *p, const float (&v)[8], bo
     }
 }
 
+__device__ __forceinline__ void store4(float *p, const float (&v)[4], bool vec) {
+    if (vec) {
+        *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) p[i] = v[i];
+    }
+}
+__device__ __forceinline__ void store4(__nv_bfloat16 *p, const float (&v)[4], bool vec) {
+    const __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
+    const unsigned u0 = *reinterpret_cast<const unsigned *>(&h0), u1 = *reinterpret_cast<const unsigned *>(&h1);
+    if (vec) {
+        *reinterpret_cast<uint2 *>(p) = make_uint2(u0, u1);
+    } else {
+        uint16_t *q = reinterpret_cast<uint16_t *>(p);
+        q[0] = (uint16_t)(u0 & 0xFFFFu);
+        q[1] = (uint16_t)(u0 >> 16);
+        q[2] = (uint16_t)(u1 & 0xFFFFu);
+        q[3] = (uint16_t)(u1 >> 16);
+    }
+}
+
 // grid = H * groups CTAs; CTA (h = blockIdx.x % H, j = blockIdx.x / H) takes
 // the tiles j, j + groups, ... of head h, tile = b * tiles_per_row + t0 / 128.
-// vec_in: a's rows allow 4-channel vector loads; vec_out: g allows 16-byte
-// stores; vec_w: w is 16-byte aligned.
+// vec_in: a's rows allow 4-channel vector loads; vec_out: g allows 16-byte stores.
 template <int C, int KT, typename IO>
 __global__ void __launch_bounds__(kGateThreads, 1)
     mhf_gate_kernel(const IO *__restrict__ a, const float *__restrict__ w, const float *__restrict__ bias,
                     IO *__restrict__ g, int L, int D, int H, int groups, int tiles_per_row, int num_tiles,
-                    int vec_in, int vec_out, int vec_w) {
+                    int vec_in, int vec_out) {
     using Cfg = GateCfg<C, KT>;
     extern __shared__ unsigned char gate_smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(((uintptr_t)gate_smem_raw + 127) & ~(uintptr_t)127);
     const unsigned sb = smem_u32(sm);
     float *sbias = reinterpret_cast<float *>(sm + Cfg::OFF_BIAS);
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + Cfg::OFF_BAR);
-    unsigned *tslot = reinterpret_cast<unsigned *>(sm + Cfg::OFF_BAR + 8);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + Cfg::OFF_BAR);  // bar[0 .. NBUF-1]
+    unsigned *tslot = reinterpret_cast<unsigned *>(sm + Cfg::OFF_BAR + 16);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.x % H;
     const int64_t col0 = (int64_t)h * C;
 
     if (warp == 0) tmem_alloc(tslot, Cfg::TMEM_COLS);
-    if (tid == 0) mbar_init(bar, 1);
-
-    // The head's weights, split into tf32 hi / lo, in the K-major layout:
-    // tap k, chunk c/4, output channel n, element c%4.  w is [D][C][K]; the
-    // head's block is C*C*K contiguous floats, read 4 at a time.
-    const float *wh = w + col0 * C * KT;
-    auto put_w = [&](int i, float x) {
-        const int k = i % KT, c = (i / KT) % C, n = i / (KT * C);
-        float hi, lo;
-        split_tf32(x, hi, lo);
-        const unsigned off = k * Cfg::W_TAP + (c >> 2) * Cfg::LBO_W + n * 16u + (c & 3) * 4u;
-        *reinterpret_cast<float *>(sm + Cfg::OFF_WHI + off) = hi;
-        *reinterpret_cast<float *>(sm + Cfg::OFF_WLO + off) = lo;
-    };
-    if (vec_w) {
-#pragma unroll 4
-        for (int i4 = tid; i4 < C * C * KT / 4; i4 += kGateThreads) {
-            const float4 x = __ldg(reinterpret_cast<const float4 *>(wh) + i4);
-            put_w(4 * i4, x.x);
-            put_w(4 * i4 + 1, x.y);
-            put_w(4 * i4 + 2, x.z);
-            put_w(4 * i4 + 3, x.w);
-        }
-    } else {
-#pragma unroll 4
-        for (int i = tid; i < C * C * KT; i += kGateThreads) put_w(i, __ldg(wh + i));
-    }
-    if (tid < C) sbias[tid] = bias ? __ldg(bias + col0 + tid) : 0.0f;
+    if (tid == 0)
+        for (int i = 0; i < Cfg::NBUF; ++i) mbar_init(bar + i, 1);
 
     Raw4<IO> raw[Cfg::NLOAD];
     auto load_tile = [&](int tile) {
@@ -232,7 +241,8 @@ __global__ void __launch_bounds__(kGateThreads, 1)
                 raw[j].zero();
         }
     };
-    auto stage_tile = [&](int tile) {
+    auto stage_tile = [&](int tile, int buf) {
+        unsigned char *ahi = sm + buf * 2 * Cfg::A_BYTES, *alo = ahi + Cfg::A_BYTES;
         const int t0 = (tile % tiles_per_row) * kGateM;
 #pragma unroll
         for (int j = 0; j < Cfg::NLOAD; ++j) {
@@ -251,13 +261,36 @@ __global__ void __launch_bounds__(kGateThreads, 1)
             split_tf32(s.z, hi.z, lo.z);
             split_tf32(s.w, hi.w, lo.w);
             const unsigned off = kc * Cfg::LBO_A + r * 16u;
-            *reinterpret_cast<float4 *>(sm + Cfg::OFF_AHI + off) = hi;
-            *reinterpret_cast<float4 *>(sm + Cfg::OFF_ALO + off) = lo;
+            *reinterpret_cast<float4 *>(ahi + off) = hi;
+            *reinterpret_cast<float4 *>(alo + off) = lo;
         }
     };
 
+    // the first tile's a is in flight while the weights are staged
     int tile = blockIdx.x / H;
     if (tile < num_tiles) load_tile(tile);
+
+    // The head's weights, split into tf32 hi / lo, in the K-major layout:
+    // tap k, chunk c/4, output channel n, element c%4.  One thread fills one
+    // 16-byte slot (k, chunk, n) from four gathered loads of w ([D][C][K]);
+    // consecutive threads take consecutive n, so the slot stores are
+    // conflict-free.  (The head's block is read once per CTA, from L2 after
+    // the first CTA of the head.)
+    const float *wh = w + col0 * C * KT;
+#pragma unroll 2
+    for (int sl = tid; sl < KT * Cfg::KC * C; sl += kGateThreads) {
+        const int n = sl % C, kc = (sl / C) % Cfg::KC, k = sl / (C * Cfg::KC);
+        const float *src = wh + ((int64_t)n * C + kc * 4) * KT + k;
+        float4 hi, lo;
+        split_tf32(__ldg(src), hi.x, lo.x);
+        split_tf32(__ldg(src + KT), hi.y, lo.y);
+        split_tf32(__ldg(src + 2 * KT), hi.z, lo.z);
+        split_tf32(__ldg(src + 3 * KT), hi.w, lo.w);
+        const unsigned off = k * Cfg::W_TAP + kc * Cfg::LBO_W + n * 16u;
+        *reinterpret_cast<float4 *>(sm + Cfg::OFF_WHI + off) = hi;
+        *reinterpret_cast<float4 *>(sm + Cfg::OFF_WLO + off) = lo;
+    }
+    if (tid < C) sbias[tid] = bias ? __ldg(bias + col0 + tid) : 0.0f;
 
     tc_fence_before_sync();
     __syncthreads();
@@ -265,74 +298,109 @@ __global__ void __launch_bounds__(kGateThreads, 1)
     const unsigned tmem = *tslot;
     constexpr uint32_t idesc = umma_idesc_tf32(kGateM, C);
 
-    unsigned parity = 0;
-    bool ok = true;
-    for (; tile < num_tiles; tile += groups) {
-        // sigmoid(a) of this tile -> shared memory (the previous tile's MMAs
-        // have completed, and its accumulator has been read by every warp)
-        stage_tile(tile);
+    // MMAs of one tile: 3 split products x K taps x C/8 steps of 8 channels,
+    // into accumulator `buf`; committed to bar[buf].  Descriptors advance by
+    // (byte offset >> 4) in their address field.
+    auto issue = [&](int buf) {
+        const unsigned d = tmem + buf * C;
+        const unsigned abase = sb + buf * 2 * Cfg::A_BYTES;
+        int step = 0;
+#pragma unroll 1
+        for (int p = 0; p < 3; ++p) {  // hi*W_hi, hi*W_lo, lo*W_hi
+            const uint64_t a0 = umma_smem_desc(abase + (p < 2 ? 0u : Cfg::A_BYTES), Cfg::LBO_A, 128u);
+            const uint64_t b0 = umma_smem_desc(sb + (p == 1 ? Cfg::OFF_WLO : Cfg::OFF_WHI), Cfg::LBO_W, 128u);
+#pragma unroll
+            for (int k = 0; k < KT; ++k) {
+#pragma unroll
+                for (int s = 0; s < C / 8; ++s) {
+                    umma_tf32(d, a0 + ((k * 16u + 2u * s * Cfg::LBO_A) >> 4),
+                              b0 + ((k * Cfg::W_TAP + 2u * s * Cfg::LBO_W) >> 4), idesc, step > 0);
+                    ++step;
+                }
+            }
+        }
+        umma_commit(bar + buf);
+    };
+    // the staged tile (generic-proxy stores) is made visible to the tensor
+    // core, and every warp's earlier reads of the accumulator are ordered
+    // before the MMAs that overwrite it
+    auto publish = [&]() {
         fence_proxy_async_smem();
         tc_fence_before_sync();
         __syncthreads();
         tc_fence_after_sync();
-        if (tid == 0) {
-            int step = 0;
-#pragma unroll 1
-            for (int p = 0; p < 3; ++p) {  // hi*W_hi, hi*W_lo, lo*W_hi
-                const unsigned A = sb + (p < 2 ? Cfg::OFF_AHI : Cfg::OFF_ALO);
-                const unsigned W = sb + (p == 1 ? Cfg::OFF_WLO : Cfg::OFF_WHI);
-#pragma unroll 1
-                for (int k = 0; k < KT; ++k) {
-#pragma unroll
-                    for (int s = 0; s < C / 8; ++s) {
-                        const uint64_t ad = umma_smem_desc(A + k * 16u + 2u * s * Cfg::LBO_A, Cfg::LBO_A, 128u);
-                        const uint64_t bd = umma_smem_desc(W + k * Cfg::W_TAP + 2u * s * Cfg::LBO_W, Cfg::LBO_W, 128u);
-                        umma_tf32(tmem, ad, bd, idesc, step > 0);
-                        ++step;
-                    }
-                }
-            }
-            umma_commit(bar);
-        }
-        // the next tile's a streams into registers while the tensor core works
-        const int next = tile + groups;
-        if (next < num_tiles) load_tile(next);
+    };
 
-        const bool done = mbar_wait_bounded(bar, parity);
-        parity ^= 1u;
+    unsigned parity = 0u, pending = 0u;  // bit i: phase parity awaited on / MMAs in flight on bar[i]
+    bool ok = true;
+    if (tile < num_tiles) {
+        stage_tile(tile, 0);
+        publish();
+        if (tid == 0) issue(0);
+        pending |= 1u;
+        if (tile + groups < num_tiles) load_tile(tile + groups);
+    }
+    for (int it = 0; tile < num_tiles; tile += groups, ++it) {
+        const int cur = Cfg::NBUF == 2 ? (it & 1) : 0;
+        const int next = tile + groups;
+        if (Cfg::NBUF == 2 && next < num_tiles) {
+            // the other buffer's MMAs completed in the previous iteration
+            stage_tile(next, cur ^ 1);
+            publish();
+            if (tid == 0) issue(cur ^ 1);
+            pending |= 1u << (cur ^ 1);
+            if (next + groups < num_tiles) load_tile(next + groups);
+        }
+        // one thread waits for this tile's MMAs; the barrier releases the rest
+        bool done = true;
+        if (tid == 0) done = mbar_wait_bounded(bar + cur, (parity >> cur) & 1u);
         if (!__syncthreads_and(done)) {
             ok = false;
             break;
         }
+        parity ^= 1u << cur;
+        pending &= ~(1u << cur);
         tc_fence_after_sync();
 
-        // accumulator row = time step t0 + 32 (warp % 4) + lane; warps 0-3
-        // take the first half of the C columns, warps 4-7 the second
+        // accumulator row = time step t0 + 32 (warp % 4) + lane; warp w takes
+        // the column quarter w / 4 (warps w and w + 4 k share a lane quarter)
         const int b = tile / tiles_per_row;
-        const int q = warp & 3, cbase = (warp >> 2) * (C / 2);
+        const int q = warp & 3, cbase = (warp >> 2) * (C / 4);
         const int t = (tile % tiles_per_row) * kGateM + q * 32 + lane;
         IO *dst = g + ((int64_t)b * L + t) * D + col0 + cbase;
-        const unsigned trow = tmem + ((unsigned)(q * 32) << 16) + cbase;
-        if constexpr (C / 2 >= 16) {
+        const unsigned trow = tmem + cur * C + ((unsigned)(q * 32) << 16) + cbase;
+        if constexpr (C / 4 == 16) {
+            float v[16];
+            tmem_ld16(trow, v);
 #pragma unroll
-            for (int c0 = 0; c0 < C / 2; c0 += 16) {
-                float v[16];
-                tmem_ld16(trow + c0, v);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] += sbias[cbase + c0 + i];
-                if (t < L) store16(dst + c0, v, vec_out != 0);
-            }
-        } else {
+            for (int i = 0; i < 16; ++i) v[i] += sbias[cbase + i];
+            if (t < L) store16(dst, v, vec_out != 0);
+        } else if constexpr (C / 4 == 8) {
             float v[8];
             tmem_ld8(trow, v);
 #pragma unroll
             for (int i = 0; i < 8; ++i) v[i] += sbias[cbase + i];
             if (t < L) store8(dst, v, vec_out != 0);
+        } else {
+            float v[4];
+            tmem_ld4(trow, v);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[i] += sbias[cbase + i];
+            if (t < L) store4(dst, v, vec_out != 0);
+        }
+        if (Cfg::NBUF == 1 && next < num_tiles) {
+            // single buffer: the next tile is staged once this one's MMAs are done
+            stage_tile(next, 0);
+            publish();
+            if (tid == 0) issue(0);
+            pending |= 1u;
+            if (next + groups < num_tiles) load_tile(next + groups);
         }
     }
-    if (!ok) {
-        if (tid == 0) atomicOr(&g_cc_fault, kFaultMmaWait);
-        mbar_wait_bounded(bar, parity ^ 1u);  // give the MMAs in flight a last chance to finish
+    if (!ok && tid == 0) {
+        atomicOr(&g_cc_fault, kFaultMmaWait);
+        for (int i = 0; i < Cfg::NBUF; ++i)  // give the MMAs in flight a last chance to finish
+            if ((pending >> i) & 1u) mbar_wait_bounded(bar + i, (parity >> i) & 1u);
     }
     tc_fence_before_sync();
     __syncthreads();

@@ -104,4 +104,17 @@ __device__ __forceinline__ void tmem_ld8(unsigned taddr, float (&v)[8]) {
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 4 consecutive fp32 columns of this thread's TMEM lane (load and wait together).
+__device__ __forceinline__ void tmem_ld4(unsigned taddr, float (&v)[4]) {
+    unsigned r[4];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];\n"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 }  // namespace ccv
