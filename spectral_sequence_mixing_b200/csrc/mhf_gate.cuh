@@ -27,11 +27,12 @@
 // stores sigmoid(a) (hi, lo) to shared memory, one thread issues 3 K C/8
 // MMAs and commits them to an mbarrier, and the sixteen warps read the
 // accumulator back (warp w: TMEM lanes 32 (w % 4) .. +31 = time steps, a
-// quarter of the columns each), add the bias and store g.  With two tile
+// quarter of the columns each), add the bias, stage the rows in shared memory
+// and store g as whole rows (coalesced).  With two tile
 // buffers and two accumulators (every head width and tap count whose tiles
 // fit twice) the tensor core works on tile i+1 while the warps drain tile i
-// and stage tile i+2; the a of the tile after that streams into registers
-// meanwhile.  Every wait is bounded; no
+// and stage tile i+2; a for the two tiles after that streams into two
+// register sets meanwhile.  Every wait is bounded; no
 // load uses cluster multicast.
 #pragma once
 
@@ -79,6 +80,8 @@ struct GateCfg {
     static constexpr unsigned TMEM_COLS = NBUF * C <= 32 ? 32u : (NBUF * C <= 64 ? 64u : 128u);
     static constexpr int NLOAD = (ROWS * KC + kGateThreads - 1) / kGateThreads;  // 4-vectors per thread
     static constexpr int NMMA = 3 * KT * (C / 8);
+    static constexpr int OPITCH = C + 4;  // row pitch (floats) of the output tile staged in a free tile buffer
+    static_assert(kGateM * OPITCH * 4u <= 2u * A_BYTES, "output tile must fit in one tile buffer");
 };
 
 __device__ __forceinline__ void split_tf32(float x, float &hi, float &lo) {
@@ -91,14 +94,22 @@ __device__ __forceinline__ void split_tf32(float x, float &hi, float &lo) {
 // large negative x gives exp = inf and 1/inf = 0.
 __device__ __forceinline__ float logistic(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 
-// Four consecutive channels of a, as loaded (fp32: one 16-byte load; bf16: 8 bytes).
+// Four consecutive channels of a, as loaded (fp32: one 16-byte load; bf16:
+// 8 bytes).  The vector loads are volatile asm so that they issue where they
+// are written -- a tile or two before their use -- and are not moved next
+// to it.
 template <typename IO>
 struct Raw4;
 template <>
 struct Raw4<float> {
     float4 x;
     __device__ __forceinline__ void load(const float *p, bool vec) {
-        x = vec ? __ldg(reinterpret_cast<const float4 *>(p)) : make_float4(p[0], p[1], p[2], p[3]);
+        if (vec)
+            asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(x.x), "=f"(x.y), "=f"(x.z), "=f"(x.w)
+                         : "l"(p));
+        else
+            x = make_float4(p[0], p[1], p[2], p[3]);
     }
     __device__ __forceinline__ void zero() { x = make_float4(0.f, 0.f, 0.f, 0.f); }
     __device__ __forceinline__ float4 f32() const { return x; }
@@ -108,7 +119,7 @@ struct Raw4<__nv_bfloat16> {
     uint2 x;
     __device__ __forceinline__ void load(const __nv_bfloat16 *p, bool vec) {
         if (vec) {
-            x = __ldg(reinterpret_cast<const uint2 *>(p));
+            asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(x.x), "=r"(x.y) : "l"(p));
         } else {
             const uint16_t *q = reinterpret_cast<const uint16_t *>(p);
             x = make_uint2((unsigned)q[0] | ((unsigned)q[1] << 16), (unsigned)q[2] | ((unsigned)q[3] << 16));
@@ -121,64 +132,7 @@ struct Raw4<__nv_bfloat16> {
     }
 };
 
-// Store 16 consecutive output channels of one time step.
-__device__ __forceinline__ void store16(float *p, const float (&v)[16], bool vec) {
-    if (vec) {
-#pragma unroll
-        for (int i = 0; i < 16; i += 4) reinterpret_cast<float4 *>(p)[i / 4] = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-    } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) p[i] = v[i];
-    }
-}
-__device__ __forceinline__ void store16(__nv_bfloat16 *p, const float (&v)[16], bool vec) {
-    unsigned u[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-        u[i] = *reinterpret_cast<const unsigned *>(&h);
-    }
-    if (vec) {
-        reinterpret_cast<uint4 *>(p)[0] = make_uint4(u[0], u[1], u[2], u[3]);
-        reinterpret_cast<uint4 *>(p)[1] = make_uint4(u[4], u[5], u[6], u[7]);
-    } else {
-        uint16_t *q = reinterpret_cast<uint16_t *>(p);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            q[2 * i] = (uint16_t)(u[i] & 0xFFFFu);
-            q[2 * i + 1] = (uint16_t)(u[i] >> 16);
-        }
-    }
-}
-
-__device__ __forceinline__ void store8(float *p, const float (&v)[8], bool vec) {
-    if (vec) {
-        reinterpret_cast<float4 *>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
-        reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) p[i] = v[i];
-    }
-}
-__device__ __forceinline__ void store8(__nv_bfloat16 *p, const float (&v)[8], bool vec) {
-    unsigned u[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-        u[i] = *reinterpret_cast<const unsigned *>(&h);
-    }
-    if (vec) {
-        reinterpret_cast<uint4 *>(p)[0] = make_uint4(u[0], u[1], u[2], u[3]);
-    } else {
-        uint16_t *q = reinterpret_cast<uint16_t *>(p);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            q[2 * i] = (uint16_t)(u[i] & 0xFFFFu);
-            q[2 * i + 1] = (uint16_t)(u[i] >> 16);
-        }
-    }
-}
-
+// Store 4 consecutive output channels of one time step.
 __device__ __forceinline__ void store4(float *p, const float (&v)[4], bool vec) {
     if (vec) {
         *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
@@ -225,8 +179,10 @@ __global__ void __launch_bounds__(kGateThreads, 1)
     if (tid == 0)
         for (int i = 0; i < Cfg::NBUF; ++i) mbar_init(bar + i, 1);
 
-    Raw4<IO> raw[Cfg::NLOAD];
-    auto load_tile = [&](int tile) {
+    // Two register sets of raw a: tile j of this CTA's sequence uses set j % 2,
+    // so the loads of tiles j+2 and j+3 are in flight while j+1 is staged.
+    Raw4<IO> raw0[Cfg::NLOAD], raw1[Cfg::NLOAD];
+    auto load_tile = [&](Raw4<IO>(&raw)[Cfg::NLOAD], int tile) {
         const int b = tile / tiles_per_row;
         const int t0 = (tile % tiles_per_row) * kGateM;
         const IO *base = a + (int64_t)b * L * D + col0;
@@ -241,7 +197,7 @@ __global__ void __launch_bounds__(kGateThreads, 1)
                 raw[j].zero();
         }
     };
-    auto stage_tile = [&](int tile, int buf) {
+    auto stage_tile = [&](Raw4<IO>(&raw)[Cfg::NLOAD], int tile, int buf) {
         unsigned char *ahi = sm + buf * 2 * Cfg::A_BYTES, *alo = ahi + Cfg::A_BYTES;
         const int t0 = (tile % tiles_per_row) * kGateM;
 #pragma unroll
@@ -266,9 +222,10 @@ __global__ void __launch_bounds__(kGateThreads, 1)
         }
     };
 
-    // the first tile's a is in flight while the weights are staged
+    // the first two tiles' a is in flight while the weights are staged
     int tile = blockIdx.x / H;
-    if (tile < num_tiles) load_tile(tile);
+    if (tile < num_tiles) load_tile(raw0, tile);
+    if (tile + groups < num_tiles) load_tile(raw1, tile + groups);
 
     // The head's weights, split into tf32 hi / lo, in the K-major layout:
     // tap k, chunk c/4, output channel n, element c%4.  One thread fills one
@@ -299,7 +256,7 @@ __global__ void __launch_bounds__(kGateThreads, 1)
     constexpr uint32_t idesc = umma_idesc_tf32(kGateM, C);
 
     // MMAs of one tile: 3 split products x K taps x C/8 steps of 8 channels,
-    // into accumulator `buf`; committed to bar[buf].  Descriptors advance by
+    // into accumulator `buf`; committed to bar[buf].  Run by all of warp 0.  Descriptors advance by
     // (byte offset >> 4) in their address field.
     auto issue = [&](int buf) {
         const unsigned d = tmem + buf * C;
@@ -313,13 +270,13 @@ __global__ void __launch_bounds__(kGateThreads, 1)
             for (int k = 0; k < KT; ++k) {
 #pragma unroll
                 for (int s = 0; s < C / 8; ++s) {
-                    umma_tf32(d, a0 + ((k * 16u + 2u * s * Cfg::LBO_A) >> 4),
+                    umma_tf32_elect(d, a0 + ((k * 16u + 2u * s * Cfg::LBO_A) >> 4),
                               b0 + ((k * Cfg::W_TAP + 2u * s * Cfg::LBO_W) >> 4), idesc, step > 0);
                     ++step;
                 }
             }
         }
-        umma_commit(bar + buf);
+        umma_commit_elect(bar + buf);
     };
     // the staged tile (generic-proxy stores) is made visible to the tensor
     // core, and every warp's earlier reads of the accumulator are ordered
@@ -331,25 +288,32 @@ __global__ void __launch_bounds__(kGateThreads, 1)
         tc_fence_after_sync();
     };
 
+    // stage tile `stile` from register set s into tile buffer `buf`, start its
+    // MMAs, then refill set s with tile `ltile` (the one two places later)
+    auto stage_issue_load = [&](int s, int stile, int buf, int ltile) {
+        if (s) stage_tile(raw1, stile, buf);
+        else stage_tile(raw0, stile, buf);
+        publish();
+        if (warp == 0) issue(buf);  // the whole warp runs the loop, one lane issues
+        if (ltile < num_tiles) {
+            if (s) load_tile(raw1, ltile);
+            else load_tile(raw0, ltile);
+        }
+    };
+
     unsigned parity = 0u, pending = 0u;  // bit i: phase parity awaited on / MMAs in flight on bar[i]
     bool ok = true;
     if (tile < num_tiles) {
-        stage_tile(tile, 0);
-        publish();
-        if (tid == 0) issue(0);
+        stage_issue_load(0, tile, 0, tile + 2 * groups);
         pending |= 1u;
-        if (tile + groups < num_tiles) load_tile(tile + groups);
     }
     for (int it = 0; tile < num_tiles; tile += groups, ++it) {
         const int cur = Cfg::NBUF == 2 ? (it & 1) : 0;
         const int next = tile + groups;
         if (Cfg::NBUF == 2 && next < num_tiles) {
             // the other buffer's MMAs completed in the previous iteration
-            stage_tile(next, cur ^ 1);
-            publish();
-            if (tid == 0) issue(cur ^ 1);
+            stage_issue_load((it + 1) & 1, next, cur ^ 1, next + 2 * groups);
             pending |= 1u << (cur ^ 1);
-            if (next + groups < num_tiles) load_tile(next + groups);
         }
         // one thread waits for this tile's MMAs; the barrier releases the rest
         bool done = true;
@@ -362,39 +326,56 @@ __global__ void __launch_bounds__(kGateThreads, 1)
         pending &= ~(1u << cur);
         tc_fence_after_sync();
 
-        // accumulator row = time step t0 + 32 (warp % 4) + lane; warp w takes
-        // the column quarter w / 4 (warps w and w + 4 k share a lane quarter)
-        const int b = tile / tiles_per_row;
-        const int q = warp & 3, cbase = (warp >> 2) * (C / 4);
-        const int t = (tile % tiles_per_row) * kGateM + q * 32 + lane;
-        IO *dst = g + ((int64_t)b * L + t) * D + col0 + cbase;
-        const unsigned trow = tmem + cur * C + ((unsigned)(q * 32) << 16) + cbase;
-        if constexpr (C / 4 == 16) {
-            float v[16];
-            tmem_ld16(trow, v);
+        // accumulator row m = 32 (warp % 4) + lane (time step t0 + m); warp w
+        // takes the column quarter w / 4.  Rows are staged (with the bias) in
+        // this tile's buffer, whose MMAs are done, then written out as whole
+        // C-channel rows by consecutive threads.
+        {
+            const int q = warp & 3, cbase = (warp >> 2) * (C / 4);
+            float *otile = reinterpret_cast<float *>(sm + cur * 2 * Cfg::A_BYTES);
+            float *orow = otile + (q * 32 + lane) * Cfg::OPITCH + cbase;
+            const unsigned trow = tmem + cur * C + ((unsigned)(q * 32) << 16) + cbase;
+            if constexpr (C / 4 == 16) {
+                float v[16];
+                tmem_ld16(trow, v);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] += sbias[cbase + i];
-            if (t < L) store16(dst, v, vec_out != 0);
-        } else if constexpr (C / 4 == 8) {
-            float v[8];
-            tmem_ld8(trow, v);
+                for (int i = 0; i < 16; i += 4)
+                    *reinterpret_cast<float4 *>(orow + i) = make_float4(
+                        v[i] + sbias[cbase + i], v[i + 1] + sbias[cbase + i + 1], v[i + 2] + sbias[cbase + i + 2],
+                        v[i + 3] + sbias[cbase + i + 3]);
+            } else if constexpr (C / 4 == 8) {
+                float v[8];
+                tmem_ld8(trow, v);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] += sbias[cbase + i];
-            if (t < L) store8(dst, v, vec_out != 0);
-        } else {
-            float v[4];
-            tmem_ld4(trow, v);
+                for (int i = 0; i < 8; i += 4)
+                    *reinterpret_cast<float4 *>(orow + i) = make_float4(
+                        v[i] + sbias[cbase + i], v[i + 1] + sbias[cbase + i + 1], v[i + 2] + sbias[cbase + i + 2],
+                        v[i + 3] + sbias[cbase + i + 3]);
+            } else {
+                float v[4];
+                tmem_ld4(trow, v);
+                *reinterpret_cast<float4 *>(orow) =
+                    make_float4(v[0] + sbias[cbase], v[1] + sbias[cbase + 1], v[2] + sbias[cbase + 2],
+                                v[3] + sbias[cbase + 3]);
+            }
+            __syncthreads();
+            const int b = tile / tiles_per_row, t0 = (tile % tiles_per_row) * kGateM;
+            IO *gt = g + ((int64_t)b * L + t0) * D + col0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) v[i] += sbias[cbase + i];
-            if (t < L) store4(dst, v, vec_out != 0);
+            for (int i = tid; i < kGateM * (C / 4); i += kGateThreads) {
+                const int m = i / (C / 4), c4 = i % (C / 4);
+                if (t0 + m < L) {
+                    const float4 x = *reinterpret_cast<const float4 *>(otile + m * Cfg::OPITCH + 4 * c4);
+                    const float xv[4] = {x.x, x.y, x.z, x.w};
+                    store4(gt + (int64_t)m * D + 4 * c4, xv, vec_out != 0);
+                }
+            }
+            __syncthreads();  // the buffer is staged into again
         }
         if (Cfg::NBUF == 1 && next < num_tiles) {
             // single buffer: the next tile is staged once this one's MMAs are done
-            stage_tile(next, 0);
-            publish();
-            if (tid == 0) issue(0);
+            stage_issue_load((it + 1) & 1, next, 0, next + 2 * groups);
             pending |= 1u;
-            if (next + groups < num_tiles) load_tile(next + groups);
         }
     }
     if (!ok && tid == 0) {
