@@ -22,7 +22,9 @@ when the true sum does not fit in (-p/2, p/2).
 
 The submodule ``oracle.mhf_gate`` adds the gate stream of the same block
 (sigmoid and the head-grouped causal Conv1d_G2, float64 numpy) and composes it
-with this sum; its pins are in tests/test_oracle_mhf_pins.py.
+with this sum; its pins are in tests/test_oracle_mhf_pins.py.  The submodule
+``oracle.mhf_dwconv`` is the block's first step, the causal depthwise
+convolution (kernel size 3 on the page); pins in tests/test_oracle_dwconv_pins.py.
 
 Pins (tests/test_oracle_pins.py): hand-computed fixtures in tests/golden/,
 delta inputs, closed-form sums, numpy.convolve on single rows, an fp64 FFT
