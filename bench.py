@@ -45,7 +45,9 @@ KERNEL_SOURCES = {
     "bigconv_kernel": ["bigconv.cuh", "configs_rows.cuh", "transpose.cuh"] + _FUSED_SOURCES,
     "ntt_conv_kernel": ["ntt.cuh"],
     "mhf_gate_kernel": ["mhf_gate.cuh", "tcgen05.cuh", "tma.cuh"],
+    "dwconv_vec_kernel": ["dwconv.cuh"],
 }
+DWCONV_METRIC = "causal depthwise conv GB/s (x in, y out) at 1 B200; % of HBM roofline"
 GATE_METRIC = "MHF gate stream + causal FFT-conv GB/s (v, a in, r out) at 1 B200; % of HBM roofline"
 
 
@@ -56,8 +58,10 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="small_f32",
-                    choices=sorted(workloads.WORKLOADS) + sorted(workloads.GATE_WORKLOADS),
-                    help="a convolution workload, or a gate workload (MHF gate stream + convolution)")
+                    choices=sorted(workloads.WORKLOADS) + sorted(workloads.GATE_WORKLOADS)
+                    + sorted(workloads.DWCONV_WORKLOADS),
+                    help="a convolution workload, a gate workload (MHF gate stream + convolution) "
+                         "or a depthwise-convolution workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--path", choices=["fwd", "bwd", "decode"], default="fwd",
@@ -678,19 +682,196 @@ def run_gated_reference(args, rank, world):
     }), flush=True)
 
 
+def run_dwconv(args, rank, world, local):
+    """The block's causal depthwise convolution: one step = one launch."""
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    dw = workloads.DWCONV_WORKLOADS[args.workload]
+    x, w, bias = workloads.generate_dwconv(dw.B, dw.L, dw.D, dw.K, dw.dtype, dw.seed + 1000 * rank)
+    es = 4 if dw.dtype == "f32" else 2
+    hx = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16) if dw.dtype == "bf16" else torch.from_numpy(x)
+    tw, tb = torch.from_numpy(w).to(dev), torch.from_numpy(bias).to(dev)
+    units = dw.units
+    set_bytes = 2 * units * es
+    n_sets = max(2, math.ceil(2.2 * L2_BYTES / set_bytes))
+    x0 = hx.to(dev)
+    sets = [(x0 if i == 0 else x0.clone(), torch.empty_like(x0)) for i in range(n_sets)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):  # on the current stream (the capture stream inside a graph capture)
+        sx, sy = sets[i % n_sets]
+        ssm.causal_dwconv(sx, tw, tb, out=sy)
+
+    def timed(fn, steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for i in range(steps):
+            fn(i)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1), pg, dev)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    # A step (~8 us of device time) is shorter than a Python call through the
+    # binding, so the steps are replayed from CUDA graphs: one graph of G
+    # consecutive steps (whole rotations of the buffer sets) and one graph per
+    # set for the remainder; every step is still one launch on its own buffers.
+    G = n_sets * max(1, 64 // n_sets)
+    big = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(big):
+        for i in range(G):
+            step(i)
+    singles = []
+    for k in range(n_sets):
+        gk = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gk):
+            step(k)
+        singles.append(gk)
+    torch.cuda.synchronize(dev)
+
+    def run_steps(n):
+        for _ in range(n // G):
+            big.replay()
+        for i in range(n % G):
+            singles[i % n_sets].replay()
+
+    run_steps(G)
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    with ClockSampler(local) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        run_steps(args.steps)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ms = max_over_ranks(e0.elapsed_time(e1), pg, dev)
+    clocks = clk.report()
+    ms_per_step = ms / args.steps
+    alg_bytes = 2 * units * es + dw.D * (dw.K + 1) * 4
+    gbs = alg_bytes * world * args.steps / (ms * 1e-3) / 1e9
+
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    phx = hx.pin_memory()
+    phy = torch.empty_like(phx).pin_memory()
+    dx_, dy_ = sets[0]
+
+    def e2e_step(_i):
+        dx_.copy_(phx, non_blocking=True)
+        ssm.causal_dwconv(dx_, tw, tb, out=dy_)
+        phy.copy_(dy_, non_blocking=True)
+
+    for i in range(2):
+        e2e_step(i)
+    ems = timed(e2e_step, e2e_steps)
+    e2e_gbs = alg_bytes * world * e2e_steps / (ems * 1e-3) / 1e9
+    peak, peak_src = measured_peaks()
+    achieved = alg_bytes / (ms_per_step * 1e-3) / 1e9
+    traffic, _, _ = recorded_counters(dw.name, "dwconv_vec_kernel")
+    line = {
+        "metric": DWCONV_METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": dw.name, "path": "dwconv", "B": dw.B, "L": dw.L, "D": dw.D, "taps": dw.K,
+                   "io_dtype": dw.dtype,
+                   "l2": f"inputs larger than L2: {n_sets} rotating (x,y) sets of {set_bytes / 2 ** 20:.0f} MiB",
+                   "launch": f"steps replayed from CUDA graphs ({G} steps per graph)",
+                   "parallelism": f"dp{world} (independent batches, no collective)"},
+        "outputs_per_s": units * world * args.steps / (ms * 1e-3),
+        "hbm_frac": gbs / world / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)", "kernel": "dwconv_vec_kernel",
+                     "algorithmic_bytes_per_launch": alg_bytes, "traffic": traffic},
+        "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": units * es, "d2h_bytes_per_step": units * es,
+                "steps": e2e_steps, "path": "pinned host x -> device; causal_dwconv; y -> pinned host"},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        import oracle.mhf_dwconv as odw
+        xf = workloads.bf16_to_f32(x) if dw.dtype == "bf16" else x
+        reps, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < 15.0 and reps < 200:
+            odw.causal_dwconv(xf, w, bias)
+            reps += 1
+        secs = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": units * reps * 2 * es / secs / 1e9, "unit": "GB/s",
+                                "cores": oracle.num_threads(), "kind": "oracle",
+                                "sample": f"oracle (float64 numpy) on the whole {dw.name}, {reps} passes",
+                                "seconds": secs}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def run_dwconv_reference(args, rank, world):
+    """The oracle (float64 numpy) on the host cores, same metric."""
+    if rank != 0:
+        return
+    dw = workloads.DWCONV_WORKLOADS[args.workload]
+    x, w, bias = workloads.generate_dwconv(dw.B, dw.L, dw.D, dw.K, "f32", dw.seed)
+    import oracle
+    import oracle.mhf_dwconv as odw
+    for _ in range(args.warmup):
+        odw.causal_dwconv(x, w, bias)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        odw.causal_dwconv(x, w, bias)
+    el = time.perf_counter() - t0
+    es = 4 if dw.dtype == "f32" else 2
+    gbs = dw.units * args.steps * 2 * es / el / 1e9
+    print(json.dumps({
+        "impl": "reference", "metric": DWCONV_METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": dw.name, "path": "dwconv", "B": dw.B, "L": dw.L, "D": dw.D, "taps": dw.K,
+                   "io_dtype": dw.dtype},
+        "outputs_per_s": dw.units * args.steps / el,
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"oracle (float64 numpy) on the whole {dw.name} per step"},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def main():
     args = parse_args()
     rank, world, local = dist_env()
     if world != args.gpus and "RANK" in os.environ:
         print(f"warning: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
     gated = args.workload in workloads.GATE_WORKLOADS
+    dwconv = args.workload in workloads.DWCONV_WORKLOADS
     if args.impl == "reference":
-        (run_gated_reference if gated else run_reference)(args, rank, world)
+        (run_gated_reference if gated else run_dwconv_reference if dwconv else run_reference)(args, rank, world)
+    elif gated:
+        run_gated(args, rank, world, local)
+    elif dwconv:
+        run_dwconv(args, rank, world, local)
     else:
-        if gated:
-            run_gated(args, rank, world, local)
-        else:
-            run_ours(args, rank, world, local)
+        run_ours(args, rank, world, local)
 
 
 if __name__ == "__main__":

@@ -311,6 +311,31 @@ CC_API int causal_mhf_gated_conv_bf16(const uint16_t *v, const uint16_t *a, cons
 CC_API size_t causal_mhf_gated_conv_workspace_bytes(int dtype, int64_t B, int64_t L, int64_t D);
 
 /*
+ * causal_dwconv_f32 / _bf16 -- the causal depthwise convolution that opens the
+ * Multi-Head Fourier block (Caracal: Causal Architecture via Spectral Mixing,
+ * "Key design 1": a causal depthwise 1-D convolution, kernel size 3):
+ *
+ *   y[b,t,d] = bias[d] + sum_{k<K} w[d][k] * x[b, t-(K-1)+k, d]
+ *
+ * terms with t-(K-1)+k < 0 left out (K-1 zeros on the left, none on the
+ * right).  The output is the convolution alone (any residual connection is
+ * the caller's).
+ *   x     [B, L, D] device array, channel-last (bf16: uint16 bit patterns);
+ *   w     [D, K] float32 device array (a depthwise Conv1d weight [D, 1, K]);
+ *   bias  [D] float32 device array, or NULL;
+ *   y     [B, L, D] device output of x's dtype (bf16: rounded to nearest
+ *         even), overlapping neither x, w nor bias (CC_ERR_ALIAS);
+ *   K     1..8 taps (the page's value is 3), else CC_ERR_UNSUPPORTED
+ *         (K < 1: CC_ERR_INVALID_ARG).  L is not limited by a transform length.
+ * fp32 arithmetic (fused multiply-adds in tap order).  Stream-ordered and
+ * asynchronous; allocates nothing; errors are returned before any launch.
+ */
+CC_API int causal_dwconv_f32(const float *x, const float *w, const float *bias, float *y, int64_t B, int64_t L,
+                             int64_t D, int64_t K, void *stream);
+CC_API int causal_dwconv_bf16(const uint16_t *x, const float *w, const float *bias, uint16_t *y, int64_t B, int64_t L,
+                              int64_t D, int64_t K, void *stream);
+
+/*
  * causal_conv_fault_flags -- the library's per-device fault word.  The pages
  * have no counterpart: it reports waits inside the kernels that ran out of
  * time.  Every wait in the kernels (on an asynchronous copy, an mbarrier) is

@@ -25,7 +25,7 @@ __all__ = [
     "causal_fftconv_f32", "causal_fftconv_bf16", "causal_ntt_conv_i32", "causal_conv", "causal_conv_bwd",
     "causal_conv_decode", "decode_workspace_bytes",
     "causal_conv_from_host", "workspace_bytes", "fast_workspace_bytes", "max_len", "ntt_params", "strerror",
-    "fault_flags", "mhf_gate", "mhf_gated_conv", "mhf_gated_conv_workspace_bytes",
+    "fault_flags", "mhf_gate", "mhf_gated_conv", "mhf_gated_conv_workspace_bytes", "causal_dwconv",
     "CausalConvError", "CC_DTYPE_F32", "CC_DTYPE_BF16", "CC_DTYPE_I32",
 ]
 
@@ -305,4 +305,39 @@ def mhf_gated_conv(v: torch.Tensor, a: torch.Tensor, w: torch.Tensor, bias: torc
                 _stream_ptr(stream))
     if st != 0:
         raise CausalConvError(st, _GATED_FN[v.dtype])
+    return out
+
+
+# ------------------------------------------------------------------ depthwise convolution
+_DW_FN = {torch.float32: "causal_dwconv_f32", torch.bfloat16: "causal_dwconv_bf16"}
+
+
+def causal_dwconv(x: torch.Tensor, w: torch.Tensor, bias: torch.Tensor | None = None, out=None,
+                  stream=None) -> torch.Tensor:
+    """y = the causal depthwise convolution of x ([B, L, D] float32 / bfloat16)
+    with w ([D, K] or [D, 1, K] float32) and bias ([D] float32 or None)."""
+    if x.dtype not in _DW_FN:
+        raise TypeError(f"unsupported dtype {x.dtype}")
+    _check(x, "x", x.dtype)
+    if not x.is_cuda:
+        raise ValueError("x must be a CUDA tensor")
+    B, L, D = x.shape
+    if not isinstance(w, torch.Tensor) or w.dtype != torch.float32:
+        raise TypeError("w must be a float32 tensor [D, K] or [D, 1, K]")
+    if w.dim() == 3 and w.shape[1] == 1:
+        w = w.reshape(w.shape[0], w.shape[2])
+    if w.dim() != 2 or w.shape[0] != D or not w.is_contiguous() or w.device != x.device:
+        raise ValueError(f"w must be contiguous [D={D}, K] on the device of x, got {tuple(w.shape)}")
+    if bias is not None and (not isinstance(bias, torch.Tensor) or bias.dtype != torch.float32
+                             or tuple(bias.shape) != (D,) or not bias.is_contiguous() or bias.device != x.device):
+        raise ValueError("bias must be a contiguous float32 tensor [D] on the device of x, or None")
+    if out is None:
+        out = torch.empty_like(x)
+    _check(out, "out", x.dtype, x.shape)
+    fn = getattr(load(), _DW_FN[x.dtype])
+    with torch.cuda.device(x.device):
+        st = fn(x.data_ptr(), w.data_ptr(), bias.data_ptr() if bias is not None else None, out.data_ptr(), B, L, D,
+                int(w.shape[1]), _stream_ptr(stream))
+    if st != 0:
+        raise CausalConvError(st, _DW_FN[x.dtype])
     return out

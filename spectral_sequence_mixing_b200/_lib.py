@@ -41,6 +41,8 @@ SIGNATURES = {
     "causal_mhf_gated_conv_f32": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "causal_mhf_gated_conv_bf16": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "causal_mhf_gated_conv_workspace_bytes": (_SZ, [ctypes.c_int, _I64, _I64, _I64]),
+    "causal_dwconv_f32": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
+    "causal_dwconv_bf16": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
 }
 
 _lib = None

@@ -24,6 +24,7 @@
 #include "decode.cuh"
 #include "transpose.cuh"
 #include "mhf_gate.cuh"
+#include "dwconv.cuh"
 #include "configs.cuh"
 
 namespace ccv {
@@ -702,6 +703,27 @@ static int gated_conv_entry(int dtype, const IO *v, const IO *a, const float *w,
     return fftconv_dispatch<IO>(v, gbuf, r, B, L, D, nullptr, 0, s, dev);
 }
 
+// ------------------------------------------------------------------ depthwise conv
+template <typename IO>
+static int dwconv_entry(int dtype, const IO *x, const float *w, const float *bias, IO *y, int64_t B, int64_t L,
+                        int64_t D, int64_t K, cudaStream_t s) {
+    if (!x || !w || !y) return CC_ERR_INVALID_ARG;
+    const size_t es = dtype_size(dtype);
+    if (B < 1 || L < 1 || D < 1 || K < 1) return CC_ERR_INVALID_ARG;
+    if (L > INT32_MAX || D > INT32_MAX || B > INT32_MAX) return CC_ERR_INVALID_ARG;
+    const int64_t lim = INT64_MAX / (int64_t)es;
+    if (L > lim / D || B > lim / (L * D)) return CC_ERR_INVALID_ARG;
+    if (K > kDwMaxTaps) return CC_ERR_UNSUPPORTED;
+    const size_t bytes = (size_t)(B * L * D) * es;
+    if (ranges_overlap(y, bytes, x, bytes) || ranges_overlap(y, bytes, w, (size_t)(D * K) * sizeof(float)) ||
+        (bias && ranges_overlap(y, bytes, bias, (size_t)D * sizeof(float))))
+        return CC_ERR_ALIAS;
+    int dev, st;
+    if ((st = check_device({x, w, y}, &dev)) != CC_OK) return st;
+    if (bias && (st = check_device_ptr(bias, dev)) != CC_OK) return st;
+    return launch_dwconv<IO>(x, w, bias, y, B, L, D, K, s, dev);
+}
+
 extern "C" {
 
 size_t causal_conv_workspace_bytes(int dtype, int64_t B, int64_t L, int64_t D) {
@@ -904,6 +926,17 @@ int causal_mhf_gated_conv_bf16(const uint16_t *v, const uint16_t *a, const float
     return gated_conv_entry<__nv_bfloat16>(CC_DTYPE_BF16, (const __nv_bfloat16 *)v, (const __nv_bfloat16 *)a, w, bias,
                                            (__nv_bfloat16 *)r, B, L, D, H, K, workspace, workspace_bytes,
                                            (cudaStream_t)stream);
+}
+
+int causal_dwconv_f32(const float *x, const float *w, const float *bias, float *y, int64_t B, int64_t L, int64_t D,
+                      int64_t K, void *stream) {
+    return dwconv_entry<float>(CC_DTYPE_F32, x, w, bias, y, B, L, D, K, (cudaStream_t)stream);
+}
+
+int causal_dwconv_bf16(const uint16_t *x, const float *w, const float *bias, uint16_t *y, int64_t B, int64_t L,
+                       int64_t D, int64_t K, void *stream) {
+    return dwconv_entry<__nv_bfloat16>(CC_DTYPE_BF16, (const __nv_bfloat16 *)x, w, bias, (__nv_bfloat16 *)y, B, L, D,
+                                       K, (cudaStream_t)stream);
 }
 
 int causal_conv_fault_flags(int device, unsigned int *flags, int clear) {

@@ -211,3 +211,19 @@ def test_gated_conv_host_side_checks(lib):
     assert f(V_, A, W_, None, R_, *ok, V_ + 64, need, None) == 3        # workspace overlaps v
     assert f(V_, A, W_, None, R_, *ok, R_ - 64, need, None) == 3        # workspace overlaps r
     assert f(V_, A, W_, None, R_, 1, 16, 96, 2, 1, S_, 16 * 96 * 4, None) == 2  # head width 48
+
+
+@pytest.mark.parametrize("fn", ["causal_dwconv_f32", "causal_dwconv_bf16"])
+def test_dwconv_host_side_argument_errors(lib, fn):
+    f = getattr(lib, fn)
+    W_, Y_ = 0x40000000, 0x50000000
+    ok = (1, 16, 64, 3)
+    assert f(None, W_, None, Y_, *ok, None) == 1
+    assert f(A, None, None, Y_, *ok, None) == 1
+    assert f(A, W_, None, None, *ok, None) == 1
+    for shape in [(0, 16, 64, 3), (1, 0, 64, 3), (1, 16, 0, 3), (1, 16, 64, 0), (2 ** 40, 2 ** 20, 2 ** 10, 3)]:
+        assert f(A, W_, None, Y_, *shape, None) == 1, shape
+    assert f(A, W_, None, Y_, 1, 16, 64, 9, None) == 2          # more than 8 taps
+    assert f(A, W_, None, A + 64, *ok, None) == 3               # y overlaps x
+    assert f(A, W_, None, W_ - 64, *ok, None) == 3              # y overlaps w
+    assert f(A, W_, Y_ + 8, Y_, *ok, None) == 3                 # y overlaps bias

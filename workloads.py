@@ -29,6 +29,13 @@ head) takes a = Linear_G1(x_norm) and the Conv1d weights instead of g
   mhf_small_f32 [8, 1024, 768]  fp32  12 heads of 64, K = 3 taps               seed 5
   v, a ~ N(0,1); w, bias ~ U(-1/sqrt(C K), 1/sqrt(C K)) (a default Conv1d's
   initialisation range, fan-in C K), w float32 [D, C, K], bias float32 [D].
+
+The block's causal depthwise convolution (``generate_dwconv``; x, then w,
+then bias):
+
+  dwconv_small_f32 [8, 1024, 768] fp32  K = 3 taps                             seed 6
+  x ~ N(0,1); w, bias ~ U(-1/sqrt(K), 1/sqrt(K)) (a default depthwise Conv1d's
+  range, fan-in K), w float32 [D, K], bias float32 [D].
 """
 from __future__ import annotations
 
@@ -181,3 +188,36 @@ def generate_gate(B: int, L: int, D: int, H: int, K: int, dtype: str, seed: int)
     if dtype == "bf16":
         return bf16_round(v), bf16_round(a), w, bias
     return v, a, w, bias
+
+
+@dataclass(frozen=True)
+class DwconvWorkload:
+    name: str
+    B: int
+    L: int
+    D: int
+    K: int
+    dtype: str
+    seed: int
+    description: str
+
+    @property
+    def units(self) -> int:
+        return self.B * self.L * self.D
+
+
+DWCONV_WORKLOADS = {
+    "dwconv_small_f32": DwconvWorkload("dwconv_small_f32", 8, 1024, 768, 3, "f32", 6,
+                                       "Caracal-Small-shaped causal depthwise conv, kernel size 3"),
+}
+
+
+def generate_dwconv(B: int, L: int, D: int, K: int, dtype: str, seed: int):
+    """(x, w, bias): x [B, L, D] in the I/O type (float32, or bf16 bit
+    patterns as uint16); w float32 [D, K]; bias float32 [D]."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    x = rng.standard_normal((B, L, D)).astype(np.float32)
+    bound = 1.0 / np.sqrt(K)
+    w = rng.uniform(-bound, bound, (D, K)).astype(np.float32)
+    bias = rng.uniform(-bound, bound, D).astype(np.float32)
+    return (bf16_round(x) if dtype == "bf16" else x), w, bias
