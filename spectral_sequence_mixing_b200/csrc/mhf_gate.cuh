@@ -24,15 +24,15 @@
 //
 // Schedule: a persistent CTA per (head, group of tiles); the head's weights
 // are split and staged in shared memory once.  Per 128-step tile the CTA
-// stores sigmoid(a) (hi, lo) to shared memory, one thread issues 3 K C/8
-// MMAs and commits them to an mbarrier, and the sixteen warps read the
-// accumulator back (warp w: TMEM lanes 32 (w % 4) .. +31 = time steps, a
-// quarter of the columns each), add the bias, stage the rows in shared memory
-// and store g as whole rows (coalesced).  With two tile
-// buffers and two accumulators (every head width and tap count whose tiles
-// fit twice) the tensor core works on tile i+1 while the warps drain tile i
-// and stage tile i+2; a for the two tiles after that streams into two
-// register sets meanwhile.  Every wait is bounded; no
+// stores sigmoid(a) (hi, lo) to shared memory, warp 0 runs the loop of
+// 3 K C/8 MMAs (one lane issues them, chosen by elect.sync) and commits them
+// to an mbarrier, and the sixteen warps read the accumulator back (warp w:
+// TMEM lanes 32 (w % 4) .. +31 = time steps, a quarter of the columns each),
+// add the bias, stage the rows in shared memory and store g as whole rows
+// (coalesced).  With two tile buffers and two accumulators (every head width
+// and tap count whose tiles fit twice) the tensor core works on tile i+1
+// while the warps drain tile i and stage tile i+2; a for the two tiles after
+// that streams into two register sets meanwhile.  Every wait is bounded; no
 // load uses cluster multicast.
 #pragma once
 
