@@ -70,8 +70,8 @@ __global__ void __launch_bounds__(kDwThreads) dwconv_vec_kernel(const IO *__rest
         float4 wk[K];
 #pragma unroll
         for (int k = 0; k < K; ++k)
-            wk[k] = make_float4(__ldg(w + (d + 0) * K + k), __ldg(w + (d + 1) * K + k), __ldg(w + (d + 2) * K + k),
-                                __ldg(w + (d + 3) * K + k));
+            wk[k] = make_float4(__ldg(w + (int64_t)(d + 0) * K + k), __ldg(w + (int64_t)(d + 1) * K + k),
+                                __ldg(w + (int64_t)(d + 2) * K + k), __ldg(w + (int64_t)(d + 3) * K + k));
         const float4 bs = bias ? make_float4(__ldg(bias + d), __ldg(bias + d + 1), __ldg(bias + d + 2),
                                              __ldg(bias + d + 3))
                                : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kDwThreads) dwconv_scalar_kernel(const IO *__r
         const int t0 = run * kDwRun;
         float wk[K];
 #pragma unroll
-        for (int k = 0; k < K; ++k) wk[k] = __ldg(w + d * K + k);
+        for (int k = 0; k < K; ++k) wk[k] = __ldg(w + (int64_t)d * K + k);
         const float bs = bias ? __ldg(bias + d) : 0.f;
         const IO *xb = x + b * (int64_t)L * D + d;
         IO *yb = y + b * (int64_t)L * D + d;
