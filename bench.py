@@ -69,6 +69,10 @@ def parse_args():
                          "decode: one autoregressive step at t = L-1 from [B, L, D] caches")
     ap.add_argument("--shape", default=None,
                     help="B,L,D override of the workload's sizes (same recipe); for small profiler captures")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per_config list (the other convolution workloads timed in the same run)")
+    ap.add_argument("--per-config-steps", type=int, default=200,
+                    help="timed steps of each per_config entry (graph-replayed)")
     return ap.parse_args()
 
 
@@ -306,6 +310,123 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def dominant_kernel(w: workloads.Workload, two_pass: bool) -> str:
+    """The kernel that does a forward call's transform on workload `w`."""
+    if w.dtype == "i32":
+        return "ntt_conv_kernel"
+    if w.L <= 1024:
+        return "fftconv_fused_kernel"
+    if w.L <= 4096:
+        return "bigrow_group_kernel"
+    return "bigconv_kernel (two-pass step: 2 transposes in, 1 out)" if two_pass else "bigconv_kernel"
+
+
+def alu_roofline(alu_ops, alu_pipe, ms_per_step, clocks):
+    """Executed lane operations of the kernel's busiest ALU pipe (ncu, same
+    sources) per launch against 148 SMs x lanes/clk of that pipe (FP32 128,
+    IMAD 64) x the SM clock sampled during the run."""
+    lanes = {"fp32": 128, "imad": 64}[alu_pipe]
+    sm_hz = clocks["sm_mhz"] * 1e6 if clocks and clocks.get("sm_mhz") else 1.965e9
+    peak = 148 * lanes * sm_hz / 1e9
+    achieved = alu_ops / (ms_per_step * 1e-3) / 1e9
+    return {"bound": "alu", "pipe": alu_pipe, "achieved": achieved, "peak": peak,
+            "unit": f"G {alu_pipe.upper()} lane-op/s", "frac": achieved / peak, "lane_ops_per_launch": alu_ops,
+            "peak_source": f"148 SMs x {lanes} lanes/clk x sampled SM clock"}
+
+
+def time_config(w: workloads.Workload, rank, world, dev, pg, steps: int, warmup: int, cpu_budget_s: float):
+    """One forward workload timed in this run: rotating buffer sets larger than
+    L2 (cold L2), the steps replayed from CUDA graphs (a step is one library
+    call, 1 or 4 launches), CUDA events on the replay stream, max over ranks;
+    plus the same steps on one set (hot L2) and a short oracle sample."""
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    v_np, g_np = workloads.generate(w, seed=rank_seed(w, rank))
+    if w.dtype == "bf16":
+        hv = torch.from_numpy(v_np.view(np.int16)).view(torch.bfloat16)
+        hg = torch.from_numpy(g_np.view(np.int16)).view(torch.bfloat16)
+    else:
+        hv, hg = torch.from_numpy(v_np), torch.from_numpy(g_np)
+    v0, g0 = hv.to(dev), hg.to(dev)
+    set_bytes = 3 * w.units * w.elem_bytes
+    n_sets = max(2, math.ceil(2.2 * L2_BYTES / set_bytes))
+    sets = [(v0, g0, torch.empty_like(v0))] + [(v0.clone(), g0.clone(), torch.empty_like(v0))
+                                                for _ in range(n_sets - 1)]
+    n_ws = ssm.fast_workspace_bytes(v0.dtype, w.B, w.L, w.D)
+    ws = torch.empty(n_ws, dtype=torch.uint8, device=dev)
+    side = torch.cuda.Stream(dev)
+
+    def step(i):
+        a, b, c = sets[i % n_sets]
+        ssm.causal_conv(a, b, out=c, workspace=ws)  # on the current (capture) stream
+
+    G = n_sets * max(1, 32 // n_sets)
+    with torch.cuda.stream(side):
+        for i in range(max(3, warmup)):
+            step(i)
+        side.synchronize()
+        cold = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cold, stream=side):
+            for i in range(G):
+                step(i)
+        hot = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(hot, stream=side):
+            for i in range(G):
+                step(0)
+    torch.cuda.synchronize(dev)
+    reps = max(1, math.ceil(steps / G))
+
+    def timed(graph):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(side):
+            graph.replay()  # warm replay
+            if pg is not None:
+                pg.barrier()
+            torch.cuda.synchronize(dev)
+            e0.record(side)
+            for _ in range(reps):
+                graph.replay()
+            e1.record(side)
+            torch.cuda.synchronize(dev)
+            if pg is not None:
+                pg.barrier()
+        return max_over_ranks(e0.elapsed_time(e1), pg, dev) / (reps * G)
+
+    with ClockSampler(dev.index) as clk:
+        ms = timed(cold)
+    ms_hot = timed(hot)
+    clocks = clk.report()
+    del cold, hot
+    alg = w.algorithmic_bytes
+    peak, peak_src = measured_peaks()
+    kernel = dominant_kernel(w, n_ws > 0)
+    achieved = alg / (ms * 1e-3) / 1e9
+    traffic, alu_ops, alu_pipe = recorded_counters(w.name, kernel)
+    entry = {
+        "workload": w.name, "B": w.B, "L": w.L, "D": w.D, "io_dtype": w.dtype,
+        "transform_len": 2 ** math.ceil(math.log2(2 * w.L)),
+        "ms_per_step": ms, "steps": reps * G, "value": achieved * world, "unit": "GB/s",
+        "outputs_per_s": w.units * world / (ms * 1e-3),
+        "launch": f"CUDA graph replay of {G} steps ({4 if n_ws else 1} launches per step)",
+        "l2": f"cold: {n_sets} rotating (v,g,r) sets of {set_bytes / 2 ** 20:.1f} MiB",
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)", "kernel": kernel,
+                     "algorithmic_bytes_per_launch": alg, "traffic": traffic},
+        "hot_l2": {"ms_per_step": ms_hot, "GB/s": alg / (ms_hot * 1e-3) / 1e9,
+                   "note": "the same steps on one (v,g,r) set"},
+        "clocks": clocks,
+    }
+    if alu_ops:
+        entry["alu_roofline"] = alu_roofline(alu_ops, alu_pipe, ms, clocks)
+    if rank == 0 and world == 1 and cpu_budget_s > 0:
+        cpu_ups, cores, desc, secs = cpu_oracle_rate(w, v_np, g_np, budget_s=cpu_budget_s)
+        entry["cpu_baseline"] = {"value": cpu_ups * 3 * w.elem_bytes / 1e9, "unit": "GB/s", "cores": cores,
+                                 "kind": "oracle", "sample": desc, "seconds": secs}
+    del sets, ws, v0, g0
+    torch.cuda.empty_cache()
+    return entry
+
+
 def run_ours(args, rank, world, local):
     import torch
     import spectral_sequence_mixing_b200 as ssm
@@ -409,18 +530,7 @@ def run_ours(args, rank, world, local):
     _, e2e_gbs = throughput(w.units, world, e2e_steps, ems, 3 * w.elem_bytes)
 
     peak, peak_src = measured_peaks()
-    if w.dtype == "i32":
-        kernel = "ntt_conv_kernel"
-    elif w.L <= 1024:
-        kernel = "fftconv_fused_kernel"
-    elif w.L <= 4096:
-        kernel = "bigrow_group_kernel"
-    else:
-        kernel = "bigconv_kernel"
-    if args.path == "decode":
-        kernel = "decode_partial_kernel"
-    if n_ws and args.path != "decode":
-        kernel = "bigconv_kernel (two-pass step: 2 transposes in, 1 out)"
+    kernel = "decode_partial_kernel" if args.path == "decode" else dominant_kernel(w, n_ws > 0)
     per_launch_bytes = bytes_per_step // 2 if args.path == "bwd" else bytes_per_step
     achieved = bytes_per_step / (ms_per_step * 1e-3) / 1e9
     traffic, alu_ops, alu_pipe = ((None, None, None) if (args.shape or args.path != "fwd")
@@ -446,18 +556,8 @@ def run_ours(args, rank, world, local):
         "clocks": clocks,
     }
     if alu_ops and launches_per_step == 1:
-        # the transform kernels are bound by ALU issue, not by HBM: executed
-        # lane operations of their busiest pipe (ncu, same sources) per launch
-        # against 148 SMs x lanes/clk of that pipe (FP32 128, IMAD 64) x the
-        # SM clock sampled during the run
-        lanes = {"fp32": 128, "imad": 64}[alu_pipe]
-        sm_hz = clocks["sm_mhz"] * 1e6 if clocks and clocks.get("sm_mhz") else 1.965e9
-        alu_peak = 148 * lanes * sm_hz / 1e9
-        alu_achieved = alu_ops / (ms_per_step * 1e-3) / 1e9
-        line["alu_roofline"] = {"bound": "alu", "pipe": alu_pipe, "achieved": alu_achieved, "peak": alu_peak,
-                                "unit": f"G {alu_pipe.upper()} lane-op/s", "frac": alu_achieved / alu_peak,
-                                "lane_ops_per_launch": alu_ops,
-                                "peak_source": f"148 SMs x {lanes} lanes/clk x sampled SM clock"}
+        # the transform kernels are bound by ALU issue, not by HBM
+        line["alu_roofline"] = alu_roofline(alu_ops, alu_pipe, ms_per_step, clocks)
     if args.path != "fwd":  # the host-buffer leg and CPU baseline describe the forward line only
         line.pop("e2e")
         args.no_cpu_baseline = True
@@ -465,6 +565,16 @@ def run_ours(args, rank, world, local):
         cpu_ups, cores, desc, secs = cpu_oracle_rate(w, v_np, g_np, budget_s=15.0)
         line["cpu_baseline"] = {"value": cpu_ups * 3 * w.elem_bytes / 1e9, "unit": "GB/s", "cores": cores,
                                 "kind": "oracle", "sample": desc, "seconds": secs}
+    if args.path == "fwd" and not args.shape and not args.no_per_config:
+        # every convolution workload on the same clock: the line's own
+        # workload again (hot and cold L2, graph-replayed), then the others
+        del sets, ws
+        torch.cuda.empty_cache()
+        order = [w.name] + [n for n in workloads.WORKLOADS if n != w.name]
+        line["per_config"] = [
+            time_config(workloads.WORKLOADS[n], rank, world, dev, pg, args.per_config_steps, args.warmup,
+                        0.0 if n == w.name or args.no_cpu_baseline else 2.5)
+            for n in order]
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg is not None:

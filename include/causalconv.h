@@ -178,8 +178,16 @@ CC_API int causal_conv_decode_bf16(const uint16_t *v, const uint16_t *g, uint16_
  * fp64 partial sums go to one static device buffer of 8 MiB inside the
  * library, which every GPU that loads the library holds until the process
  * exits.  The first call on a device looks the buffer's address up (once,
- * with that device current); make that first call before any stream capture.
+ * with that device current; again after a cudaDeviceReset replaced the
+ * device's context); make that first call before any stream capture.
  * The function calls no cudaMalloc, cudaFree or other allocating routine.
+ * Under CUDA's lazy module loading (the default since CUDA 12) the first call
+ * into this library on a device -- any entry point -- loads the library's
+ * device code there, and that load reserves all its static device memory at
+ * once: this 8 MiB buffer plus under 1 MiB of transform tables.  A caller
+ * whose memory pool must see no reservation later should make one warm-up
+ * call (of this or any entry point) before it hands memory control to the
+ * pool; after that, calls reserve nothing.
  *
  * Limit: a problem whose partial sums need more than 8 MiB, i.e. for which
  * causal_conv_decode_workspace_bytes(CC_DTYPE_F32, B, D, t) > 8388608 (the

@@ -97,6 +97,36 @@ static cudaError_t set_big_attr() {
 
 static std::mutex g_init_mu;
 static bool g_init_done[128];
+// Context the per-device state was built in (0: none yet).
+static unsigned long long g_init_ctx[128];
+
+// Identifier of the calling thread's current CUDA context (cuCtxGetId through
+// the runtime's driver entry points; 0 when there is none or it cannot be
+// read).  Per-device state -- the tables' contents, kernel attributes, the
+// no-allocation scratch address -- belongs to one context; a cudaDeviceReset
+// destroys it, so the state is rebuilt when the identifier changes.
+static unsigned long long current_ctx_id() {
+    typedef CUresult (*CtxGetCurrent)(CUcontext *);
+    typedef CUresult (*CtxGetId)(CUcontext, unsigned long long *);
+    static CtxGetCurrent get_cur = nullptr;
+    static CtxGetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_cur = reinterpret_cast<CtxGetCurrent>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetId>(p);
+        cudaGetLastError();
+    });
+    CUcontext c = nullptr;
+    unsigned long long id = 0;
+    if (!get_cur || !get_id || get_cur(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 
 // Per device: SM count and, per kernel instantiation, resident CTAs per SM.
@@ -117,7 +147,8 @@ static cudaError_t set_smem_attr() {
 static cudaError_t ensure_init(int dev) {
     if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lk(g_init_mu);
-    if (g_init_done[dev]) return cudaSuccess;
+    if (g_init_done[dev] && g_init_ctx[dev] == current_ctx_id()) return cudaSuccess;
+    g_init_done[dev] = false;
     cudaError_t e;
     float2 w128[128];
     for (int k = 0; k < 128; ++k) w128[k] = omega(k, 128);
@@ -168,6 +199,7 @@ static cudaError_t ensure_init(int dev) {
     if ((e = cudaGetSymbolAddress(&g_tw_addr[dev][2], g_tw_bl)) != cudaSuccess) return e;
     if ((e = cudaGetSymbolAddress(&g_tw_addr[dev][3], g_tw_bx)) != cudaSuccess) return e;
     if ((e = cudaGetSymbolAddress(&g_tw_addr[dev][4], g_tw_bm)) != cudaSuccess) return e;
+    g_init_ctx[dev] = current_ctx_id();
     g_init_done[dev] = true;
     return cudaSuccess;
 }
@@ -503,20 +535,24 @@ static __device__ __align__(256) double g_noalloc_scratch[kNoAllocScratchBytes /
 
 // Device address of g_noalloc_scratch per device.  In host code the symbol
 // only names a host-side stand-in, so the address is looked up with the
-// device current on first use and cached.
+// device current on first use and cached together with the context it
+// belongs to (looked up again if a device reset replaced that context).
 static std::mutex g_noalloc_mu;
 static double *g_noalloc_ptr[128];
+static unsigned long long g_noalloc_ctx[128];
 
 static int noalloc_scratch(int dev, double **out) {
     if (dev < 0 || dev >= 128) return CC_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    const unsigned long long ctx = current_ctx_id();
+    if (!g_noalloc_ptr[dev] || ctx == 0 || g_noalloc_ctx[dev] != ctx) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
             cudaGetLastError();
             return CC_ERR_CUDA;
         }
         g_noalloc_ptr[dev] = (double *)p;
+        g_noalloc_ctx[dev] = ctx;
     }
     *out = g_noalloc_ptr[dev];
     return CC_OK;
@@ -597,12 +633,14 @@ template <int C, int KT, typename IO>
 static int launch_gate_ck(const IO *a, const float *w, const float *bias, IO *g, int64_t B, int64_t L, int64_t D,
                           int64_t H, cudaStream_t s, int dev) {
     using Cfg = GateCfg<C, KT>;
-    static std::atomic<bool> attr_set[128];
-    if (!attr_set[dev].load(std::memory_order_acquire)) {
+    // the attribute belongs to the context it was set in (see current_ctx_id)
+    static std::atomic<unsigned long long> attr_ctx[128];
+    const unsigned long long ctx = current_ctx_id();
+    if (ctx == 0 || attr_ctx[dev].load(std::memory_order_acquire) != ctx) {
         if (cudaFuncSetAttribute(mhf_gate_kernel<C, KT, IO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)Cfg::SMEM_BYTES) != cudaSuccess)
             return CC_ERR_CUDA;
-        attr_set[dev].store(true, std::memory_order_release);
+        attr_ctx[dev].store(ctx, std::memory_order_release);
     }
     const int64_t per_row = (L + kGateM - 1) / kGateM;
     const int64_t tiles = B * per_row;  // tiles of one head
