@@ -44,6 +44,7 @@ KERNEL_SOURCES = {
     "bigrow_group_kernel": ["bigconv.cuh", "configs_rows.cuh"] + _FUSED_SOURCES,
     "bigconv_kernel": ["bigconv.cuh", "configs_rows.cuh", "transpose.cuh"] + _FUSED_SOURCES,
     "ntt_conv_kernel": ["ntt.cuh"],
+    "tcconv_kernel": ["tcconv.cuh", "tcgen05.cuh", "tma.cuh"],
     "mhf_gate_kernel": ["mhf_gate.cuh", "tcgen05.cuh", "tma.cuh"],
     "dwconv_vec_kernel": ["dwconv.cuh"],
 }
@@ -316,8 +317,10 @@ def dominant_kernel(w: workloads.Workload, two_pass: bool) -> str:
         return "ntt_conv_kernel"
     if w.L <= 1024:
         return "fftconv_fused_kernel"
-    if w.L <= 4096:
+    if w.L <= 2048:
         return "bigrow_group_kernel"
+    if w.L <= 4096:
+        return "tcconv_kernel" if w.dtype == "bf16" else "bigrow_group_kernel"
     return "bigconv_kernel (two-pass step: 2 transposes in, 1 out)" if two_pass else "bigconv_kernel"
 
 
@@ -493,17 +496,47 @@ def run_ours(args, rank, world, local):
         fn(a, b, out=c, stream=stream)
     torch.cuda.synchronize(dev)
 
+    # The timed steps are replayed from CUDA graphs of the same library calls
+    # (one graph of G consecutive steps, whole rotations of the buffer sets,
+    # and one graph per set for the remainder), so exactly K steps run with
+    # no host launch gaps between them.
+    side = torch.cuda.Stream(dev)
+    G = n_sets * max(1, 32 // n_sets)
+    with torch.cuda.stream(side):
+        big = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(big, stream=side):
+            for i in range(G):
+                a, b, c = sets[i % n_sets]
+                fn(a, b, out=c, stream=side)
+        singles = []
+        for k in range(n_sets):
+            gk = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gk, stream=side):
+                a, b, c = sets[k]
+                fn(a, b, out=c, stream=side)
+            singles.append(gk)
+    torch.cuda.synchronize(dev)
+
+    def run_steps(n):
+        for _ in range(n // G):
+            big.replay()
+        for i in range(n % G):
+            singles[i % n_sets].replay()
+
+    with torch.cuda.stream(side):
+        run_steps(min(G, max(1, args.warmup)))
+    torch.cuda.synchronize(dev)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier()
         torch.cuda.synchronize(dev)
-        start.record(stream)
-        for i in range(args.steps):
-            a, b, c = sets[i % n_sets]
-            fn(a, b, out=c, stream=stream)
-        end.record(stream)
+        with torch.cuda.stream(side):
+            start.record(side)
+            run_steps(args.steps)
+            end.record(side)
         torch.cuda.synchronize(dev)
         barrier()
+    del big, singles
     ms = max_over_ranks(start.elapsed_time(end), pg, dev)
     ms_per_step = ms / args.steps
     units_step = w.units if args.path != "decode" else w.B * w.D
@@ -543,6 +576,7 @@ def run_ours(args, rank, world, local):
         "config": {"workload": w.name, "path": args.path, "B": w.B, "L": w.L, "D": w.D, "io_dtype": w.dtype,
                    "transform_len": 2 ** math.ceil(math.log2(2 * w.L)),
                    "l2": f"inputs larger than L2: {n_sets} rotating (v,g,r) sets of {set_bytes / 2 ** 20:.0f} MiB",
+                   "launch": f"timed steps replayed from CUDA graphs ({G} steps per graph)",
                    "parallelism": f"dp{world} (independent batches, no collective)"},
         "outputs_per_s": ups,
         "hbm_frac": gbs / world / peak,

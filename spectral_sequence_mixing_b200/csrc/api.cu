@@ -25,6 +25,7 @@
 #include "transpose.cuh"
 #include "mhf_gate.cuh"
 #include "dwconv.cuh"
+#include "tcconv.cuh"
 #include "configs.cuh"
 
 namespace ccv {
@@ -82,6 +83,66 @@ static std::vector<float2> big_twiddles() {
     }
     for (int k = 0; k < RB; ++k)
         for (int lo = 0; lo < RC; ++lo) t[Cfg::TB + k * RC + lo] = omega((int64_t)lo * k, RB * RC);
+    return t;
+}
+
+// ---- tensor-core transform (tcconv.cuh): stage matrices and twiddle pairs
+static uint16_t h_half(double x) { return __half_as_ushort(__float2half_rn((float)x)); }
+
+// byte offset of fp16 element (row, k) in a K-major no-swizzle operand of 128 rows
+static size_t tc_kmajor(int row, int k) { return (size_t)(k / 8) * kTcChunkPitch + (size_t)row * 16 + (size_t)(k % 8) * 2; }
+
+static std::vector<uint16_t> tc_const_table() {
+    // A1 (F1 / 4, rows = lanes (k1, re/im), K = 2 n1 + re/im), B2 (F64 / 8,
+    // rows 2 q + re/im, K = 2 m + re/im), A4 (conj F1 / 4, real part only:
+    // rows n1 < 32, K = 2 k1 + re/im), each in its shared-memory layout; then
+    // the twiddle table F0[k1][m] = theta^(m (2 k1 + 1)) / 2, w[m] = omega_128^m
+    // and c64[k1] = theta^(64 (2 k1 + 1)) as float2 (theta = omega_2N)
+    std::vector<uint16_t> t(kTcConstBytes / 2, 0);
+    auto put = [&](unsigned off, int row, int k, double x) { t[(off + tc_kmajor(row, k)) / 2] = h_half(x); };
+    auto putf2 = [&](unsigned off, int i, double re, double im) {
+        const float f[2] = {(float)re, (float)im};
+        memcpy(&t[(off + 8u * (unsigned)i) / 2], f, 8);
+    };
+    const double pi = kTwoPi / 2;
+    for (int l = 0; l < 128; ++l) {
+        const int k1 = tc_kappa(l);
+        for (int n1 = 0; n1 < 32; ++n1) {
+            const double a = -pi * n1 * (2 * k1 + 1) / 64.0, fr = 0.25 * cos(a), fi = 0.25 * sin(a);
+            if ((l & 1) == 0) {
+                put(kTcOffA1, l, 2 * n1, fr);
+                put(kTcOffA1, l, 2 * n1 + 1, -fi);
+            } else {
+                put(kTcOffA1, l, 2 * n1, fi);
+                put(kTcOffA1, l, 2 * n1 + 1, fr);
+            }
+        }
+    }
+    for (int q = 0; q < 64; ++q)
+        for (int m = 0; m < 64; ++m) {
+            const double a = -kTwoPi * (double)((m * q) % 64) / 64.0, fr = 0.125 * cos(a), fi = 0.125 * sin(a);
+            put(kTcOffB2, 2 * q, 2 * m, fr);
+            put(kTcOffB2, 2 * q, 2 * m + 1, -fi);
+            put(kTcOffB2, 2 * q + 1, 2 * m, fi);
+            put(kTcOffB2, 2 * q + 1, 2 * m + 1, fr);
+        }
+    for (int n1 = 0; n1 < 32; ++n1)
+        for (int k1 = 0; k1 < 64; ++k1) {
+            const double a = pi * n1 * (2 * k1 + 1) / 64.0, gr = 0.25 * cos(a), gi = 0.25 * sin(a);
+            put(kTcOffA4, n1, 2 * k1, gr);
+            put(kTcOffA4, n1, 2 * k1 + 1, -gi);
+        }
+    const int64_t N2 = 2 * (int64_t)kTcN;  // theta = omega_2N
+    auto ang = [&](int64_t e) { return -kTwoPi * (double)(e % N2) / (double)N2; };
+    for (int k1 = 0; k1 < 64; ++k1) {
+        for (int m = 0; m < 64; ++m) {
+            const double a = ang((int64_t)m * (2 * k1 + 1));
+            putf2(kTcOffTw, k1 * kTcTwPitch + m, 0.5 * cos(a), 0.5 * sin(a));
+        }
+        const double a = ang((int64_t)64 * (2 * k1 + 1));
+        putf2(kTcOffW, 64 + k1, cos(a), sin(a));
+    }
+    for (int m = 0; m < 64; ++m) putf2(kTcOffW, m, cos(kTwoPi * m / 128.0), -sin(kTwoPi * m / 128.0));
     return t;
 }
 
@@ -189,6 +250,13 @@ static cudaError_t ensure_init(int dev) {
     if ((e = set_big_attr<BigX<float>, float, kMinbBigX>()) != cudaSuccess) return e;
     if ((e = set_big_attr<BigX<__nv_bfloat16>, __nv_bfloat16, kMinbBigX>()) != cudaSuccess) return e;
     if ((e = ntt_init_device()) != cudaSuccess) return e;
+    {
+        auto t = tc_const_table();
+        if ((e = cudaMemcpyToSymbol(g_tc_consts, t.data(), t.size() * sizeof(uint16_t))) != cudaSuccess) return e;
+        if ((e = cudaFuncSetAttribute(tcconv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kTcSmemBytes)) != cudaSuccess)
+            return e;
+    }
     if ((e = set_smem_attr<CfgS<float>, float, kMinbS>()) != cudaSuccess) return e;
     if ((e = set_smem_attr<CfgS<__nv_bfloat16>, __nv_bfloat16, kMinbS>()) != cudaSuccess) return e;
     if ((e = set_smem_attr<CfgM<float>, float, kMinbM>()) != cudaSuccess) return e;
@@ -445,6 +513,40 @@ static int launch_group(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, i
     return CC_OK;
 }
 
+// bf16 rows with 2048 < L <= 4096 on the tensor cores: clusters of 4 CTAs
+// (8 adjacent channels, two per CTA), persistent over the channel groups.
+static int launch_tcconv(const __nv_bfloat16 *v, const __nv_bfloat16 *g, __nv_bfloat16 *r, int64_t B, int64_t L,
+                         int64_t D, cudaStream_t s, int dev, int rev) {
+    const int64_t gpb = (D + kTcGroup - 1) / kTcGroup;
+    const int64_t groups = B * gpb;
+    if (groups > INT32_MAX / kTcCluster) return CC_ERR_UNSUPPORTED;
+    static std::atomic<int> max_clusters[128];
+    int mc = max_clusters[dev].load(std::memory_order_relaxed);
+    if (mc == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(kTcCluster * 64);
+        cfg.blockDim = dim3(kTcThreads);
+        cfg.dynamicSmemBytes = kTcSmemBytes;
+        if (cudaOccupancyMaxActiveClusters(&mc, tcconv_kernel, &cfg) != cudaSuccess || mc < 1) {
+            cudaGetLastError();
+            return CC_ERR_CUDA;
+        }
+        max_clusters[dev].store(mc, std::memory_order_relaxed);
+    }
+    const int64_t clusters = std::min<int64_t>(groups, mc);
+    const bool vec = (D * 2) % 16 == 0 && ((uintptr_t)v % 16) == 0 && ((uintptr_t)g % 16) == 0 &&
+                     ((uintptr_t)r % 16) == 0;
+    // inputs staged by TMA boxes [256 t][8 d] when the layout allows a tensor map
+    CUtensorMap tmv, tmg;
+    memset(&tmv, 0, sizeof(tmv));
+    memset(&tmg, 0, sizeof(tmg));
+    const bool tma = encode_btd_map<__nv_bfloat16>(&tmv, v, B, L, D, kTcGroup, kTcBoxT) &&
+                     encode_btd_map<__nv_bfloat16>(&tmg, g, B, L, D, kTcGroup, kTcBoxT);
+    tcconv_kernel<<<(unsigned)(clusters * kTcCluster), kTcThreads, kTcSmemBytes, s>>>(
+        v, g, r, (int)L, (int)D, (int)gpb, (int)groups, rev, vec ? 1 : 0, tmv, tmg, tma ? 1 : 0);
+    return cudaGetLastError() == cudaSuccess ? CC_OK : CC_ERR_CUDA;
+}
+
 template <typename IO>
 static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, void *ws,
                             size_t ws_bytes, cudaStream_t s, int dev, int rev = 0) {
@@ -455,8 +557,12 @@ static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t 
         return launch_fused<CfgM<IO>, kMinbM>(v, g, r, B, L, D, (const float2 *)tws[1], s, dev, rev);
     if (L <= BigM<IO>::LMAX)
         return launch_group<BigM<IO>, kMinbBigM>(v, g, r, B, L, D, (const float2 *)tws[4], s, rev);
-    if (L <= BigL<IO>::LMAX)
+    if (L <= BigL<IO>::LMAX) {
+        if constexpr (sizeof(IO) == 2)
+            return launch_tcconv((const __nv_bfloat16 *)v, (const __nv_bfloat16 *)g, (__nv_bfloat16 *)r, B, L, D, s,
+                                 dev, rev);
         return launch_group<BigL<IO>, kMinbBigL>(v, g, r, B, L, D, (const float2 *)tws[2], s, rev);
+    }
     if (L <= BigX<IO>::LMAX) {
         const void *tw = tws[3];
         const size_t fast = fast_ws_bytes(sizeof(IO) == 4 ? CC_DTYPE_F32 : CC_DTYPE_BF16, B, L, D);

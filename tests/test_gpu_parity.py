@@ -522,3 +522,33 @@ def test_partitioned_call_equals_whole_call(case):
         got = as_f32(b, dtype)[pts[:, 0], pts[:, 1], pts[:, 2]]
         n_bad, worst = float_violations(got, ref, den, F32_TOL if dtype == "f32" else BF16_TOL)
         assert n_bad == 0, f"{n_bad} sampled outputs beyond the bound, worst ratio {worst:.3g}"
+
+
+# bf16 rows with 2048 < L <= 4096 run on the tensor cores (clusters of 8 channels):
+# whole groups, ragged last groups (D not a multiple of 8), single channels,
+# and bases that are not 16-byte aligned (element-wise group accesses)
+TC_SHAPES = [(2, 2049, 8), (1, 3000, 13), (1, 4096, 24), (3, 2500, 1), (1, 4095, 40)]
+
+
+@pytest.mark.parametrize("shape", TC_SHAPES, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("offset", [0, 1])
+def test_tensor_core_rows_bf16(shape, offset):
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    B, L, D = shape
+    v, g = _rand_float(shape, seed=300 + L + D, scale_g=0.125)
+    vb, gb = workloads.bf16_round(v), workloads.bf16_round(g)
+    n = B * L * D
+
+    def place(x):  # a bf16 tensor starting `offset` elements into its allocation
+        buf = torch.zeros(n + offset, dtype=torch.bfloat16, device="cuda")
+        buf[offset:] = to_dev(x, "bf16").reshape(-1)
+        return buf[offset:].view(B, L, D)
+
+    out = torch.empty(n + offset, dtype=torch.bfloat16, device="cuda")[offset:].view(B, L, D)
+    ssm.causal_fftconv_bf16(place(vb), place(gb), out=out)
+    torch.cuda.synchronize()
+    r = as_f32(from_dev(out, "bf16"), "bf16")
+    r_ref, den = oracle.causal_conv(as_f32(vb, "bf16"), as_f32(gb, "bf16"))
+    n_bad, worst = float_violations(r, r_ref, den, BF16_TOL)
+    assert n_bad == 0, f"{n_bad} elements beyond the bf16 bound, worst ratio {worst:.3g}"
