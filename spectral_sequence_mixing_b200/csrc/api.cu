@@ -766,8 +766,13 @@ static int launch_gate_ck(const IO *a, const float *w, const float *bias, IO *g,
     if (grid > INT32_MAX) return CC_ERR_UNSUPPORTED;
     const int vec_in = ((uintptr_t)a % (sizeof(IO) == 4 ? 16 : 8)) == 0;
     const int vec_out = ((uintptr_t)g % 16) == 0;
+    // fp32 input tiles [ROWS t][C ch] staged by TMA when the layout allows a tensor map
+    CUtensorMap tma_a;
+    memset(&tma_a, 0, sizeof(tma_a));
+    const bool tma = sizeof(IO) == 4 && encode_btd_map<IO>(&tma_a, a, B, L, D, C, Cfg::ROWS);
     mhf_gate_kernel<C, KT, IO><<<(unsigned)grid, kGateThreads, Cfg::SMEM_BYTES, s>>>(
-        a, w, bias, g, (int)L, (int)D, (int)H, (int)groups, (int)per_row, (int)tiles, vec_in, vec_out);
+        a, w, bias, g, (int)L, (int)D, (int)H, (int)groups, (int)per_row, (int)tiles, vec_in, vec_out, tma_a,
+        tma ? 1 : 0);
     return cudaGetLastError() == cudaSuccess ? CC_OK : CC_ERR_CUDA;
 }
 

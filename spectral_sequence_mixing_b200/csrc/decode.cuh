@@ -14,7 +14,9 @@
 // over j into `splits` ranges so the whole GPU streams the caches: kernel 1
 // (each thread four adjacent channels, one 16-byte fp32 or 8-byte bf16
 // access per cache row) writes fp64 partial sums part[split][b][d] (caller's
-// workspace), kernel 2 adds them in a fixed order and rounds once.  Accumulating in fp64 keeps the
+// workspace), kernel 2 adds them in a fixed order and rounds once (launched
+// as a programmatic dependent of kernel 1, so its launch latency overlaps
+// kernel 1's tail).  Accumulating in fp64 keeps the
 // result within one fp32 rounding of the exact sum and makes it
 // deterministic.
 #pragma once
@@ -101,11 +103,17 @@ __global__ void __launch_bounds__(kDecodeThreads)
 #pragma unroll
     for (int q = 0; q < kDecodeVec; ++q)
         if (d0 + q < D) pp[q] = acc[q];
+    // the reduction kernel may be scheduled now; it waits for this grid's
+    // completion (griddepcontrol.wait) before it reads the partial sums
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 template <typename IO>
 __global__ void __launch_bounds__(kReduceThreads)
     decode_reduce_kernel(const double *__restrict__ part, IO *__restrict__ r, int64_t BD, int splits) {
+    // launched as a programmatic dependent of the partial kernel: wait until
+    // that grid has completed and its partial sums are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int64_t i = (int64_t)blockIdx.x * kReduceThreads + threadIdx.x;
     if (i >= BD) return;
     double s = 0.0;
@@ -126,9 +134,22 @@ static int decode_launch(const IO *v, const IO *g, IO *r, int64_t B, int64_t Lca
                                                               vec);
     if (cudaGetLastError() != cudaSuccess) return 5;  // CC_ERR_CUDA
     const int64_t BD = B * D;
-    decode_reduce_kernel<IO><<<(unsigned)((BD + kReduceThreads - 1) / kReduceThreads), kReduceThreads, 0, s>>>(
-        part, r, BD, splits);
-    return cudaGetLastError() == cudaSuccess ? 0 : 5;
+    // programmatic dependent launch: the reduction's launch overlaps the
+    // partial kernel's tail instead of waiting for it on the stream
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((BD + kReduceThreads - 1) / kReduceThreads));
+    cfg.blockDim = dim3(kReduceThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, decode_reduce_kernel<IO>, (const double *)part, r, BD, splits) != cudaSuccess) {
+        cudaGetLastError();
+        return 5;
+    }
+    return 0;
 }
 
 }  // namespace ccv

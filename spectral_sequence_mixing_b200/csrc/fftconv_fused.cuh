@@ -238,10 +238,6 @@ __device__ __forceinline__ float2 shfl_xor2(float2 a, int m) {
     return make_float2(__shfl_xor_sync(0xffffffffu, a.x, m), __shfl_xor_sync(0xffffffffu, a.y, m));
 }
 
-// Named barrier over `count` threads (a multiple of 32), id 1..15.
-__device__ __forceinline__ void bar_sync(int id, int count) {
-    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
-}
 
 template <int N2, int ROWS, int MINB, typename IO, bool REVA>
 __global__ void __launch_bounds__(ROWS * 2 * N2, MINB)

@@ -16,27 +16,30 @@
 // operand is the same tile started k rows later (16 bytes in the K-major
 // no-swizzle layout).
 //
-// fp32 accuracy from tf32 tensor cores: every operand x is split into
-// hi = x with its 13 low mantissa bits cleared (exact in tf32) and
-// lo = x - hi (exact in fp32, |lo| <= 2^-10 |x|), and the product is
-// hi*W_hi + hi*W_lo + lo*W_hi.  The dropped lo*W_lo term and the tf32 view of
-// the lo parts are below 2^-20 of |x W|, so g carries fp32-level error.
+// fp32 accuracy from fp16 tensor cores (kind::f16, fp32 accumulation):
+// every operand x is split into hi = fp16(x) and lo = fp16(x - hi), and the
+// product is hi*W_hi + hi*W_lo + lo*W_hi.  The dropped lo*W_lo term and the
+// rounding of the lo parts are below 2^-21 of |x W| (sigmoid values lie in
+// (0, 1) and the weights near 1/sqrt(C K), well inside fp16's range), so g
+// carries fp32-level error.  fp16 operands take half the shared-memory bytes
+// of tf32 per multiply-add: at M = 128, N = 64 the tensor core's operand
+// reads are what bound it, so this halves the MMA time of a tile.
 //
 // Schedule: a persistent CTA per (head, group of tiles); the head's weights
-// are split and staged in shared memory once.  Per 128-step tile the CTA
-// stores sigmoid(a) (hi, lo) to shared memory, warp 0 runs the loop of
-// 3 K C/8 MMAs (one lane issues them, chosen by elect.sync) and commits them
-// to an mbarrier, and the sixteen warps read the accumulator back (warp w:
-// TMEM lanes 32 (w % 4) .. +31 = time steps, a quarter of the columns each),
-// add the bias, stage the rows in shared memory and store g as whole rows
-// (coalesced).  With two tile buffers and two accumulators (every head width
-// and tap count whose tiles fit twice) the tensor core works on tile i+1
-// while the warps drain tile i and stage tile i+2; a for the two tiles after
-// that streams into two register sets meanwhile.  Every wait is bounded; no
-// load uses cluster multicast.
+// are split and staged in shared memory once.  Then the warps take roles:
+// eight producer warps store sigmoid(a) (hi, lo) of 128-step tiles into a
+// ring of tile buffers, one warp issues each tile's 3 K C/8 MMAs (one lane,
+// elect.sync) into a ring of TMEM accumulators, and four warps read each
+// accumulator back (warp w: TMEM lanes 32 w .. +31 = time steps, all C
+// columns), add the bias and store g.  Buffers and accumulators pass between
+// the roles on mbarriers (tcgen05.commit frees a tile buffer and publishes
+// its accumulator), so the tensor core, the sigmoid and the stores of
+// different tiles overlap with no CTA-wide barrier.  Every wait is bounded;
+// no load uses cluster multicast.
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "tcgen05.cuh"
@@ -54,39 +57,56 @@ struct GateCfg {
     static_assert(C == 16 || C == 32 || C == 64, "head width");
     static_assert(KT >= 1 && KT <= kGateMaxTaps, "taps");
     static constexpr int ROWS = kGateM + KT - 1;          // staged time steps
-    static constexpr int KC = C / 4;                       // 16-byte chunks along the contraction axis
-    // Two sigmoid tiles (one being staged while the tensor core reads the
-    // other) when they fit next to the weights; an odd row count keeps the
-    // 16-byte stores conflict-free, an even one (2-way conflicts) is taken
-    // when only that fits.
-    static constexpr unsigned kMaxSmem = 232448;
-    static constexpr unsigned FIXED = 2u * KT * C * C * 4u + C * 4u + 48u + 128u;
-    static constexpr bool DB_ODD = 4u * KC * (ROWS | 1) * 16u + FIXED <= kMaxSmem;
-    static constexpr bool DB_EVEN = (ROWS % 2 == 0) && 4u * KC * ROWS * 16u + FIXED <= kMaxSmem;
-    static constexpr int NBUF = (DB_ODD || DB_EVEN) ? 2 : 1;
-    static constexpr int R = DB_ODD ? (ROWS | 1) : (DB_EVEN ? ROWS : (ROWS | 1));
+    static constexpr int KC = C / 8;                       // 16-byte chunks (8 fp16) along the contraction axis
+    static constexpr int C4 = C / 4;                       // 4-channel groups of a row
+    static constexpr int NBUF = 2;                         // sigmoid tiles / accumulators in flight
+    static constexpr int R = ROWS | 1;                     // rows of a tile chunk (odd: conflict-free stores)
     static constexpr unsigned LBO_A = R * 16u;             // chunk pitch of the sigmoid tile
-    static constexpr unsigned A_BYTES = KC * LBO_A;
+    static constexpr unsigned A_BYTES = (KC * LBO_A + 127u) / 128u * 128u;  // one half (hi or lo)
+    static constexpr unsigned RAW_BYTES = (ROWS * C * 4u + 127u) / 128u * 128u;  // fp32 input tile [ROWS][C]
     static constexpr unsigned LBO_W = C * 16u;             // chunk pitch of one tap's weights
-    static constexpr unsigned W_TAP = KC * LBO_W;          // = C * C * 4
+    static constexpr unsigned W_TAP = KC * LBO_W;          // = C * C * 2
     static constexpr unsigned W_BYTES = KT * W_TAP;
-    // buffer b: hi at OFF_A(b), lo at OFF_A(b) + A_BYTES
-    static constexpr unsigned OFF_WHI = NBUF * 2 * A_BYTES, OFF_WLO = OFF_WHI + W_BYTES;
+    // buffer b: hi at b * 2 A_BYTES, lo A_BYTES later; then the input tiles, weights hi / lo, bias
+    static constexpr unsigned OFF_RAW = NBUF * 2 * A_BYTES;
+    static constexpr unsigned OFF_WHI = OFF_RAW + NBUF * RAW_BYTES, OFF_WLO = OFF_WHI + W_BYTES;
     static constexpr unsigned OFF_BIAS = OFF_WLO + W_BYTES;
-    static constexpr unsigned OFF_BAR = (OFF_BIAS + C * 4u + 15u) & ~15u;  // NBUF mbarriers, then the TMEM slot
-    static constexpr unsigned SMEM_BYTES = OFF_BAR + 32u + 128u;           // + alignment slack
-    static_assert(SMEM_BYTES <= kMaxSmem, "shared memory");
+    static constexpr unsigned OFF_BAR = (OFF_BIAS + C * 4u + 15u) & ~15u;  // 5 NBUF mbarriers, then the TMEM slot
+    static constexpr unsigned SMEM_BYTES = OFF_BAR + 96u + 128u;           // + alignment slack
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
     // one fp32 accumulator of C columns per buffer, in a power-of-two allocation >= 32
     static constexpr unsigned TMEM_COLS = NBUF * C <= 32 ? 32u : (NBUF * C <= 64 ? 64u : 128u);
-    static constexpr int NLOAD = (ROWS * KC + kGateThreads - 1) / kGateThreads;  // 4-vectors per thread
-    static constexpr int NMMA = 3 * KT * (C / 8);
-    static constexpr int OPITCH = C + 4;  // row pitch (floats) of the output tile staged in a free tile buffer
-    static_assert(kGateM * OPITCH * 4u <= 2u * A_BYTES, "output tile must fit in one tile buffer");
 };
 
-__device__ __forceinline__ void split_tf32(float x, float &hi, float &lo) {
-    hi = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
-    lo = x - hi;
+// fp16 split of x: hi = x rounded to fp16, lo = the remainder rounded to fp16
+// (|x - hi - lo| <= 2^-22 |x| while the parts are normal numbers).
+__device__ __forceinline__ void split_f16(float x, __half &hi, __half &lo) {
+    hi = __float2half_rn(x);
+    lo = __float2half_rn(x - __half2float(hi));
+}
+// four consecutive channels split, packed as two 8-byte words (hi, lo);
+// two channels per conversion (packed fp32 -> fp16x2 and back)
+__device__ __forceinline__ void split4_f16(float4 x, uint2 &hi, uint2 &lo) {
+    const __half2 h01 = __floats2half2_rn(x.x, x.y), h23 = __floats2half2_rn(x.z, x.w);
+    const float2 b01 = __half22float2(h01), b23 = __half22float2(h23);
+    const __half2 l01 = __floats2half2_rn(x.x - b01.x, x.y - b01.y), l23 = __floats2half2_rn(x.z - b23.x, x.w - b23.y);
+    hi = make_uint2(*reinterpret_cast<const uint32_t *>(&h01), *reinterpret_cast<const uint32_t *>(&h23));
+    lo = make_uint2(*reinterpret_cast<const uint32_t *>(&l01), *reinterpret_cast<const uint32_t *>(&l23));
+}
+
+// Instruction descriptor of a dense kind::f16 MMA with fp16 A and B, fp32
+// accumulator, both operands K-major, M = 128, N = n.
+__host__ __device__ constexpr uint32_t gate_idesc_f16(int n) {
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16_elect(unsigned tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               bool accumulate) {
+    asm volatile(
+        "{\n .reg .pred p, e;\n setp.ne.b32 p, %4, 0;\n elect.sync _|e, 0xffffffff;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"((unsigned)accumulate)
+        : "memory");
 }
 
 // Logistic function from the fast exponential and reciprocal (both within a
@@ -155,6 +175,16 @@ __device__ __forceinline__ void store4(__nv_bfloat16 *p, const float (&v)[4], bo
     }
 }
 
+// Warp roles (sixteen warps): warps 0-7 drain the accumulators (warp w
+// reads TMEM lanes 32 (w % 4) .. +31, i.e. time steps, and the column half
+// w / 4), warp 8 issues the MMAs (one lane, elect.sync), warps 9-15 stage
+// sigmoid tiles.  Tiles and accumulators (NBUF of each) are handed over on
+// mbarriers -- full / empty for the sigmoid tiles, acc_full / acc_empty for
+// the accumulators -- so no role waits at a CTA-wide barrier in the steady
+// state.
+constexpr int kGateEpiWarps = 8, kGateMmaWarp = 8, kGateProdWarp0 = 9;
+constexpr int kGateProdThreads = kGateThreads - 32 * kGateProdWarp0;
+
 // grid = H * groups CTAs; CTA (h = blockIdx.x % H, j = blockIdx.x / H) takes
 // the tiles j, j + groups, ... of head h, tile = b * tiles_per_row + t0 / 128.
 // vec_in: a's rows allow 4-channel vector loads; vec_out: g allows 16-byte stores.
@@ -162,74 +192,36 @@ template <int C, int KT, typename IO>
 __global__ void __launch_bounds__(kGateThreads, 1)
     mhf_gate_kernel(const IO *__restrict__ a, const float *__restrict__ w, const float *__restrict__ bias,
                     IO *__restrict__ g, int L, int D, int H, int groups, int tiles_per_row, int num_tiles,
-                    int vec_in, int vec_out) {
+                    int vec_in, int vec_out, const __grid_constant__ CUtensorMap tma_a, int use_tma) {
     using Cfg = GateCfg<C, KT>;
+    constexpr int NB = Cfg::NBUF;
     extern __shared__ unsigned char gate_smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(((uintptr_t)gate_smem_raw + 127) & ~(uintptr_t)127);
     const unsigned sb = smem_u32(sm);
     float *sbias = reinterpret_cast<float *>(sm + Cfg::OFF_BIAS);
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + Cfg::OFF_BAR);  // bar[0 .. NBUF-1]
-    unsigned *tslot = reinterpret_cast<unsigned *>(sm + Cfg::OFF_BAR + 16);
+    // full[NB], empty[NB], acc_full[NB], acc_empty[NB], loaded[NB], then the TMEM slot
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + Cfg::OFF_BAR);
+    uint64_t *empty = full + NB, *acc_full = full + 2 * NB, *acc_empty = full + 3 * NB, *loaded = full + 4 * NB;
+    unsigned *tslot = reinterpret_cast<unsigned *>(loaded + NB);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.x % H;
     const int64_t col0 = (int64_t)h * C;
+    const int first = blockIdx.x / H;
 
     if (warp == 0) tmem_alloc(tslot, Cfg::TMEM_COLS);
     if (tid == 0)
-        for (int i = 0; i < Cfg::NBUF; ++i) mbar_init(bar + i, 1);
-
-    // Two register sets of raw a: tile j of this CTA's sequence uses set j % 2,
-    // so the loads of tiles j+2 and j+3 are in flight while j+1 is staged.
-    Raw4<IO> raw0[Cfg::NLOAD], raw1[Cfg::NLOAD];
-    auto load_tile = [&](Raw4<IO>(&raw)[Cfg::NLOAD], int tile) {
-        const int b = tile / tiles_per_row;
-        const int t0 = (tile % tiles_per_row) * kGateM;
-        const IO *base = a + (int64_t)b * L * D + col0;
-#pragma unroll
-        for (int j = 0; j < Cfg::NLOAD; ++j) {
-            const int i = tid + j * kGateThreads;
-            const int r = i / Cfg::KC, kc = i % Cfg::KC;
-            const int t = t0 - (KT - 1) + r;
-            if (i < Cfg::ROWS * Cfg::KC && t >= 0 && t < L)
-                raw[j].load(base + (int64_t)t * D + kc * 4, vec_in != 0);
-            else
-                raw[j].zero();
+        for (int i = 0; i < NB; ++i) {
+            mbar_init(full + i, kGateThreads / 32 - kGateProdWarp0);  // one arrival per producer warp
+            mbar_init(empty + i, 1);                                  // tcgen05.commit
+            mbar_init(acc_full + i, 1);                               // tcgen05.commit
+            mbar_init(acc_empty + i, kGateEpiWarps);                  // one arrival per epilogue warp
+            mbar_init(loaded + i, 1);                                 // TMA of a tile's input
         }
-    };
-    auto stage_tile = [&](Raw4<IO>(&raw)[Cfg::NLOAD], int tile, int buf) {
-        unsigned char *ahi = sm + buf * 2 * Cfg::A_BYTES, *alo = ahi + Cfg::A_BYTES;
-        const int t0 = (tile % tiles_per_row) * kGateM;
-#pragma unroll
-        for (int j = 0; j < Cfg::NLOAD; ++j) {
-            const int i = tid + j * kGateThreads;
-            if (i >= Cfg::ROWS * Cfg::KC) break;
-            const int r = i / Cfg::KC, kc = i % Cfg::KC;
-            const int t = t0 - (KT - 1) + r;
-            float4 s = make_float4(0.f, 0.f, 0.f, 0.f);  // the convolution's zero padding
-            if (t >= 0 && t < L) {
-                const float4 x = raw[j].f32();
-                s = make_float4(logistic(x.x), logistic(x.y), logistic(x.z), logistic(x.w));
-            }
-            float4 hi, lo;
-            split_tf32(s.x, hi.x, lo.x);
-            split_tf32(s.y, hi.y, lo.y);
-            split_tf32(s.z, hi.z, lo.z);
-            split_tf32(s.w, hi.w, lo.w);
-            const unsigned off = kc * Cfg::LBO_A + r * 16u;
-            *reinterpret_cast<float4 *>(ahi + off) = hi;
-            *reinterpret_cast<float4 *>(alo + off) = lo;
-        }
-    };
 
-    // the first two tiles' a is in flight while the weights are staged
-    int tile = blockIdx.x / H;
-    if (tile < num_tiles) load_tile(raw0, tile);
-    if (tile + groups < num_tiles) load_tile(raw1, tile + groups);
-
-    // The head's weights, split into tf32 hi / lo, in the K-major layout:
-    // tap k, chunk c/4, output channel n, element c%4.  One thread fills one
-    // 16-byte slot (k, chunk, n) from four gathered loads of w ([D][C][K]);
+    // The head's weights, split into fp16 hi / lo, in the K-major layout: tap
+    // k, chunk c/8, output channel n, element c%8.  One thread fills one
+    // 16-byte slot (k, chunk, n) from eight gathered loads of w ([D][C][K]);
     // consecutive threads take consecutive n, so the slot stores are
     // conflict-free.  (The head's block is read once per CTA, from L2 after
     // the first CTA of the head.)
@@ -237,152 +229,223 @@ __global__ void __launch_bounds__(kGateThreads, 1)
 #pragma unroll 2
     for (int sl = tid; sl < KT * Cfg::KC * C; sl += kGateThreads) {
         const int n = sl % C, kc = (sl / C) % Cfg::KC, k = sl / (C * Cfg::KC);
-        const float *src = wh + ((int64_t)n * C + kc * 4) * KT + k;
-        float4 hi, lo;
-        split_tf32(__ldg(src), hi.x, lo.x);
-        split_tf32(__ldg(src + KT), hi.y, lo.y);
-        split_tf32(__ldg(src + 2 * KT), hi.z, lo.z);
-        split_tf32(__ldg(src + 3 * KT), hi.w, lo.w);
+        const float *src = wh + ((int64_t)n * C + kc * 8) * KT + k;
+        uint2 h0, l0, h1, l1;
+        split4_f16(make_float4(__ldg(src), __ldg(src + KT), __ldg(src + 2 * KT), __ldg(src + 3 * KT)), h0, l0);
+        split4_f16(make_float4(__ldg(src + 4 * KT), __ldg(src + 5 * KT), __ldg(src + 6 * KT), __ldg(src + 7 * KT)), h1,
+                   l1);
         const unsigned off = k * Cfg::W_TAP + kc * Cfg::LBO_W + n * 16u;
-        *reinterpret_cast<float4 *>(sm + Cfg::OFF_WHI + off) = hi;
-        *reinterpret_cast<float4 *>(sm + Cfg::OFF_WLO + off) = lo;
+        *reinterpret_cast<uint4 *>(sm + Cfg::OFF_WHI + off) = make_uint4(h0.x, h0.y, h1.x, h1.y);
+        *reinterpret_cast<uint4 *>(sm + Cfg::OFF_WLO + off) = make_uint4(l0.x, l0.y, l1.x, l1.y);
     }
     if (tid < C) sbias[tid] = bias ? __ldg(bias + col0 + tid) : 0.0f;
-
+    fence_proxy_async_smem();  // the weights are read by the tensor core
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const unsigned tmem = *tslot;
-    constexpr uint32_t idesc = umma_idesc_tf32(kGateM, C);
+    bool ok = true;    // every wait of this thread's role completed
+    int last_it = -1;  // MMA warp: the last tile whose MMAs it committed
 
-    // MMAs of one tile: 3 split products x K taps x C/8 steps of 8 channels,
-    // into accumulator `buf`; committed to bar[buf].  Run by all of warp 0.  Descriptors advance by
-    // (byte offset >> 4) in their address field.
-    auto issue = [&](int buf) {
-        const unsigned d = tmem + buf * C;
-        const unsigned abase = sb + buf * 2 * Cfg::A_BYTES;
-        int step = 0;
+    if (warp >= kGateProdWarp0) {
+        // ---- producers: sigmoid tiles, split into fp16 hi / lo, into buffer it % NB.
+        // Item i of a tile is time step r = i / (C/4) (tile row, t = t0 - (KT-1) + r)
+        // and channels 4 c4 .. 4 c4 + 3, c4 = i % (C/4): 8-byte halves of 16-byte chunks.
+        const int pt = tid - 32 * kGateProdWarp0;
+        constexpr int NITEM = Cfg::ROWS * Cfg::C4;
+        constexpr int NU = (NITEM + kGateProdThreads - 1) / kGateProdThreads;
+        // sigmoid of item j of this thread (zero outside [0, L): the convolution's padding),
+        // split and stored into buffer buf
+        auto put = [&](int buf, int t0, int j, float4 x) {
+            const int i = pt + j * kGateProdThreads;
+            const int r = i / Cfg::C4, c4 = i % Cfg::C4;
+            const int t = t0 - (KT - 1) + r;
+            float4 sg = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (t >= 0 && t < L) sg = make_float4(logistic(x.x), logistic(x.y), logistic(x.z), logistic(x.w));
+            uint2 hi, lo;
+            split4_f16(sg, hi, lo);
+            unsigned char *ahi = sm + buf * 2 * Cfg::A_BYTES;
+            const unsigned off = (c4 >> 1) * Cfg::LBO_A + r * 16u + (c4 & 1) * 8u;
+            *reinterpret_cast<uint2 *>(ahi + off) = hi;
+            *reinterpret_cast<uint2 *>(ahi + Cfg::A_BYTES + off) = lo;
+        };
+        auto publish = [&](int buf) {
+            fence_proxy_async_smem();  // this thread's tile stores, before the tensor core reads them
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full + buf);
+        };
+        int it = 0;
+        constexpr bool kTmaIn = sizeof(IO) == 4;
+        if (kTmaIn && use_tma) {
+            // a tile's input [ROWS t][C ch] arrives by one TMA box in the buffer's input
+            // tile (rows outside [0, L) read as zero and are masked in put)
+            auto fetch = [&](int tile, int buf) {
+                const int b = tile / tiles_per_row, t0 = (tile % tiles_per_row) * kGateM;
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(loaded + buf, (unsigned)(Cfg::ROWS * C * 4));
+                tma_load_3d(sm + Cfg::OFF_RAW + buf * Cfg::RAW_BYTES, &tma_a, (int)col0, t0 - (KT - 1), b,
+                            loaded + buf);
+            };
+            int fetched = -1;  // thread pt == 0: the last tile iteration whose input it requested
+            if (pt == 0 && first < num_tiles) {
+                fetch(first, 0);
+                fetched = 0;
+            }
+            for (int tile = first; tile < num_tiles; tile += groups, ++it) {
+                const int buf = it % NB;
+                // every producer agrees on whether the input arrived in time
+                if (!bar_and(1, kGateProdThreads, mbar_wait_bounded(loaded + buf, (it / NB) & 1u))) {
+                    ok = false;
+                    break;
+                }
+                const int t0 = (tile % tiles_per_row) * kGateM;
+                const unsigned char *raw = sm + Cfg::OFF_RAW + buf * Cfg::RAW_BYTES;
+#pragma unroll
+                for (int j = 0; j < NU; ++j) {
+                    const int i = pt + j * kGateProdThreads;
+                    if (i >= NITEM) break;
+                    put(buf, t0, j, *reinterpret_cast<const float4 *>(raw + (i / Cfg::C4) * (C * 4) + (i % Cfg::C4) * 16));
+                }
+                publish(buf);
+                // the next tile's input, once its buffer's previous MMAs are done (which also
+                // means every producer has read that buffer's input tile)
+                const int nt = tile + groups, nbuf = (it + 1) % NB;
+                if (pt == 0 && nt < num_tiles) {
+                    if (it + 1 >= NB && !mbar_wait_bounded(empty + nbuf, ((it + 1) / NB - 1) & 1u)) {
+                        ok = false;  // nothing more is requested; the others time out on loaded
+                    } else {
+                        fetch(nt, nbuf);
+                        fetched = it + 1;
+                    }
+                }
+            }
+            // a request still in flight lands before the CTA's shared memory is released
+            if (pt == 0 && fetched >= it && fetched >= 0) mbar_wait_bounded(loaded + fetched % NB, (fetched / NB) & 1u);
+        } else {
+            // loads from global memory, the next tile's into the other register set
+            // before this tile's sigmoid is computed
+            Raw4<IO> raw0[NU], raw1[NU];
+            auto load = [&](Raw4<IO>(&rw)[NU], int tile) {
+                const int b = tile / tiles_per_row;
+                const int t0 = (tile % tiles_per_row) * kGateM;
+                const IO *base = a + (int64_t)b * L * D + col0;
+#pragma unroll
+                for (int j = 0; j < NU; ++j) {
+                    const int i = pt + j * kGateProdThreads;
+                    const int r = i / Cfg::C4, c4 = i % Cfg::C4;
+                    const int t = t0 - (KT - 1) + r;
+                    if (i < NITEM && t >= 0 && t < L)
+                        rw[j].load(base + (int64_t)t * D + c4 * 4, vec_in != 0);
+                    else
+                        rw[j].zero();
+                }
+            };
+            auto produce = [&](Raw4<IO>(&rw)[NU], int tile, int itx) -> bool {
+                const int buf = itx % NB;
+                if (itx >= NB && !mbar_wait_bounded(empty + buf, ((itx / NB) - 1) & 1u)) return false;
+                const int t0 = (tile % tiles_per_row) * kGateM;
+#pragma unroll
+                for (int j = 0; j < NU; ++j) {
+                    if (pt + j * kGateProdThreads >= NITEM) break;
+                    put(buf, t0, j, rw[j].f32());
+                }
+                publish(buf);
+                return true;
+            };
+            if (first < num_tiles) load(raw0, first);
+            for (int tile = first; tile < num_tiles && ok; tile += 2 * groups, it += 2) {
+                const int t1 = tile + groups, t2 = tile + 2 * groups;
+                if (t1 < num_tiles) load(raw1, t1);
+                ok = produce(raw0, tile, it);
+                if (!ok || t1 >= num_tiles) break;
+                if (t2 < num_tiles) load(raw0, t2);
+                ok = produce(raw1, t1, it + 1);
+            }
+        }
+    } else if (warp == kGateMmaWarp) {
+        // ---- MMA issue: 3 split products x K taps x C/16 steps of 16 channels per tile
+        constexpr uint32_t idesc = gate_idesc_f16(C);
+        int it = 0;
+        last_it = -1;
+        for (int tile = first; tile < num_tiles; tile += groups, ++it) {
+            const int buf = it % NB;
+            bool got = mbar_wait_bounded(full + buf, (it / NB) & 1u);
+            if (got && it >= NB) got = mbar_wait_bounded(acc_empty + buf, ((it / NB) - 1) & 1u);
+            if (!__all_sync(0xffffffffu, got)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after_sync();
+            const unsigned d = tmem + buf * C;
+            const unsigned abase = sb + buf * 2 * Cfg::A_BYTES;
+            int step = 0;
 #pragma unroll 1
-        for (int p = 0; p < 3; ++p) {  // hi*W_hi, hi*W_lo, lo*W_hi
-            const uint64_t a0 = umma_smem_desc(abase + (p < 2 ? 0u : Cfg::A_BYTES), Cfg::LBO_A, 128u);
-            const uint64_t b0 = umma_smem_desc(sb + (p == 1 ? Cfg::OFF_WLO : Cfg::OFF_WHI), Cfg::LBO_W, 128u);
+            for (int p = 0; p < 3; ++p) {  // hi*W_hi, hi*W_lo, lo*W_hi
+                const uint64_t a0 = umma_smem_desc(abase + (p < 2 ? 0u : Cfg::A_BYTES), Cfg::LBO_A, 128u);
+                const uint64_t b0 = umma_smem_desc(sb + (p == 1 ? Cfg::OFF_WLO : Cfg::OFF_WHI), Cfg::LBO_W, 128u);
 #pragma unroll
-            for (int k = 0; k < KT; ++k) {
+                for (int k = 0; k < KT; ++k) {
 #pragma unroll
-                for (int s = 0; s < C / 8; ++s) {
-                    umma_tf32_elect(d, a0 + ((k * 16u + 2u * s * Cfg::LBO_A) >> 4),
-                              b0 + ((k * Cfg::W_TAP + 2u * s * Cfg::LBO_W) >> 4), idesc, step > 0);
-                    ++step;
+                    for (int s2 = 0; s2 < C / 16; ++s2) {
+                        umma_f16_elect(d, a0 + ((k * 16u + 2u * s2 * Cfg::LBO_A) >> 4),
+                                       b0 + ((k * Cfg::W_TAP + 2u * s2 * Cfg::LBO_W) >> 4), idesc, step > 0);
+                        ++step;
+                    }
                 }
             }
+            umma_commit_elect(empty + buf);     // the sigmoid tile may be restaged
+            umma_commit_elect(acc_full + buf);  // the accumulator is ready
+            last_it = it;
         }
-        umma_commit_elect(bar + buf);
-    };
-    // the staged tile (generic-proxy stores) is made visible to the tensor
-    // core, and every warp's earlier reads of the accumulator are ordered
-    // before the MMAs that overwrite it
-    auto publish = [&]() {
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
-        tc_fence_after_sync();
-    };
-
-    // stage tile `stile` from register set s into tile buffer `buf`, start its
-    // MMAs, then refill set s with tile `ltile` (the one two places later)
-    auto stage_issue_load = [&](int s, int stile, int buf, int ltile) {
-        if (s) stage_tile(raw1, stile, buf);
-        else stage_tile(raw0, stile, buf);
-        publish();
-        if (warp == 0) issue(buf);  // the whole warp runs the loop, one lane issues
-        if (ltile < num_tiles) {
-            if (s) load_tile(raw1, ltile);
-            else load_tile(raw0, ltile);
-        }
-    };
-
-    unsigned parity = 0u, pending = 0u;  // bit i: phase parity awaited on / MMAs in flight on bar[i]
-    bool ok = true;
-    if (tile < num_tiles) {
-        stage_issue_load(0, tile, 0, tile + 2 * groups);
-        pending |= 1u;
-    }
-    for (int it = 0; tile < num_tiles; tile += groups, ++it) {
-        const int cur = Cfg::NBUF == 2 ? (it & 1) : 0;
-        const int next = tile + groups;
-        if (Cfg::NBUF == 2 && next < num_tiles) {
-            // the other buffer's MMAs completed in the previous iteration
-            stage_issue_load((it + 1) & 1, next, cur ^ 1, next + 2 * groups);
-            pending |= 1u << (cur ^ 1);
-        }
-        // one thread waits for this tile's MMAs; the barrier releases the rest
-        bool done = true;
-        if (tid == 0) done = mbar_wait_bounded(bar + cur, (parity >> cur) & 1u);
-        if (!__syncthreads_and(done)) {
-            ok = false;
-            break;
-        }
-        parity ^= 1u << cur;
-        pending &= ~(1u << cur);
-        tc_fence_after_sync();
-
-        // accumulator row m = 32 (warp % 4) + lane (time step t0 + m); warp w
-        // takes the column quarter w / 4.  Rows are staged (with the bias) in
-        // this tile's buffer, whose MMAs are done, then written out as whole
-        // C-channel rows by consecutive threads.
-        {
-            const int q = warp & 3, cbase = (warp >> 2) * (C / 4);
-            float *otile = reinterpret_cast<float *>(sm + cur * 2 * Cfg::A_BYTES);
-            float *orow = otile + (q * 32 + lane) * Cfg::OPITCH + cbase;
-            const unsigned trow = tmem + cur * C + ((unsigned)(q * 32) << 16) + cbase;
-            if constexpr (C / 4 == 16) {
-                float v[16];
+    } else if (warp < kGateEpiWarps) {
+        // ---- epilogue: accumulator rows 32 warp + lane (time steps), all C columns, + bias, store
+        int it = 0;
+        for (int tile = first; tile < num_tiles; tile += groups, ++it) {
+            const int buf = it % NB;
+            const bool got = mbar_wait_bounded(acc_full + buf, (it / NB) & 1u);
+            if (!__all_sync(0xffffffffu, got)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after_sync();
+            constexpr int CH = C / 2;  // this warp's columns: [CH (warp / 4), +CH)
+            const int cb = CH * (warp >> 2);
+            float v[CH];
+            const unsigned trow = tmem + buf * C + cb + ((unsigned)(32 * (warp & 3)) << 16);
+            if constexpr (CH == 32) {
+                float x0[16], x1[16];
+                tmem_ld16x2(trow, trow + 16, x0, x1);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    v[i] = x0[i];
+                    v[16 + i] = x1[i];
+                }
+            } else if constexpr (CH == 16) {
                 tmem_ld16(trow, v);
-#pragma unroll
-                for (int i = 0; i < 16; i += 4)
-                    *reinterpret_cast<float4 *>(orow + i) = make_float4(
-                        v[i] + sbias[cbase + i], v[i + 1] + sbias[cbase + i + 1], v[i + 2] + sbias[cbase + i + 2],
-                        v[i + 3] + sbias[cbase + i + 3]);
-            } else if constexpr (C / 4 == 8) {
-                float v[8];
-                tmem_ld8(trow, v);
-#pragma unroll
-                for (int i = 0; i < 8; i += 4)
-                    *reinterpret_cast<float4 *>(orow + i) = make_float4(
-                        v[i] + sbias[cbase + i], v[i + 1] + sbias[cbase + i + 1], v[i + 2] + sbias[cbase + i + 2],
-                        v[i + 3] + sbias[cbase + i + 3]);
             } else {
-                float v[4];
-                tmem_ld4(trow, v);
-                *reinterpret_cast<float4 *>(orow) =
-                    make_float4(v[0] + sbias[cbase], v[1] + sbias[cbase + 1], v[2] + sbias[cbase + 2],
-                                v[3] + sbias[cbase + 3]);
+                tmem_ld8(trow, v);
             }
-            __syncthreads();
-            const int b = tile / tiles_per_row, t0 = (tile % tiles_per_row) * kGateM;
-            IO *gt = g + ((int64_t)b * L + t0) * D + col0;
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty + buf);  // the MMAs of tile it + NB may overwrite it
+            const int b = tile / tiles_per_row, m = 32 * (warp & 3) + lane;
+            const int t = (tile % tiles_per_row) * kGateM + m;
+            if (t < L) {
+                IO *gt = g + ((int64_t)b * L + t) * D + col0 + cb;
 #pragma unroll
-            for (int i = tid; i < kGateM * (C / 4); i += kGateThreads) {
-                const int m = i / (C / 4), c4 = i % (C / 4);
-                if (t0 + m < L) {
-                    const float4 x = *reinterpret_cast<const float4 *>(otile + m * Cfg::OPITCH + 4 * c4);
-                    const float xv[4] = {x.x, x.y, x.z, x.w};
-                    store4(gt + (int64_t)m * D + 4 * c4, xv, vec_out != 0);
+                for (int c = 0; c < CH; c += 4) {
+                    const float xv[4] = {v[c] + sbias[cb + c], v[c + 1] + sbias[cb + c + 1],
+                                         v[c + 2] + sbias[cb + c + 2], v[c + 3] + sbias[cb + c + 3]};
+                    store4(gt + c, xv, vec_out != 0);
                 }
             }
-            __syncthreads();  // the buffer is staged into again
-        }
-        if (Cfg::NBUF == 1 && next < num_tiles) {
-            // single buffer: the next tile is staged once this one's MMAs are done
-            stage_issue_load((it + 1) & 1, next, 0, next + 2 * groups);
-            pending |= 1u;
         }
     }
-    if (!ok && tid == 0) {
-        atomicOr(&g_cc_fault, kFaultMmaWait);
-        for (int i = 0; i < Cfg::NBUF; ++i)  // give the MMAs in flight a last chance to finish
-            if ((pending >> i) & 1u) mbar_wait_bounded(bar + i, (parity >> i) & 1u);
-    }
+    if (!ok && lane == 0) atomicOr(&g_cc_fault, kFaultMmaWait);
+    // every MMA this CTA issued has completed before the accumulators are
+    // freed: the last commit tracks all of them (a phase the epilogue has
+    // already seen completes the wait at once)
+    if (warp == kGateMmaWarp && last_it >= 0) mbar_wait_bounded(acc_full + last_it % NB, (last_it / NB) & 1u);
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 0) {

@@ -252,6 +252,70 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
         if (tid == 0) prefetch(cid);
         in_flight = true;
     }
+    // The direct head's inputs (thread tid < 256: row tid >> 7, v or g, time
+    // step tid & 63) of group gi, loaded a group ahead so their latency hides
+    // behind the previous group's stages.
+    auto load_head = [&](int gi) -> float {
+        if (tid >= 4 * kTcHead || gi >= num_groups) return 0.f;
+        const int bb = gi / groups_per_batch, dd = (gi - bb * groups_per_batch) * kTcGroup;
+        const int x = tid >> 7, arr = (tid >> 6) & 1, t = tid & 63, c = 2 * q + x;
+        if (t >= L || c >= D - dd) return 0.f;
+        const int ts = (arr == 0 && (rev & 1)) ? L - 1 - t : t;
+        return __bfloat162float((arr ? g : v)[(int64_t)bb * L * D + dd + c + (int64_t)ts * D]);
+    };
+    float hreg = load_head(cid);
+    // Row norms of group gi: the CTA's partial sums over its time steps (tot)
+    // are published by a cluster barrier.  For every group after the first,
+    // they are computed from the staged input at the end of the previous
+    // group (before its last barrier), so that group needs no barrier of
+    // its own for them.
+    bool have_norms = false;
+    // partial sums of the squares of this thread's (v, g) elements -> warp partials in red2 -> tot
+    auto norms = [&](const float (&av)[4][4], const float (&ag)[4][4], float *red2) {
+        float sq[8];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            sq[c] = 0.f;
+            sq[4 + c] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                sq[c] = fmaf(av[i][c], av[i][c], sq[c]);
+                sq[4 + c] = fmaf(ag[i][c], ag[i][c], sq[4 + c]);
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sq[c] += __shfl_xor_sync(0xffffffffu, sq[c], o);
+        }
+        if (lane == 0)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) red2[warp * 8 + c] = sq[c];
+        __syncthreads();
+        if (tid < 16) {  // channel c = tid & 7 (half c / 4: warps 8 (c / 4) .. +8), stream tid >> 3
+            const int c = tid & 7, st = tid >> 3, h = c >> 2;
+            float acc = 0.f;
+            for (int w2 = 8 * h; w2 < 8 * h + 8; ++w2) acc += red2[w2 * 8 + 4 * st + (c & 3)];
+            tot[tid] = acc;
+        }
+    };
+    // this thread's staged elements (time steps n2 + 128 (4 (2q + kl) + i), channels [4 hf, +4))
+    auto read_staged = [&](int n2i, int kl, int hf, float (&av)[4][4], float (&ag)[4][4]) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int tl = n2i + 128 * (4 * kl + i);
+            const uint2 wv = *reinterpret_cast<const uint2 *>(sin_v + ((rev & 1) ? kTcSpan - 1 - tl : tl) * 8 + 4 * hf);
+            const uint2 wg = *reinterpret_cast<const uint2 *>(sin_g + tl * 8 + 4 * hf);
+            av[i][0] = __uint_as_float(wv.x << 16);
+            av[i][1] = __uint_as_float(wv.x & 0xFFFF0000u);
+            av[i][2] = __uint_as_float(wv.y << 16);
+            av[i][3] = __uint_as_float(wv.y & 0xFFFF0000u);
+            ag[i][0] = __uint_as_float(wg.x << 16);
+            ag[i][1] = __uint_as_float(wg.x & 0xFFFF0000u);
+            ag[i][2] = __uint_as_float(wg.y << 16);
+            ag[i][3] = __uint_as_float(wg.y & 0xFFFF0000u);
+        }
+    };
 
     // stage s (1..4) of row x: 4 or 8 MMAs of K = 16 (two 16-byte chunks each), one thread issues
     auto issue = [&](int s, int x) {
@@ -304,29 +368,20 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
         const int nh = max(0, min(4, nch - 4 * hf));  // channels of this thread's half that exist
         float xv[4][4], xg[4][4];
         bool staged = true;
-        __syncthreads();  // the previous group's stores have read the output staging (reused below)
-        if (use_tma) {
+        if (use_tma && in_flight) {
             // the copy engine zero-filled t >= L (and t < 0 for a reversed v) and d >= D
-            if (tid == 0 && in_flight) staged = mbar_wait_bounded(bar + 2, in_phase);
-            staged = __syncthreads_and(staged) && in_flight;
+            if (tid == 0) staged = mbar_wait_bounded(bar + 2, in_phase);
+            staged = __syncthreads_and(staged);
             if (staged) {
                 in_phase ^= 1u;
                 in_flight = false;
             }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int tl = n2i + 128 * (4 * kl + i);
-                const uint2 wv = *reinterpret_cast<const uint2 *>(sin_v + ((rev & 1) ? kTcSpan - 1 - tl : tl) * 8 + 4 * hf);
-                const uint2 wg = *reinterpret_cast<const uint2 *>(sin_g + tl * 8 + 4 * hf);
-                xv[i][0] = __uint_as_float(wv.x << 16);
-                xv[i][1] = __uint_as_float(wv.x & 0xFFFF0000u);
-                xv[i][2] = __uint_as_float(wv.y << 16);
-                xv[i][3] = __uint_as_float(wv.y & 0xFFFF0000u);
-                xg[i][0] = __uint_as_float(wg.x << 16);
-                xg[i][1] = __uint_as_float(wg.x & 0xFFFF0000u);
-                xg[i][2] = __uint_as_float(wg.y << 16);
-                xg[i][3] = __uint_as_float(wg.y & 0xFFFF0000u);
-            }
+        } else {
+            __syncthreads();  // the previous group's stores have read the output staging (reused below)
+        }
+        ok = ok && staged;
+        if (use_tma) {
+            read_staged(n2i, kl, hf, xv, xg);
         } else {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -337,47 +392,11 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
                 tc_load4(g + base + 4 * hf + (int64_t)(in ? t : 0) * D, nh, vec, in, xg[i]);
             }
         }
-        ok = ok && staged;
-        // this CTA's rows' first time steps, for the direct head (one element per thread)
-        if (tid < 4 * kTcHead) {
-            const int x = tid >> 7, arr = (tid >> 6) & 1, t = tid & 63;
-            const int c = 2 * q + x;
-            float val = 0.f;
-            if (t < L && c < nch) {
-                const int ts = (arr == 0 && (rev & 1)) ? L - 1 - t : t;
-                val = __bfloat162float((arr ? g : v)[base + c + (int64_t)ts * D]);
-            }
-            head[(x * 2 + arr) * kTcHead + t] = val;
+        if (tid < 4 * kTcHead) head[((tid >> 7) * 2 + ((tid >> 6) & 1)) * kTcHead + (tid & 63)] = hreg;
+        if (!have_norms) {
+            norms(xv, xg, red);  // red aliases the output staging, which no peer writes before barrier #2
+            cluster.sync();      // #1: partial sums visible
         }
-        {
-            float s[8];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                s[c] = 0.f;
-                s[4 + c] = 0.f;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    s[c] = fmaf(xv[i][c], xv[i][c], s[c]);
-                    s[4 + c] = fmaf(xg[i][c], xg[i][c], s[4 + c]);
-                }
-            }
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) s[c] += __shfl_xor_sync(0xffffffffu, s[c], o);
-            }
-            if (lane == 0)
-#pragma unroll
-                for (int c = 0; c < 8; ++c) red[warp * 8 + c] = s[c];
-        }
-        __syncthreads();
-        if (tid < 16) {  // channel c = tid & 7 (half c / 4: warps 8 (c / 4) .. +8), stream tid >> 3
-            const int c = tid & 7, st = tid >> 3, h = c >> 2;
-            float a = 0.f;
-            for (int w = 8 * h; w < 8 * h + 8; ++w) a += red[w * 8 + 4 * st + (c & 3)];
-            tot[tid] = a;
-        }
-        cluster.sync();  // #1: partial sums visible; every CTA is done with the previous group
         if (tid < 16) {
             float a = 0.f;
             const uint32_t ad = smem_u32(tot + tid);
@@ -410,6 +429,7 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
             if (tid == 0) prefetch(grp + nclusters);
             in_flight = true;
         }
+        hreg = load_head(grp + nclusters);
 
         issue(1, 0);
         issue(1, 1);
@@ -573,7 +593,24 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
                 if (s < 4) issue(s + 1, x);
             }
         }
-        cluster.sync();  // #3: every output of this CTA's time steps has arrived
+        // the next group's partial norms, from its staged input (the head buffer is free now)
+        have_norms = false;
+        if (use_tma && in_flight && ok) {
+            bool got = true;
+            if (tid == 0) got = mbar_wait_bounded(bar + 2, in_phase);
+            got = __syncthreads_and(got);
+            if (got) {
+                in_phase ^= 1u;
+                in_flight = false;
+                float nv[4][4], ng[4][4];
+                read_staged(n2i, kl, hf, nv, ng);
+                norms(nv, ng, head);
+                have_norms = true;
+            } else {
+                ok = false;
+            }
+        }
+        cluster.sync();  // #3: every output of this CTA's time steps has arrived; norms published
         // ---- store time steps [1024 q, 1024 q + 1024) of the 8 channels
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
