@@ -220,23 +220,33 @@ __global__ void __launch_bounds__(kGateThreads, 1)
         }
 
     // The head's weights, split into fp16 hi / lo, in the K-major layout: tap
-    // k, chunk c/8, output channel n, element c%8.  One thread fills one
-    // 16-byte slot (k, chunk, n) from eight gathered loads of w ([D][C][K]);
-    // consecutive threads take consecutive n, so the slot stores are
-    // conflict-free.  (The head's block is read once per CTA, from L2 after
-    // the first CTA of the head.)
-    const float *wh = w + col0 * C * KT;
+    // k, chunk c/8, output channel n, element c%8.  The head's block of w
+    // ([D][C][K], C K contiguous floats per output channel n) is read with
+    // coalesced 16-byte loads (vec_w: the block is 16-byte aligned) and each
+    // element is split and placed by 2-byte stores.  (The block is read once
+    // per CTA, from L2 after the first CTA of the head.)
+    {
+        const float *wh = w + col0 * C * KT;
+        constexpr int NW = C * C * KT;  // the head's weights
+        auto place = [&](int e, float x) {  // element e = (n C + c) KT + k
+            const int k = e % KT, c = (e / KT) % C, n = e / (KT * C);
+            const unsigned off = k * Cfg::W_TAP + (c >> 3) * Cfg::LBO_W + n * 16u + (c & 7) * 2u;
+            const __half hi = __float2half_rn(x), lo = __float2half_rn(x - __half2float(hi));
+            *reinterpret_cast<__half *>(sm + Cfg::OFF_WHI + off) = hi;
+            *reinterpret_cast<__half *>(sm + Cfg::OFF_WLO + off) = lo;
+        };
+        if (((uintptr_t)wh & 15) == 0) {
 #pragma unroll 2
-    for (int sl = tid; sl < KT * Cfg::KC * C; sl += kGateThreads) {
-        const int n = sl % C, kc = (sl / C) % Cfg::KC, k = sl / (C * Cfg::KC);
-        const float *src = wh + ((int64_t)n * C + kc * 8) * KT + k;
-        uint2 h0, l0, h1, l1;
-        split4_f16(make_float4(__ldg(src), __ldg(src + KT), __ldg(src + 2 * KT), __ldg(src + 3 * KT)), h0, l0);
-        split4_f16(make_float4(__ldg(src + 4 * KT), __ldg(src + 5 * KT), __ldg(src + 6 * KT), __ldg(src + 7 * KT)), h1,
-                   l1);
-        const unsigned off = k * Cfg::W_TAP + kc * Cfg::LBO_W + n * 16u;
-        *reinterpret_cast<uint4 *>(sm + Cfg::OFF_WHI + off) = make_uint4(h0.x, h0.y, h1.x, h1.y);
-        *reinterpret_cast<uint4 *>(sm + Cfg::OFF_WLO + off) = make_uint4(l0.x, l0.y, l1.x, l1.y);
+            for (int q4 = tid; q4 < NW / 4; q4 += kGateThreads) {
+                const float4 x = __ldg(reinterpret_cast<const float4 *>(wh) + q4);
+                place(4 * q4, x.x);
+                place(4 * q4 + 1, x.y);
+                place(4 * q4 + 2, x.z);
+                place(4 * q4 + 3, x.w);
+            }
+        } else {
+            for (int e = tid; e < NW; e += kGateThreads) place(e, __ldg(wh + e));
+        }
     }
     if (tid < C) sbias[tid] = bias ? __ldg(bias + col0 + tid) : 0.0f;
     fence_proxy_async_smem();  // the weights are read by the tensor core
