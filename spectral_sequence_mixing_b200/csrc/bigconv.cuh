@@ -27,6 +27,10 @@
 //
 // With CL > 1 (CL == R0) the CTA with cluster rank q holds the slots of
 // k0 == q; only pass 0, the mirror read and the inverse pass 0 cross CTAs.
+// With CL == R0 / 2 ("mirror pairs") CTA q holds k0 == q at local offsets
+// [0, SL) and k0 == R0-1-q at [SL, 2 SL): a bin and its mirror then share a
+// CTA (local offsets o and 2 SL-1-o), so the spectral product stays in the
+// CTA and only pass 0 and the inverse pass 0 exchange data between CTAs.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -50,6 +54,7 @@ struct BigCfg {
     static constexpr int HEAD = kHeadT0;
     static constexpr int WORDS = SC + SC / 16;  // padded float2 words
     static constexpr int PER0 = COLS0 / T;  // pass-0 columns per thread
+    static constexpr bool MIRROR = CL > 1 && 2 * CL == R0;  // k0 pairs (q, R0-1-q) per CTA
     static constexpr size_t SMEM_BYTES = (size_t)WORDS * 8 + (size_t)HEAD * 8 + (size_t)(T / 32 + 1) * 8;
     // Twiddle tables (float2), each factored into two small tables that stay
     // in L1 (value = product of two correctly rounded unit numbers):
@@ -68,7 +73,7 @@ struct BigCfg {
     static constexpr int TB = TAB + RA * (STA / QA);
     static constexpr int TW_SIZE = TB + RB * RC;
     static constexpr int LAST_R = RC > 1 ? RC : RB;
-    static_assert(CL == 1 || CL == R0, "a cluster splits the most significant digit");
+    static_assert(CL == 1 || CL == R0 || 2 * CL == R0, "a cluster splits the most significant digit");
     static_assert(LAST_R == 16, "innermost radix must be 16 (conflict-free padded layout)");
     static_assert(R0 <= 64 && RA <= 32 && RB <= 32 && RC <= 32, "register DFT sizes");
     static_assert(SC % (2 * T) == 0 && COLS0 % T == 0, "pass work split");
@@ -176,12 +181,21 @@ __global__ void __launch_bounds__(T, MINB)
     };
     if constexpr (CL > 1) cluster_sync();  // all CTAs of the cluster resident before any remote store
     // Slot (k0, n) of the row lives in CTA k0 / K0C at local offset
-    // (k0 % K0C) SL + n; with a cluster it is reached through the shared
-    // window address of that CTA (same layout in every CTA).
+    // (k0 % K0C) SL + n (mirror pairs: CTA min(k0, R0-1-k0), offset SL + n for
+    // the upper k0); with a cluster it is reached through the shared window
+    // address of that CTA (same layout in every CTA).
     const uint32_t xs_addr = smem_addr(xs);
     auto slot_addr = [&](int k0, int n) -> uint32_t {
-        const int owner = k0 / C::K0C;
-        const uint32_t local = xs_addr + 8u * (uint32_t)bc_pad((k0 - owner * C::K0C) * SL + n);
+        int owner, lk;
+        if constexpr (C::MIRROR) {
+            const bool up = k0 >= R0 / 2;
+            owner = up ? R0 - 1 - k0 : k0;
+            lk = up ? 1 : 0;
+        } else {
+            owner = k0 / C::K0C;
+            lk = k0 - owner * C::K0C;
+        }
+        const uint32_t local = xs_addr + 8u * (uint32_t)bc_pad(lk * SL + n);
         if constexpr (CL > 1) return cluster_map(local, owner);
         return local;
     };
@@ -283,26 +297,42 @@ __global__ void __launch_bounds__(T, MINB)
     } else {
         bc_local_pass<RB, 1, 1, SL, SC, T, false>(xs, tw, tw);
     }
-    cluster_sync();
+    if constexpr (C::MIRROR)
+        __syncthreads();
+    else
+        cluster_sync();
 
     // ---- spectral product X' = 4 V G.  The pair (s, S-1-s) is handled by the
     // thread that owns s at local offset o < SC/2 (the mirror then sits at a
-    // local offset >= SC/2, here or in CTA R0-1-rank): it reads both bins and
-    // writes X'_s and X'_{S-1-s} = conj(X'_s), so every slot is read and
-    // written by one thread only.
+    // local offset >= SC/2: SC-1-o in this CTA with mirror pairs, else in CTA
+    // R0-1-rank): it reads both bins and writes X'_s and X'_{S-1-s} =
+    // conj(X'_s), so every slot is read and written by one thread only.
     {
         constexpr int PER2 = SC / (2 * T);
+        if constexpr (C::MIRROR) {
 #pragma unroll 4
-        for (int i = 0; i < PER2; ++i) {
-            const int o = tid + i * T;
-            const int sm = S - 1 - (rank * SC + o);
-            const uint32_t am = slot_addr(sm / SL, sm % SL);
-            const float2 xk = spectral_product(xs[bc_pad(o)], slot_ld(am));
-            xs[bc_pad(o)] = xk;
-            slot_st(am, cconj(xk));
+            for (int i = 0; i < PER2; ++i) {
+                const int o = tid + i * T;
+                const float2 xk = spectral_product(xs[bc_pad(o)], xs[bc_pad(SC - 1 - o)]);
+                xs[bc_pad(o)] = xk;
+                xs[bc_pad(SC - 1 - o)] = cconj(xk);
+            }
+        } else {
+#pragma unroll 4
+            for (int i = 0; i < PER2; ++i) {
+                const int o = tid + i * T;
+                const int sm = S - 1 - (rank * SC + o);
+                const uint32_t am = slot_addr(sm / SL, sm % SL);
+                const float2 xk = spectral_product(xs[bc_pad(o)], slot_ld(am));
+                xs[bc_pad(o)] = xk;
+                slot_st(am, cconj(xk));
+            }
         }
     }
-    cluster_sync();
+    if constexpr (C::MIRROR)
+        __syncthreads();
+    else
+        cluster_sync();
 
     // ---- inverse local passes
     if constexpr (RC > 1) {
