@@ -74,6 +74,9 @@ def parse_args():
                     help="skip the per_config list (the other convolution workloads timed in the same run)")
     ap.add_argument("--per-config-steps", type=int, default=200,
                     help="timed steps of each per_config entry (graph-replayed)")
+    ap.add_argument("--probe", action="store_true",
+                    help="measure the per-SM rates behind the ALU rooflines (FFMA, FFMA2, IMAD, IMAD.HI, "
+                         "shared memory, distributed shared memory) and print them as one JSON line")
     return ap.parse_args()
 
 
@@ -324,17 +327,34 @@ def dominant_kernel(w: workloads.Workload, two_pass: bool) -> str:
     return "bigconv_kernel (two-pass step: 2 transposes in, 1 out)" if two_pass else "bigconv_kernel"
 
 
+def probe_rates():
+    """Measured lane operations per clock per SM of each pipe, from
+    profiles/probe_rates.txt (written from a `bench.py --probe` run), or {}."""
+    p = os.path.join(ROOT, "profiles", "probe_rates.txt")
+    rates = {}
+    if os.path.exists(p):
+        for line in open(p):
+            f = line.split()
+            if len(f) == 2 and not line.startswith("#"):
+                rates[f[0]] = float(f[1])
+    return rates
+
+
 def alu_roofline(alu_ops, alu_pipe, ms_per_step, clocks):
     """Executed lane operations of the kernel's busiest ALU pipe (ncu, same
-    sources) per launch against 148 SMs x lanes/clk of that pipe (FP32 128,
-    IMAD 64) x the SM clock sampled during the run."""
-    lanes = {"fp32": 128, "imad": 64}[alu_pipe]
+    sources) per launch against 148 SMs x the measured lanes/clk of that pipe
+    (bench.py --probe; nominal FP32 128, IMAD 64 when no probe is recorded) x
+    the SM clock sampled during the run."""
+    measured = probe_rates().get(alu_pipe)
+    lanes = measured if measured else {"fp32": 128, "imad": 64}[alu_pipe]
     sm_hz = clocks["sm_mhz"] * 1e6 if clocks and clocks.get("sm_mhz") else 1.965e9
     peak = 148 * lanes * sm_hz / 1e9
     achieved = alu_ops / (ms_per_step * 1e-3) / 1e9
+    src = (f"148 SMs x {lanes:g} lanes/clk measured by bench.py --probe x sampled SM clock" if measured
+           else f"148 SMs x {lanes} lanes/clk (nominal) x sampled SM clock")
     return {"bound": "alu", "pipe": alu_pipe, "achieved": achieved, "peak": peak,
             "unit": f"G {alu_pipe.upper()} lane-op/s", "frac": achieved / peak, "lane_ops_per_launch": alu_ops,
-            "peak_source": f"148 SMs x {lanes} lanes/clk x sampled SM clock"}
+            "peak_source": src}
 
 
 def time_config(w: workloads.Workload, rank, world, dev, pg, steps: int, warmup: int, cpu_budget_s: float):
@@ -1002,9 +1022,50 @@ def run_dwconv_reference(args, rank, world):
     }), flush=True)
 
 
+def run_probe(args, rank):
+    """Time the rate probes of libccprobe.so (one warm-up launch, one timed
+    launch each, CUDA events) with the SM clock sampled meanwhile, and report
+    each as a rate per SM per clock and per second on the whole GPU."""
+    import ctypes
+    import torch
+    if rank != 0:
+        return
+    from spectral_sequence_mixing_b200 import build as b
+    b.build()
+    lib = ctypes.CDLL(b.PROBE_LIB)
+    lib.ccp_run.restype = ctypes.c_int
+    lib.ccp_run.argtypes = [ctypes.c_int] * 4 + [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_double)]
+    torch.cuda.init()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    # (name, kind, blocks, threads, iters, unit)
+    probes = [("ffma", 0, 2 * sms, 1024, 100000, "lane-op"), ("ffma2", 1, 2 * sms, 1024, 100000, "lane-op"),
+              ("imad", 2, 2 * sms, 1024, 50000, "lane-op"), ("imad_hi", 3, 2 * sms, 1024, 50000, "lane-op"),
+              ("smem_read", 4, 2 * sms, 1024, 10000, "byte"), ("dsmem_store_8cta", 5, (sms // 8) * 8, 512, 1000, "byte")]
+    out = {}
+    with ClockSampler(0) as clk:
+        for name, kind, blocks, threads, iters, unit in probes:
+            ms, units = ctypes.c_float(0), ctypes.c_double(0)
+            st = lib.ccp_run(kind, blocks, threads, iters, ctypes.byref(ms), ctypes.byref(units))
+            if st != 0:
+                raise RuntimeError(f"probe {name}: CUDA error {st}")
+            out[name] = {"ms": ms.value, "units": units.value, "unit": unit,
+                         "sms_used": min(sms, blocks) if kind != 5 else blocks}
+    clocks = clk.report()
+    mhz = clocks["sm_mhz"] if clocks and clocks.get("sm_mhz") else 1965.0
+    for name, r in out.items():
+        per_s = r["units"] / (r["ms"] * 1e-3)
+        r["per_s_gpu"] = per_s
+        r["per_clk_per_sm"] = per_s / r["sms_used"] / (mhz * 1e6)
+    print(json.dumps({"probe": out, "sm_count": sms, "clocks": clocks,
+                      "note": "per_clk_per_sm at the median sampled SM clock"}), flush=True)
+
+
 def main():
     args = parse_args()
     rank, world, local = dist_env()
+    if args.probe:
+        run_probe(args, rank)
+        return
     if world != args.gpus and "RANK" in os.environ:
         print(f"warning: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
     gated = args.workload in workloads.GATE_WORKLOADS

@@ -18,6 +18,9 @@ LIB = os.path.join(PKG, "libcausalconv.so")
 SOURCES = [os.path.join(CSRC, "api.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
     os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
+# rate probes for the benchmark's --probe mode (not part of the C-ABI library)
+PROBE_LIB = os.path.join(PKG, "libccprobe.so")
+PROBE_SOURCES = [os.path.join(CSRC, "probe.cu")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -34,22 +37,27 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def needs_rebuild() -> bool:
-    if not os.path.exists(LIB):
+def needs_rebuild(lib: str = LIB, deps=DEPS) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
-    return any(os.path.getmtime(p) > t for p in DEPS)
+    t = os.path.getmtime(lib)
+    return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
-    if not force and not needs_rebuild():
-        return LIB
+def _nvcc(lib: str, sources, verbose: bool, extra_flags) -> None:
     cmd = [nvcc_path(), *NVCC_FLAGS, *(extra_flags or []), "-I", INCLUDE, "-I", CSRC, "-shared",
-           "-o", LIB + ".tmp", *SOURCES]
+           "-o", lib + ".tmp", *sources]
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(lib + ".tmp", lib)
+
+
+def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
+    if force or needs_rebuild(PROBE_LIB, PROBE_SOURCES):
+        _nvcc(PROBE_LIB, PROBE_SOURCES, verbose, extra_flags)
+    if force or needs_rebuild():
+        _nvcc(LIB, SOURCES, verbose, extra_flags)
     return LIB
 
 
