@@ -99,12 +99,13 @@ constexpr unsigned kTcOffOut = kTcOffIn + kTcInBytes;     // outputs of this CTA
 constexpr unsigned kTcOffHead = kTcOffOut + kTcGroup * kTcSpan * 2;  // [2 rows][v, g][64] fp32
 constexpr unsigned kTcOffRed = kTcOffHead + kTcRows * 2 * kTcHead * 4;  // [16] CTA sums, [16] scales
 constexpr unsigned kTcOffBar = kTcOffRed + (16 + 16) * 4;
-constexpr unsigned kTcSmemBytes = kTcOffBar + 32 + 128;  // + 3 barriers, TMEM slot, alignment slack
+constexpr unsigned kTcSmemBytes = kTcOffBar + 40 + 128;  // + 3 barriers, TMEM slot, 2 counters, alignment slack
 constexpr int kTcBoxT = 256;                             // TMA box: [kTcBoxT t][8 ch]
 constexpr unsigned kTcTmemCols = 256;                    // one 128-column accumulator per row
 constexpr float kTcOutScale = 8.0f;  // 1 / (4 N) times the inverse of the stage scales (1/64)^2 (1/64)
 constexpr unsigned kFaultTcWait = 4u;
 static_assert(kTcSmemBytes <= 232448, "shared memory");
+static_assert(((kTcThreads / 32) & (kTcThreads / 32 - 1)) == 0, "the MMA issue counter counts warps in powers of two");
 
 // Stage matrices and twiddle tables in their shared-memory byte layout;
 // filled once per device from fp64 values.
@@ -208,6 +209,7 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
     uint16_t *outs = reinterpret_cast<uint16_t *>(sm + kTcOffOut);  // [8 channels][1024 slots]
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kTcOffBar);   // one per row, then the input barrier
     unsigned *tslot = reinterpret_cast<unsigned *>(sm + kTcOffBar + 24);
+    unsigned *icnt = reinterpret_cast<unsigned *>(sm + kTcOffBar + 32);  // per row: warps done with its operand
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = (int)cluster.block_rank();  // this CTA: channels 2q, 2q+1 of the group; time steps [1024 q, +1024)
@@ -218,6 +220,8 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
         mbar_init(bar, 1);
         mbar_init(bar + 1, 1);
         mbar_init(bar + 2, 1);
+        icnt[0] = 0u;
+        icnt[1] = 0u;
     }
     // TMA: this CTA's time steps of group gi (v reversed in time when rev & 1:
     // its staged rows then run backwards), completing on bar[2]
@@ -317,35 +321,55 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
         }
     };
 
-    // stage s (1..4) of row x: 4 or 8 MMAs of K = 16 (two 16-byte chunks each), one thread issues
+    // stage s (1..4) of row x: 4 or 8 MMAs of K = 16 (two 16-byte chunks each).
+    // No CTA barrier: each warp, once its part of the operand is written and
+    // its accumulator reads are done, counts itself on icnt[x] (acquire-
+    // release); the last of the 16 warps issues the MMAs and the commit, so
+    // no thread waits here.  The counter only grows (a multiple of 16 marks
+    // the last arrival), so it needs no reset.  If the issuing thread's
+    // earlier waits ran out it completes bar[x] itself instead, so that no
+    // thread waits for a commit that will not come; the failure reaches
+    // every thread at the end of the group.
     auto issue = [&](int s, int x) {
         fence_proxy_async_smem();
         tc_fence_before_sync();
-        __syncthreads();
-        tc_fence_after_sync();
-        if (!ok) return;  // a completion wait ran out: issue nothing more (uniform over the CTA)
-        if (tid == 0) {
-            const unsigned data = kTcOffData + (unsigned)x * 32768u;
-            const unsigned a_off = s == 1 ? kTcOffA1 : (s == 4 ? kTcOffA4 : data);
-            const unsigned b_off = (s == 1 || s == 4) ? data : kTcOffB2;
-            const int nk = s == 1 ? 4 : 8;
-            const bool b_mn = s == 4;
-            const uint32_t idesc = tc_idesc(b_mn);
-            for (int k = 0; k < nk; ++k) {
-                const uint64_t ad = umma_smem_desc(sb + a_off + 2u * k * kTcChunkPitch, kTcChunkPitch, 128u);
-                const uint64_t bd = b_mn ? umma_smem_desc(sb + b_off + 2u * k * 2048u, 2048u, 128u)
-                                         : umma_smem_desc(sb + b_off + 2u * k * kTcChunkPitch, kTcChunkPitch, 128u);
-                umma_f16(tmem + 128u * x, ad, bd, idesc, k > 0);
-            }
-            umma_commit(bar + x);
-        }
         pending |= 1u << x;
+        __syncwarp();
+        if (lane == 0) {
+            unsigned n;
+            asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;"
+                         : "=r"(n)
+                         : "r"(smem_u32(icnt + x))
+                         : "memory");
+            if (((n + 1u) & (kTcThreads / 32 - 1)) == 0u) {
+                if (!ok) {
+                    mbar_arrive(bar + x);
+                    return;
+                }
+                tc_fence_after_sync();
+                const unsigned data = kTcOffData + (unsigned)x * 32768u;
+                const unsigned a_off = s == 1 ? kTcOffA1 : (s == 4 ? kTcOffA4 : data);
+                const unsigned b_off = (s == 1 || s == 4) ? data : kTcOffB2;
+                const int nk = s == 1 ? 4 : 8;
+                const bool b_mn = s == 4;
+                const uint32_t idesc = tc_idesc(b_mn);
+                for (int k = 0; k < nk; ++k) {
+                    const uint64_t ad = umma_smem_desc(sb + a_off + 2u * k * kTcChunkPitch, kTcChunkPitch, 128u);
+                    const uint64_t bd = b_mn ? umma_smem_desc(sb + b_off + 2u * k * 2048u, 2048u, 128u)
+                                             : umma_smem_desc(sb + b_off + 2u * k * kTcChunkPitch, kTcChunkPitch, 128u);
+                    umma_f16(tmem + 128u * x, ad, bd, idesc, k > 0);
+                }
+                umma_commit(bar + x);
+            }
+        }
     };
+    // Every thread observes the completion itself (no CTA barrier): the
+    // next commit to the same barrier comes only after every warp has
+    // counted itself in the next issue(), which each thread reaches after
+    // this wait.
     auto wait = [&](int x) {
-        bool done = true;
-        if (((pending >> x) & 1u) && tid == 0) done = mbar_wait_bounded(bar + x, (phase >> x) & 1u);
-        done = __syncthreads_and(done);
         if ((pending >> x) & 1u) {
+            const bool done = mbar_wait_bounded(bar + x, (phase >> x) & 1u);
             if (done) {
                 phase ^= 1u << x;
                 pending &= ~(1u << x);
@@ -593,6 +617,7 @@ __global__ void __cluster_dims__(kTcCluster, 1, 1) __launch_bounds__(kTcThreads,
                 if (s < 4) issue(s + 1, x);
             }
         }
+        ok = __syncthreads_and(ok);  // the last two waits had no issue() after them
         // the next group's partial norms, from its staged input (the head buffer is free now)
         have_norms = false;
         if (use_tma && in_flight && ok) {
