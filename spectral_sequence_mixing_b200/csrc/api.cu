@@ -83,6 +83,19 @@ static std::vector<float2> big_twiddles() {
     }
     for (int k = 0; k < RB; ++k)
         for (int lo = 0; lo < RC; ++lo) t[Cfg::TB + k * RC + lo] = omega((int64_t)lo * k, RB * RC);
+    if constexpr (Cfg::MIRROR) {
+        // half-length real-output inverse, see BigCfg
+        constexpr int RCH = Cfg::RCH, STAH = Cfg::STAH;
+        for (int ka = 0; ka < RA; ++ka) t[Cfg::TPA + ka] = omega(ka, SL);
+        for (int j = 0; j < STAH; ++j) t[Cfg::TPB + j] = omega(j, SL / RA);
+        for (int k = 0; k < RB; ++k)
+            for (int lo = 0; lo < RCH; ++lo) t[Cfg::TBH + k * RCH + lo] = omega((int64_t)lo * k, RB * RCH);
+        for (int k = 0; k < RA; ++k) {
+            for (int ll = 0; ll < QA; ++ll) t[Cfg::TAHA + k * QA + ll] = omega((int64_t)ll * k, SL / 2);
+            for (int lh = 0; lh < STAH / QA; ++lh)
+                t[Cfg::TAHB + k * (STAH / QA) + lh] = omega((int64_t)QA * lh * k, SL / 2);
+        }
+    }
     return t;
 }
 

@@ -71,12 +71,28 @@ struct BigCfg {
     static constexpr int TAA = T0B + R0 * (SL / Q0);
     static constexpr int TAB = TAA + RA * QA;
     static constexpr int TB = TAB + RA * (STA / QA);
-    static constexpr int TW_SIZE = TB + RB * RC;
+    // Real-output inverse (mirror pairs only; see bigconv_kernel): a transform
+    // of half the length, M = S / 2, whose innermost digit has RC / 2 values.
+    //   packing: theta^(2 R0 k'') = omega_SL^k'', k'' = kA + RA j (j < RB RC / 2)
+    //            = TPA[kA] * TPB[j]          (omega_SL^kA, omega_(SL / RA)^j)
+    //   pass B:  omega_(RB RC/2)^(lo k) = TBH[k][lo], lo < RC / 2
+    //   pass A:  omega_(SL/2)^(lo k), lo = lh QA + ll < RB RC / 2
+    //            = TAHA[k][ll] * TAHB[k][lh]
+    static constexpr int RCH = RC / 2;
+    static constexpr int STAH = RB * RCH;  // logical stride of the half-length pass A
+    static constexpr int TPA = TB + RB * RC;
+    static constexpr int TPB = TPA + RA;
+    static constexpr int TBH = TPB + STAH;
+    static constexpr int TAHA = TBH + RB * RCH;
+    static constexpr int TAHB = TAHA + RA * QA;
+    static constexpr int TW_SIZE = MIRROR ? TAHB + RA * (STAH / QA) : TB + RB * RC;
     static constexpr int LAST_R = RC > 1 ? RC : RB;
     static_assert(CL == 1 || CL == R0 || 2 * CL == R0, "a cluster splits the most significant digit");
     static_assert(LAST_R == 16, "innermost radix must be 16 (conflict-free padded layout)");
     static_assert(R0 <= 64 && RA <= 32 && RB <= 32 && RC <= 32, "register DFT sizes");
     static_assert(SC % (2 * T) == 0 && COLS0 % T == 0, "pass work split");
+    static_assert(!MIRROR || (R0 == 16 && RA == 32 && RB == 16 && RC == 16 && CL == 8 && T == 512),
+                  "the real-output inverse is written for the 16 x 32 x 16 x 16 cluster rows");
 };
 
 __device__ __forceinline__ int bc_pad(int p) { return p + (p >> 4); }
@@ -302,6 +318,116 @@ __global__ void __launch_bounds__(T, MINB)
     else
         cluster_sync();
 
+    // ---- real-output inverse (mirror pairs).  r is real, so the S-point
+    // inverse y_n = sum_k X_k theta^(-n (2k+1)) is taken as one M = S/2-point
+    // odd-frequency inverse whose outputs are w_m = y_2m + i y_2m+1:
+    //   C_k = E_k + i O_k,  E_k = X_k + X_(k+M),  O_k = (X_k - X_(k+M)) theta^-(2k+1),
+    //   w_m = sum_(k<M) C_k phi^(m (2k+1)),  phi = theta^-2
+    // (bin k + M is the same slot with the innermost digit kC + RC/2, so the
+    // packing stays in the CTA; it runs with the spectral product, below, and
+    // leaves C_k in the slots with kC < RC/2).  With k = k0 + R0 k'' and m = m0 (SL/2) + m',
+    // the M-point inverse splits like the S-point one: for each k0 an
+    // (SL/2)-point inverse DFT over k'' (passes over kC < RC/2, kB, kA in
+    // the slots' lower halves), then across the cluster the twiddle
+    // conj(theta^(2m' (2 k0 + 1))), the inverse R0-point DFT over k0
+    // (outputs m0 < R0/2) and the untwist.  Half the work and half the
+    // distributed-shared-memory reads of the S-point inverse.
+    auto inverse_real_output = [&]() {
+        constexpr int RCH = C::RCH, STAH = C::STAH;
+        constexpr int PSTB = RC + RC / 16, PSTA = RB * RC + (RB * RC) / 16;
+        // innermost digit kC < RCH (slot stride 1): inverse RCH-point DFT, no twiddle
+#pragma unroll 1
+        for (int q = tid; q < SC / RC; q += T) {
+            float2 *xp = xs + bc_pad(q * RC);
+            float2 x[RCH];
+#pragma unroll
+            for (int k = 0; k < RCH; ++k) x[bitrev(k, ilog2(RCH))] = xp[k];
+            fft_dit<RCH, true>(x);
+#pragma unroll
+            for (int j = 0; j < RCH; ++j) xp[j] = x[j];
+        }
+        __syncthreads();
+        // digit kB (slot stride RC), lo = the kC digit's output (< RCH):
+        // twiddle conj(omega_(RB RCH)^(lo kB)), inverse RB-point DFT
+#pragma unroll 1
+        for (int q = tid; q < 2 * RA * RCH; q += T) {
+            const int lk = q / (RA * RCH), w = q - lk * (RA * RCH), ka = w / RCH, lo = w - ka * RCH;
+            float2 *xp = xs + bc_pad(lk * SL + ka * (RB * RC) + lo);
+            float2 x[RB];
+#pragma unroll
+            for (int k = 0; k < RB; ++k) {
+                float2 y = xp[k * PSTB];
+                if (k > 0) y = cmul_conj(y, __ldg(tw + C::TBH + k * RCH + lo));
+                x[bitrev(k, ilog2(RB))] = y;
+            }
+            fft_dit<RB, true>(x);
+#pragma unroll
+            for (int j = 0; j < RB; ++j) xp[j * PSTB] = x[j];
+        }
+        __syncthreads();
+        // digit kA (slot stride RB RC), logical lo = (kB output) RCH + (kC output) < STAH:
+        // twiddle conj(omega_(SL/2)^(lo kA)), inverse RA-point DFT
+#pragma unroll 1
+        for (int q = tid; q < 2 * STAH; q += T) {
+            const int lk = q / STAH, lol = q - lk * STAH;
+            float2 *xp = xs + bc_pad(lk * SL + (lol / RCH) * RC + lol % RCH);
+            float2 x[RA];
+#pragma unroll
+            for (int k = 0; k < RA; ++k) {
+                float2 y = xp[k * PSTA];
+                if (k > 0)
+                    y = cmul_conj(y, cmul(__ldg(tw + C::TAHA + k * C::QA + lol % C::QA),
+                                          __ldg(tw + C::TAHB + k * (STAH / C::QA) + lol / C::QA)));
+                x[bitrev(k, ilog2(RA))] = y;
+            }
+            fft_dit<RA, true>(x);
+#pragma unroll
+            for (int j = 0; j < RA; ++j) xp[j * PSTA] = x[j];
+        }
+        // the direct sums r_t, t < HEAD (time steps of CTA 0's first columns),
+        // into the norm-partials area, which is free by now
+        float *hsum = reinterpret_cast<float *>(head + HEAD);
+        static_assert(2 * (T / 32 + 1) >= HEAD, "head sums fit the norm-partials area");
+        if (rank == 0 && tid < HEAD) {
+            float a = 0.f;
+            for (int j = 0; j <= tid; ++j) a = fmaf(head[j].x, head[tid - j].y, a);
+            hsum[tid] = a;
+        }
+        cluster_sync();
+        // across the cluster: column m' of both k0 halves of every CTA, twiddle,
+        // inverse R0-point DFT over k0 (outputs m0 < R0/2), untwist; w_m gives
+        // r_(2m) and r_(2m+1), m = m0 (SL/2) + m'
+        {
+            const float s = live ? 1.f / (4.f * (float)S * alpha) : 0.f;
+            constexpr int COLSH = SL / 2 / CL;  // columns m' per CTA
+#pragma unroll 1
+            for (int c = tid; c < COLSH; c += T) {
+                const int mp = rank * COLSH + c;
+                // m' = a (RB RCH) + b RCH + e sits at slot a (RB RC) + b RC + e
+                const int phys = (mp / (RB * RCH)) * (RB * RC) + ((mp / RCH) % RB) * RC + mp % RCH;
+                float2 x[R0];
+#pragma unroll
+                for (int k0 = 0; k0 < R0; ++k0)
+                    x[bitrev(k0, LOG_R0)] = cmul_conj(slot_ld(slot_addr(k0, phys)), tw0(k0, 2 * mp));
+                fft_dit<R0, true, false, true>(x);
+#pragma unroll
+                for (int m0 = 0; m0 < R0 / 2; ++m0) {
+                    const int t = 2 * (m0 * (SL / 2) + mp);
+                    if (t >= L) continue;
+                    // untwist conj(omega_2R0^m0)
+                    const float2 z = m0 == 0 ? x[0] : cmul_conj(x[m0], tw_const(m0, 2 * R0));
+                    float o0 = z.x * s, o1 = z.y * s;
+                    if (t < HEAD) {  // HEAD is even, so t + 1 < HEAD too
+                        o0 = hsum[t];
+                        o1 = hsum[t + 1];
+                    }
+                    IO_t<IO>::st(r + base + (int64_t)((rev & 2) ? L - 1 - t : t) * tstep, o0);
+                    if (t + 1 < L) IO_t<IO>::st(r + base + (int64_t)((rev & 2) ? L - 2 - t : t + 1) * tstep, o1);
+                }
+            }
+        }
+    };
+
     // ---- spectral product X' = 4 V G.  The pair (s, S-1-s) is handled by the
     // thread that owns s at local offset o < SC/2 (the mirror then sits at a
     // local offset >= SC/2: SC-1-o in this CTA with mirror pairs, else in CTA
@@ -310,12 +436,32 @@ __global__ void __launch_bounds__(T, MINB)
     {
         constexpr int PER2 = SC / (2 * T);
         if constexpr (C::MIRROR) {
-#pragma unroll 4
-            for (int i = 0; i < PER2; ++i) {
-                const int o = tid + i * T;
-                const float2 xk = spectral_product(xs[bc_pad(o)], xs[bc_pad(SC - 1 - o)]);
-                xs[bc_pad(o)] = xk;
-                xs[bc_pad(SC - 1 - o)] = cconj(xk);
+            // With the real-output packing: a thread takes o (k0 = rank, kC < RC/2),
+            // o + RC/2 (bin k + M), and their mirrors SC-1-o and p = SC-1-o-RC/2
+            // (k0 = R0-1-rank; p's innermost digit is RC/2-1-kC, and p + RC/2 is
+            // SC-1-o): two spectral products give all four X', then
+            // C_o = pack(X'_o, X'_(o+RC/2)) and C_p = pack(X'_p, X'_(p+RC/2)).
+            constexpr int RCH = C::RCH;
+            // theta^(2 k0 + 1) for this CTA's two k0 (rank, R0-1-rank)
+            const float2 tk0 = __ldg(tw + C::T0A + rank * C::Q0 + 1);
+            const float2 tk1 = __ldg(tw + C::T0A + (R0 - 1 - rank) * C::Q0 + 1);
+            // C = E + i O, E = a + b, O = (a - b) conj(w), w = theta^(2k+1)
+            auto pack = [](float2 a, float2 b, float2 w) -> float2 {
+                const float2 ov = cmul_conj(csub(a, b), w), ev = cadd(a, b);
+                return make_float2(ev.x - ov.y, ev.y + ov.x);
+            };
+#pragma unroll 2
+            for (int i = tid; i < SC / 4; i += T) {
+                const int kc = i % RCH, kb = (i / RCH) % RB, ka = i / (RCH * RB);
+                const int o = ka * (RB * RC) + kb * RC + kc, p = SC - 1 - o - RCH;
+                const float2 xo = spectral_product(xs[bc_pad(o)], xs[bc_pad(SC - 1 - o)]);
+                const float2 xo8 = spectral_product(xs[bc_pad(o + RCH)], xs[bc_pad(p)]);
+                // theta^(2k+1) = theta^(2 k0 + 1) omega_SL^k'', k'' = kA + RA (kB + RB kC)
+                const float2 wo = cmul(cmul(tk0, __ldg(tw + C::TPA + ka)), __ldg(tw + C::TPB + kb + RB * kc));
+                const float2 wp = cmul(cmul(tk1, __ldg(tw + C::TPA + RA - 1 - ka)),
+                                       __ldg(tw + C::TPB + (RB - 1 - kb) + RB * (RCH - 1 - kc)));
+                xs[bc_pad(o)] = pack(xo, xo8, wo);
+                xs[bc_pad(p)] = pack(cconj(xo8), cconj(xo), wp);
             }
         } else {
 #pragma unroll 4
@@ -334,43 +480,47 @@ __global__ void __launch_bounds__(T, MINB)
     else
         cluster_sync();
 
-    // ---- inverse local passes
-    if constexpr (RC > 1) {
-        bc_local_pass<RC, 1, 1, SL, SC, T, true>(xs, tw, tw);
-        __syncthreads();
-        bc_local_pass<RB, RC, RC, SL, SC, T, true>(xs, tw + C::TB, tw + C::TB);
+    if constexpr (C::MIRROR) {
+        inverse_real_output();
     } else {
-        bc_local_pass<RB, 1, 1, SL, SC, T, true>(xs, tw, tw);
-    }
-    __syncthreads();
-    bc_local_pass<RA, C::STA, C::QA, SL, SC, T, true>(xs, tw + C::TAA, tw + C::TAB);
-    cluster_sync();
+        // ---- inverse local passes
+        if constexpr (RC > 1) {
+            bc_local_pass<RC, 1, 1, SL, SC, T, true>(xs, tw, tw);
+            __syncthreads();
+            bc_local_pass<RB, RC, RC, SL, SC, T, true>(xs, tw + C::TB, tw + C::TB);
+        } else {
+            bc_local_pass<RB, 1, 1, SL, SC, T, true>(xs, tw, tw);
+        }
+        __syncthreads();
+        bc_local_pass<RA, C::STA, C::QA, SL, SC, T, true>(xs, tw + C::TAA, tw + C::TAB);
+        cluster_sync();
 
-    // ---- inverse pass 0: twiddle, inverse R0-point DFT (outputs n0 < R0/2), untwist, store t < L
-    {
-        const float s = live ? 1.f / (4.f * (float)S * alpha) : 0.f;
-#pragma unroll 1
-        for (int c = tid; c < C::COLS0; c += T) {
-            const int n = rank * C::COLS0 + c;
-            float2 x[R0];
-#pragma unroll
-            for (int k0 = 0; k0 < R0; ++k0) {
-                x[bitrev(k0, LOG_R0)] = cmul_conj(slot_ld(slot_addr(k0, n)), tw0(k0, n));
-            }
-            fft_dit<R0, true, false, true>(x);
-#pragma unroll
-            for (int n0 = 0; n0 < R0 / 2; ++n0) {
-                const int t = n0 * SL + n;
-                if (t >= L) continue;
-                // untwist omega_2R0^-n0; only the real part is the output
-                const float2 w = tw_const(n0, 2 * R0);
-                float out = (n0 == 0 ? x[0].x : fmaf(x[n0].x, w.x, x[n0].y * w.y)) * s;
-                if (t < HEAD) {
-                    float a = 0.f;
-                    for (int j = 0; j <= t; ++j) a = fmaf(head[j].x, head[t - j].y, a);
-                    out = a;
+        // ---- inverse pass 0: twiddle, inverse R0-point DFT (outputs n0 < R0/2), untwist, store t < L
+        {
+            const float s = live ? 1.f / (4.f * (float)S * alpha) : 0.f;
+    #pragma unroll 1
+            for (int c = tid; c < C::COLS0; c += T) {
+                const int n = rank * C::COLS0 + c;
+                float2 x[R0];
+    #pragma unroll
+                for (int k0 = 0; k0 < R0; ++k0) {
+                    x[bitrev(k0, LOG_R0)] = cmul_conj(slot_ld(slot_addr(k0, n)), tw0(k0, n));
                 }
-                IO_t<IO>::st(r + base + (int64_t)((rev & 2) ? L - 1 - t : t) * tstep, out);
+                fft_dit<R0, true, false, true>(x);
+    #pragma unroll
+                for (int n0 = 0; n0 < R0 / 2; ++n0) {
+                    const int t = n0 * SL + n;
+                    if (t >= L) continue;
+                    // untwist omega_2R0^-n0; only the real part is the output
+                    const float2 w = tw_const(n0, 2 * R0);
+                    float out = (n0 == 0 ? x[0].x : fmaf(x[n0].x, w.x, x[n0].y * w.y)) * s;
+                    if (t < HEAD) {
+                        float a = 0.f;
+                        for (int j = 0; j <= t; ++j) a = fmaf(head[j].x, head[t - j].y, a);
+                        out = a;
+                    }
+                    IO_t<IO>::st(r + base + (int64_t)((rev & 2) ? L - 1 - t : t) * tstep, out);
+                }
             }
         }
     }
