@@ -430,6 +430,33 @@ def test_bwd_sampled_oracle(shape):
         assert n_bad == 0, f"{name}: {n_bad} violations, worst ratio {worst:.3g}"
 
 
+@pytest.mark.parametrize("two_pass", [True, False], ids=["two_pass", "single_pass"])
+@pytest.mark.parametrize("shape", [(1, 4099, 3), (2, 9001, 2)], ids=lambda s: "x".join(map(str, s)))
+def test_bwd_cluster_rows_odd_length(shape, two_pass):
+    """Backward on cluster rows (v read and r written reversed in time) with an
+    odd length, so the last output pair of the real-output inverse is cut in
+    half; with and without the transposing workspace."""
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    B, L, D = shape
+    rng = np.random.Generator(np.random.PCG64(500 + L))
+    dr, v, g = (rng.standard_normal(shape).astype(np.float32) for _ in range(3))
+    n_ws = ssm.fast_workspace_bytes(torch.float32, B, L, D) if two_pass else 0
+    ws = torch.empty(n_ws, dtype=torch.uint8, device="cuda")
+    dv, dg = ssm.causal_conv_bwd(to_dev(dr, "f32"), to_dev(v, "f32"), to_dev(g, "f32"), workspace=ws)
+    torch.cuda.synchronize()
+    dv, dg = from_dev(dv, "f32"), from_dev(dg, "f32")
+    pts = workloads.sample_points(B, L, D, 1024, seed=9)
+    # the first and last time steps of every row, where the reversal and the cut pair meet
+    ends = np.array([[b, t, d] for b in range(B) for d in range(D) for t in (0, 1, L - 2, L - 1)], dtype=pts.dtype)
+    pts = np.concatenate([pts, ends])
+    ref_dv, den_dv, ref_dg, den_dg = oracle.causal_conv_bwd_points(dr, v, g, pts)
+    ix = (pts[:, 0], pts[:, 1], pts[:, 2])
+    for name, got, ref, den in (("dv", dv[ix], ref_dv, den_dv), ("dg", dg[ix], ref_dg, den_dg)):
+        n_bad, worst = float_violations(got, ref, den, F32_TOL)
+        assert n_bad == 0, f"{name}: {n_bad} violations, worst ratio {worst:.3g}"
+
+
 def test_bwd_consistent_with_forward_adjoint():
     """<dr, r(v, g)> = <dv, v> = <dg, g> with the GPU forward and backward."""
     import spectral_sequence_mixing_b200 as ssm
