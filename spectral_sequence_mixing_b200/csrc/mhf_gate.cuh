@@ -27,11 +27,12 @@
 //
 // Schedule: a persistent CTA per (head, group of tiles); the head's weights
 // are split and staged in shared memory once.  Then the warps take roles:
-// eight producer warps store sigmoid(a) (hi, lo) of 128-step tiles into a
-// ring of tile buffers, one warp issues each tile's 3 K C/8 MMAs (one lane,
-// elect.sync) into a ring of TMEM accumulators, and four warps read each
-// accumulator back (warp w: TMEM lanes 32 w .. +31 = time steps, all C
-// columns), add the bias and store g.  Buffers and accumulators pass between
+// seven producer warps store sigmoid(a) (hi, lo) of 128-step tiles into a
+// ring of tile buffers (the fp32 input tile arrives by TMA when the tensor
+// allows a tensor map), one warp issues each tile's 3 K C/16 MMAs (one lane,
+// elect.sync) into a ring of TMEM accumulators, and eight warps read each
+// accumulator back (two per TMEM lane quarter: lanes 32 (w % 4) .. +31 =
+// time steps, half of the C columns each), add the bias and store g.  Buffers and accumulators pass between
 // the roles on mbarriers (tcgen05.commit frees a tile buffer and publishes
 // its accumulator), so the tensor core, the sigmoid and the stores of
 // different tiles overlap with no CTA-wide barrier.  Every wait is bounded;
@@ -303,8 +304,20 @@ __global__ void __launch_bounds__(kGateThreads, 1)
             }
             for (int tile = first; tile < num_tiles; tile += groups, ++it) {
                 const int buf = it % NB;
-                // every producer agrees on whether the input arrived in time
+                // every producer agrees on whether the input arrived in time; past this
+                // barrier no producer reads the previous tile's input tile any more
                 if (!bar_and(1, kGateProdThreads, mbar_wait_bounded(loaded + buf, (it / NB) & 1u))) {
+                    ok = false;
+                    break;
+                }
+                // the next tile's input into the other input tile, while this one is converted
+                const int nt = tile + groups;
+                if (pt == 0 && nt < num_tiles) {
+                    fetch(nt, (it + 1) % NB);
+                    fetched = it + 1;
+                }
+                // the sigmoid buffer is free once the MMAs of the tile NB back are done
+                if (it >= NB && !bar_and(1, kGateProdThreads, mbar_wait_bounded(empty + buf, (it / NB - 1) & 1u))) {
                     ok = false;
                     break;
                 }
@@ -317,17 +330,6 @@ __global__ void __launch_bounds__(kGateThreads, 1)
                     put(buf, t0, j, *reinterpret_cast<const float4 *>(raw + (i / Cfg::C4) * (C * 4) + (i % Cfg::C4) * 16));
                 }
                 publish(buf);
-                // the next tile's input, once its buffer's previous MMAs are done (which also
-                // means every producer has read that buffer's input tile)
-                const int nt = tile + groups, nbuf = (it + 1) % NB;
-                if (pt == 0 && nt < num_tiles) {
-                    if (it + 1 >= NB && !mbar_wait_bounded(empty + nbuf, ((it + 1) / NB - 1) & 1u)) {
-                        ok = false;  // nothing more is requested; the others time out on loaded
-                    } else {
-                        fetch(nt, nbuf);
-                        fetched = it + 1;
-                    }
-                }
             }
             // a request still in flight lands before the CTA's shared memory is released
             if (pt == 0 && fetched >= it && fetched >= 0) mbar_wait_bounded(loaded + fetched % NB, (fetched / NB) & 1u);
