@@ -72,7 +72,14 @@ struct GateCfg {
     static constexpr unsigned OFF_RAW = NBUF * 2 * A_BYTES;
     static constexpr unsigned OFF_WHI = OFF_RAW + NBUF * RAW_BYTES, OFF_WLO = OFF_WHI + W_BYTES;
     static constexpr unsigned OFF_BIAS = OFF_WLO + W_BYTES;
-    static constexpr unsigned OFF_BAR = (OFF_BIAS + C * 4u + 15u) & ~15u;  // 5 NBUF mbarriers, then the TMEM slot
+    // output staging [kGateM t][OUT_PITCH] fp32 (rows 16 bytes longer than C channels,
+    // so one thread per row writes and a warp per row pair reads without bank conflicts),
+    // where it fits (not for four taps of 64 channels)
+    static constexpr unsigned OUT_PITCH = C + 4;
+    static constexpr unsigned OFF_OUT = (OFF_BIAS + C * 4u + 15u) & ~15u;
+    static constexpr unsigned OUT_BYTES = kGateM * OUT_PITCH * 4u;
+    static constexpr bool STAGE_OUT = OFF_OUT + OUT_BYTES + 96u + 128u <= 232448u;
+    static constexpr unsigned OFF_BAR = STAGE_OUT ? OFF_OUT + OUT_BYTES : OFF_OUT;  // 5 NBUF mbarriers, then the TMEM slot
     static constexpr unsigned SMEM_BYTES = OFF_BAR + 96u + 128u;           // + alignment slack
     static_assert(SMEM_BYTES <= 232448, "shared memory");
     // one fp32 accumulator of C columns per buffer, in a power-of-two allocation >= 32
@@ -176,14 +183,16 @@ __device__ __forceinline__ void store4(__nv_bfloat16 *p, const float (&v)[4], bo
     }
 }
 
-// Warp roles (sixteen warps): warps 0-7 drain the accumulators (warp w
-// reads TMEM lanes 32 (w % 4) .. +31, i.e. time steps, and the column half
-// w / 4), warp 8 issues the MMAs (one lane, elect.sync), warps 9-15 stage
-// sigmoid tiles.  Tiles and accumulators (NBUF of each) are handed over on
+// Warp roles (sixteen warps): warps 0-3 drain the accumulators (warp w
+// reads TMEM lanes 32 w .. +31, i.e. time steps, and all the columns,
+// stages its rows with the bias and then the four warps store the tile in
+// whole rows), warp 4 issues the MMAs (one lane, elect.sync), warps 5-15
+// stage sigmoid tiles (the conversion is the slowest role, so it gets the
+// most warps).  Tiles and accumulators (NBUF of each) are handed over on
 // mbarriers -- full / empty for the sigmoid tiles, acc_full / acc_empty for
 // the accumulators -- so no role waits at a CTA-wide barrier in the steady
 // state.
-constexpr int kGateEpiWarps = 8, kGateMmaWarp = 8, kGateProdWarp0 = 9;
+constexpr int kGateEpiWarps = 4, kGateMmaWarp = 4, kGateProdWarp0 = 5;
 constexpr int kGateProdThreads = kGateThreads - 32 * kGateProdWarp0;
 
 // grid = H * groups CTAs; CTA (h = blockIdx.x % H, j = blockIdx.x / H) takes
@@ -411,20 +420,37 @@ __global__ void __launch_bounds__(kGateThreads, 1)
         }
     } else if (warp < kGateEpiWarps) {
         // ---- epilogue: accumulator rows 32 warp + lane (time steps), all C columns, + bias, store
+        float *stg = reinterpret_cast<float *>(sm + Cfg::OFF_OUT);
+        constexpr int EPT = 32 * kGateEpiWarps;  // epilogue threads
         int it = 0;
         for (int tile = first; tile < num_tiles; tile += groups, ++it) {
             const int buf = it % NB;
-            const bool got = mbar_wait_bounded(acc_full + buf, (it / NB) & 1u);
-            if (!__all_sync(0xffffffffu, got)) {
+            // the epilogue warps agree on whether the accumulator arrived (with the
+            // staging this is also their barrier: the previous tile's rows are read back)
+            bool got = mbar_wait_bounded(acc_full + buf, (it / NB) & 1u);
+            if constexpr (Cfg::STAGE_OUT)
+                got = bar_and(2, EPT, got);
+            else
+                got = __all_sync(0xffffffffu, got);
+            if (!got) {
                 ok = false;
                 break;
             }
             tc_fence_after_sync();
-            constexpr int CH = C / 2;  // this warp's columns: [CH (warp / 4), +CH)
-            const int cb = CH * (warp >> 2);
-            float v[CH];
-            const unsigned trow = tmem + buf * C + cb + ((unsigned)(32 * (warp & 3)) << 16);
-            if constexpr (CH == 32) {
+            float v[C];
+            const unsigned trow = tmem + buf * C + ((unsigned)(32 * warp) << 16);
+            if constexpr (C == 64) {
+                float x0[16], x1[16], x2[16], x3[16];
+                tmem_ld16x2(trow, trow + 16, x0, x1);
+                tmem_ld16x2(trow + 32, trow + 48, x2, x3);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    v[i] = x0[i];
+                    v[16 + i] = x1[i];
+                    v[32 + i] = x2[i];
+                    v[48 + i] = x3[i];
+                }
+            } else if constexpr (C == 32) {
                 float x0[16], x1[16];
                 tmem_ld16x2(trow, trow + 16, x0, x1);
 #pragma unroll
@@ -432,23 +458,40 @@ __global__ void __launch_bounds__(kGateThreads, 1)
                     v[i] = x0[i];
                     v[16 + i] = x1[i];
                 }
-            } else if constexpr (CH == 16) {
-                tmem_ld16(trow, v);
             } else {
-                tmem_ld8(trow, v);
+                tmem_ld16(trow, v);
             }
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(acc_empty + buf);  // the MMAs of tile it + NB may overwrite it
-            const int b = tile / tiles_per_row, m = 32 * (warp & 3) + lane;
-            const int t = (tile % tiles_per_row) * kGateM + m;
-            if (t < L) {
-                IO *gt = g + ((int64_t)b * L + t) * D + col0 + cb;
+            const int b = tile / tiles_per_row, t0 = (tile % tiles_per_row) * kGateM, m = 32 * warp + lane;
+            if constexpr (Cfg::STAGE_OUT) {
+                // row m into the staging, then the tile in whole rows: C / 4 threads per time step
+                float *srow = stg + m * Cfg::OUT_PITCH;
 #pragma unroll
-                for (int c = 0; c < CH; c += 4) {
-                    const float xv[4] = {v[c] + sbias[cb + c], v[c + 1] + sbias[cb + c + 1],
-                                         v[c + 2] + sbias[cb + c + 2], v[c + 3] + sbias[cb + c + 3]};
-                    store4(gt + c, xv, vec_out != 0);
+                for (int c = 0; c < C; c += 4)
+                    *reinterpret_cast<float4 *>(srow + c) =
+                        make_float4(v[c] + sbias[c], v[c + 1] + sbias[c + 1], v[c + 2] + sbias[c + 2], v[c + 3] + sbias[c + 3]);
+                bar_sync(2, EPT);
+#pragma unroll 4
+                for (int q = tid; q < kGateM * Cfg::C4; q += EPT) {
+                    const int row = q / Cfg::C4, c4 = q - row * Cfg::C4, t = t0 + row;
+                    if (t < L) {
+                        const float4 x = *reinterpret_cast<const float4 *>(stg + row * Cfg::OUT_PITCH + 4 * c4);
+                        const float xv[4] = {x.x, x.y, x.z, x.w};
+                        store4(g + ((int64_t)b * L + t) * D + col0 + 4 * c4, xv, vec_out != 0);
+                    }
+                }
+            } else {
+                const int t = t0 + m;
+                if (t < L) {
+                    IO *gt = g + ((int64_t)b * L + t) * D + col0;
+#pragma unroll
+                    for (int c = 0; c < C; c += 4) {
+                        const float xv[4] = {v[c] + sbias[c], v[c + 1] + sbias[c + 1], v[c + 2] + sbias[c + 2],
+                                             v[c + 3] + sbias[c + 3]};
+                        store4(gt + c, xv, vec_out != 0);
+                    }
                 }
             }
         }
