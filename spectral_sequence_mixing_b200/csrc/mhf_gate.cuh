@@ -219,7 +219,6 @@ __global__ void __launch_bounds__(kGateThreads, 1)
     const int64_t col0 = (int64_t)h * C;
     const int first = blockIdx.x / H;
 
-    if (warp == 0) tmem_alloc(tslot, Cfg::TMEM_COLS);
     if (tid == 0)
         for (int i = 0; i < NB; ++i) {
             mbar_init(full + i, kGateThreads / 32 - kGateProdWarp0);  // one arrival per producer warp
@@ -228,42 +227,52 @@ __global__ void __launch_bounds__(kGateThreads, 1)
             mbar_init(acc_empty + i, kGateEpiWarps);                  // one arrival per epilogue warp
             mbar_init(loaded + i, 1);                                 // TMA of a tile's input
         }
+    __syncthreads();  // the barriers are initialised before any role uses them
 
-    // The head's weights, split into fp16 hi / lo, in the K-major layout: tap
-    // k, chunk c/8, output channel n, element c%8.  The head's block of w
-    // ([D][C][K], C K contiguous floats per output channel n) is read with
-    // coalesced 16-byte loads (vec_w: the block is 16-byte aligned) and each
-    // element is split and placed by 2-byte stores.  (The block is read once
-    // per CTA, from L2 after the first CTA of the head.)
-    {
-        const float *wh = w + col0 * C * KT;
-        constexpr int NW = C * C * KT;  // the head's weights
-        auto place = [&](int e, float x) {  // element e = (n C + c) KT + k
-            const int k = e % KT, c = (e / KT) % C, n = e / (KT * C);
-            const unsigned off = k * Cfg::W_TAP + (c >> 3) * Cfg::LBO_W + n * 16u + (c & 7) * 2u;
-            const __half hi = __float2half_rn(x), lo = __float2half_rn(x - __half2float(hi));
-            *reinterpret_cast<__half *>(sm + Cfg::OFF_WHI + off) = hi;
-            *reinterpret_cast<__half *>(sm + Cfg::OFF_WLO + off) = lo;
-        };
-        if (((uintptr_t)wh & 15) == 0) {
+    // The producers start on their first tiles at once; meanwhile the other
+    // warps (MMA and epilogue) allocate TMEM and stage the head's weights and
+    // bias, which only they use.
+    constexpr int SET = 32 * kGateProdWarp0;  // threads of the MMA and epilogue roles
+    unsigned tmem = 0;
+    if (warp < kGateProdWarp0) {
+        if (warp == 0) tmem_alloc(tslot, Cfg::TMEM_COLS);
+        // The head's weights, split into fp16 hi / lo, in the K-major layout: tap
+        // k, chunk c/8, output channel n, element c%8.  The head's block of w
+        // ([D][C][K], C K contiguous floats per output channel n) is read with
+        // coalesced 16-byte loads (vec_w: the block is 16-byte aligned) and each
+        // element is split and placed by 2-byte stores.  (The block is read once
+        // per CTA, from L2 after the first CTA of the head.)
+        {
+            const float *wh = w + col0 * C * KT;
+            constexpr int NW = C * C * KT;  // the head's weights
+            auto place = [&](int e, float x) {  // element e = (n C + c) KT + k
+                const int k = e % KT, c = (e / KT) % C, n = e / (KT * C);
+                const unsigned off = k * Cfg::W_TAP + (c >> 3) * Cfg::LBO_W + n * 16u + (c & 7) * 2u;
+                const __half hi = __float2half_rn(x), lo = __float2half_rn(x - __half2float(hi));
+                *reinterpret_cast<__half *>(sm + Cfg::OFF_WHI + off) = hi;
+                *reinterpret_cast<__half *>(sm + Cfg::OFF_WLO + off) = lo;
+            };
+            if (((uintptr_t)wh & 15) == 0) {
 #pragma unroll 2
-            for (int q4 = tid; q4 < NW / 4; q4 += kGateThreads) {
-                const float4 x = __ldg(reinterpret_cast<const float4 *>(wh) + q4);
-                place(4 * q4, x.x);
-                place(4 * q4 + 1, x.y);
-                place(4 * q4 + 2, x.z);
-                place(4 * q4 + 3, x.w);
+                for (int q4 = tid; q4 < NW / 4; q4 += SET) {
+                    const float4 x = __ldg(reinterpret_cast<const float4 *>(wh) + q4);
+                    place(4 * q4, x.x);
+                    place(4 * q4 + 1, x.y);
+                    place(4 * q4 + 2, x.z);
+                    place(4 * q4 + 3, x.w);
+                }
+            } else {
+                for (int e = tid; e < NW; e += SET) place(e, __ldg(wh + e));
             }
-        } else {
-            for (int e = tid; e < NW; e += kGateThreads) place(e, __ldg(wh + e));
         }
+        static_assert(SET >= 64, "the bias is staged by the first 64 threads");
+        if (tid < C) sbias[tid] = bias ? __ldg(bias + col0 + tid) : 0.0f;
+        fence_proxy_async_smem();  // the weights are read by the tensor core
+        tc_fence_before_sync();
+        bar_sync(3, SET);
+        tc_fence_after_sync();
+        tmem = *tslot;
     }
-    if (tid < C) sbias[tid] = bias ? __ldg(bias + col0 + tid) : 0.0f;
-    fence_proxy_async_smem();  // the weights are read by the tensor core
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-    const unsigned tmem = *tslot;
     bool ok = true;    // every wait of this thread's role completed
     int last_it = -1;  // MMA warp: the last tile whose MMAs it committed
 
