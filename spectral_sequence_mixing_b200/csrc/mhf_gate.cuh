@@ -50,7 +50,7 @@ namespace ccv {
 
 constexpr unsigned kFaultMmaWait = 2u;  // fault bit: an MMA completion wait ran out
 constexpr int kGateM = 128;             // time steps per tile (MMA M)
-constexpr int kGateThreads = 512;       // sixteen warps: four per TMEM lane quarter, a quarter of the columns each
+constexpr int kGateThreads = 640;       // twenty warps: eight epilogue, one MMA, eleven producer warps
 constexpr int kGateMaxTaps = 4;
 
 template <int C, int KT>
@@ -183,16 +183,16 @@ __device__ __forceinline__ void store4(__nv_bfloat16 *p, const float (&v)[4], bo
     }
 }
 
-// Warp roles (sixteen warps): warps 0-3 drain the accumulators (warp w
-// reads TMEM lanes 32 w .. +31, i.e. time steps, and all the columns,
-// stages its rows with the bias and then the four warps store the tile in
-// whole rows), warp 4 issues the MMAs (one lane, elect.sync), warps 5-15
+// Warp roles (twenty warps): warps 0-7 drain the accumulators (warp w
+// reads TMEM lanes 32 (w % 4) .. +31, i.e. time steps, and the column half
+// w / 4, stages them with the bias, and the eight warps then store the tile
+// in whole rows), warp 8 issues the MMAs (one lane, elect.sync), warps 9-19
 // stage sigmoid tiles (the conversion is the slowest role, so it gets the
 // most warps).  Tiles and accumulators (NBUF of each) are handed over on
 // mbarriers -- full / empty for the sigmoid tiles, acc_full / acc_empty for
 // the accumulators -- so no role waits at a CTA-wide barrier in the steady
 // state.
-constexpr int kGateEpiWarps = 4, kGateMmaWarp = 4, kGateProdWarp0 = 5;
+constexpr int kGateEpiWarps = 8, kGateMmaWarp = 8, kGateProdWarp0 = 9;
 constexpr int kGateProdThreads = kGateThreads - 32 * kGateProdWarp0;
 
 // grid = H * groups CTAs; CTA (h = blockIdx.x % H, j = blockIdx.x / H) takes
@@ -428,7 +428,7 @@ __global__ void __launch_bounds__(kGateThreads, 1)
             last_it = it;
         }
     } else if (warp < kGateEpiWarps) {
-        // ---- epilogue: accumulator rows 32 warp + lane (time steps), all C columns, + bias, store
+        // ---- epilogue: accumulator rows 32 (warp % 4) + lane (time steps), column half warp / 4, + bias, store
         float *stg = reinterpret_cast<float *>(sm + Cfg::OFF_OUT);
         constexpr int EPT = 32 * kGateEpiWarps;  // epilogue threads
         int it = 0;
@@ -446,20 +446,11 @@ __global__ void __launch_bounds__(kGateThreads, 1)
                 break;
             }
             tc_fence_after_sync();
-            float v[C];
-            const unsigned trow = tmem + buf * C + ((unsigned)(32 * warp) << 16);
-            if constexpr (C == 64) {
-                float x0[16], x1[16], x2[16], x3[16];
-                tmem_ld16x2(trow, trow + 16, x0, x1);
-                tmem_ld16x2(trow + 32, trow + 48, x2, x3);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    v[i] = x0[i];
-                    v[16 + i] = x1[i];
-                    v[32 + i] = x2[i];
-                    v[48 + i] = x3[i];
-                }
-            } else if constexpr (C == 32) {
+            constexpr int CH = C / 2;  // this warp's columns: [cb, cb + CH)
+            const int cb = CH * (warp >> 2);
+            float v[CH];
+            const unsigned trow = tmem + buf * C + cb + ((unsigned)(32 * (warp & 3)) << 16);
+            if constexpr (CH == 32) {
                 float x0[16], x1[16];
                 tmem_ld16x2(trow, trow + 16, x0, x1);
 #pragma unroll
@@ -467,20 +458,23 @@ __global__ void __launch_bounds__(kGateThreads, 1)
                     v[i] = x0[i];
                     v[16 + i] = x1[i];
                 }
-            } else {
+            } else if constexpr (CH == 16) {
                 tmem_ld16(trow, v);
+            } else {
+                tmem_ld8(trow, v);
             }
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(acc_empty + buf);  // the MMAs of tile it + NB may overwrite it
-            const int b = tile / tiles_per_row, t0 = (tile % tiles_per_row) * kGateM, m = 32 * warp + lane;
+            const int b = tile / tiles_per_row, t0 = (tile % tiles_per_row) * kGateM, m = 32 * (warp & 3) + lane;
             if constexpr (Cfg::STAGE_OUT) {
-                // row m into the staging, then the tile in whole rows: C / 4 threads per time step
-                float *srow = stg + m * Cfg::OUT_PITCH;
+                // this warp's half of row m into the staging, then the tile in whole rows:
+                // C / 4 threads per time step
+                float *srow = stg + m * Cfg::OUT_PITCH + cb;
 #pragma unroll
-                for (int c = 0; c < C; c += 4)
-                    *reinterpret_cast<float4 *>(srow + c) =
-                        make_float4(v[c] + sbias[c], v[c + 1] + sbias[c + 1], v[c + 2] + sbias[c + 2], v[c + 3] + sbias[c + 3]);
+                for (int c = 0; c < CH; c += 4)
+                    *reinterpret_cast<float4 *>(srow + c) = make_float4(
+                        v[c] + sbias[cb + c], v[c + 1] + sbias[cb + c + 1], v[c + 2] + sbias[cb + c + 2], v[c + 3] + sbias[cb + c + 3]);
                 bar_sync(2, EPT);
 #pragma unroll 4
                 for (int q = tid; q < kGateM * Cfg::C4; q += EPT) {
@@ -494,11 +488,11 @@ __global__ void __launch_bounds__(kGateThreads, 1)
             } else {
                 const int t = t0 + m;
                 if (t < L) {
-                    IO *gt = g + ((int64_t)b * L + t) * D + col0;
+                    IO *gt = g + ((int64_t)b * L + t) * D + col0 + cb;
 #pragma unroll
-                    for (int c = 0; c < C; c += 4) {
-                        const float xv[4] = {v[c] + sbias[c], v[c + 1] + sbias[c + 1], v[c + 2] + sbias[c + 2],
-                                             v[c + 3] + sbias[c + 3]};
+                    for (int c = 0; c < CH; c += 4) {
+                        const float xv[4] = {v[c] + sbias[cb + c], v[c + 1] + sbias[cb + c + 1],
+                                             v[c + 2] + sbias[cb + c + 2], v[c + 3] + sbias[cb + c + 3]};
                         store4(gt + c, xv, vec_out != 0);
                     }
                 }
