@@ -146,6 +146,7 @@ def recorded_counters(workload: str, kernel: str):
     p = os.path.join(ROOT, "profiles", "kernel_counters.txt")
     if not os.path.exists(p):
         return None, None, None
+    kernel = kernel.split(" (")[0]  # "bigconv_kernel (two-pass step: ...)" -> the row kernel
     for line in open(p):
         f = line.split()
         if len(f) == 6 and not line.startswith("#") and f[0] == workload and f[1] == kernel:
