@@ -227,3 +227,19 @@ def test_dwconv_host_side_argument_errors(lib, fn):
     assert f(A, W_, None, A + 64, *ok, None) == 3               # y overlaps x
     assert f(A, W_, None, W_ - 64, *ok, None) == 3              # y overlaps w
     assert f(A, W_, Y_ + 8, Y_, *ok, None) == 3                 # y overlaps bias
+
+
+def test_probe_library_builds_and_exports_its_entry():
+    """The rate probes behind `bench.py --probe` build with the library
+    (their own .so, outside the C ABI) and export ccp_run; a bad kind is
+    refused before any CUDA call."""
+    from spectral_sequence_mixing_b200 import build
+    build.build()
+    assert os.path.exists(build.PROBE_LIB)
+    probe = ctypes.CDLL(build.PROBE_LIB)
+    assert hasattr(probe, "ccp_run")
+    probe.ccp_run.restype = ctypes.c_int
+    probe.ccp_run.argtypes = [ctypes.c_int] * 4 + [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_double)]
+    ms, units = ctypes.c_float(0), ctypes.c_double(0)
+    assert probe.ccp_run(99, 1, 32, 1, ctypes.byref(ms), ctypes.byref(units)) != 0
+    assert probe.ccp_run(0, 0, 32, 1, ctypes.byref(ms), ctypes.byref(units)) != 0
