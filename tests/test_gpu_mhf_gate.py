@@ -2,8 +2,8 @@
 convolution with the oracle (oracle/mhf_gate.py), through the C ABI.
 
 Bounds, from the arithmetic (the gate's contraction is fp32-exact up to the
-tf32 split, 3 * 2^-20 of |w| sigmoid(a) per term at worst, and sigmoid is
-evaluated in fp32):
+fp16 hi/lo split, whose dropped lo*lo term and rounded lo parts stay below
+2^-21 of |w| sigmoid(a) per term, and sigmoid is evaluated in fp32):
   gate, fp32 I/O:   |g - g_ref| <= 1e-5 * gabs,  gabs = |bias| + sum |w| sigmoid(a)
   gate, bf16 I/O:   |g - g_ref| <= 2e-2 * gabs   (g rounded to bf16: <= 2^-9 gabs)
   gated conv:       |r - r_ref| <= tol * sum_j |v_j| gabs_{t-j},  tol 1e-5 / 2e-2
