@@ -126,7 +126,11 @@ CC_API int causal_ntt_conv_i32(const int32_t *v, const int32_t *g, int32_t *r,
  * Both are anti-causal correlations; with rev(x)_t = x_{L-1-t} they equal
  * rev(conv(rev(dr), g)) and rev(conv(rev(dr), v)), which is how they are
  * computed: two launches of the forward kernels with time-reversed input and
- * output indexing (no extra copies).
+ * output indexing (no extra copies).  For L <= 1024 the dg launch runs on a
+ * library-owned stream of the device, forked from `stream` by an event and
+ * joined back to it, so it fills the SMs the dv launch's last wave leaves
+ * idle; `stream` still orders everything after the call (capturable in a
+ * CUDA graph like any fork and join).
  *   dr, v, g  [B, L, D] float32 (device); dv, dg [B, L, D] float32 outputs
  *   (device), overlapping none of the inputs or each other.
  * Accuracy, ranges, workspace and errors as causal_fftconv_f32, with the

@@ -597,10 +597,52 @@ static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t 
     return CC_ERR_UNSUPPORTED;
 }
 
+// A library-owned stream per device for work that may run beside the
+// caller's stream, with the events that fork it from and join it back to
+// that stream.
+struct SidePipe {
+    cudaStream_t s2 = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    std::mutex mu;
+};
+
+static SidePipe *side_pipe(int dev) {
+    static SidePipe pipes[128];
+    static std::once_flag once[128];
+    static bool ok[128];
+    std::call_once(once[dev], [dev] {
+        SidePipe &p = pipes[dev];
+        ok[dev] = cudaStreamCreateWithFlags(&p.s2, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&p.fork, cudaEventDisableTiming) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&p.join, cudaEventDisableTiming) == cudaSuccess;
+        cudaGetLastError();
+    });
+    return ok[dev] ? &pipes[dev] : nullptr;
+}
+
 // Backward: dv = rev(conv(rev(dr), g)), dg = rev(conv(rev(dr), v)).
 template <typename IO>
 static int fftconv_bwd(const IO *dr, const IO *v, const IO *g, IO *dv, IO *dg, int64_t B, int64_t L, int64_t D,
                        void *ws, size_t ws_bytes, cudaStream_t s, int dev) {
+    // Rows of the fused kernel (no workspace involved): dg goes on a library
+    // stream forked from the caller's, so its CTAs take the SMs that dv's last,
+    // partial wave leaves idle; the caller's stream then waits for both.
+    SidePipe *sp = L <= CfgM<IO>::LMAX ? side_pipe(dev) : nullptr;
+    if (sp) {
+        std::lock_guard<std::mutex> lk(sp->mu);
+        if (cudaEventRecord(sp->fork, s) != cudaSuccess || cudaStreamWaitEvent(sp->s2, sp->fork, 0) != cudaSuccess) {
+            cudaGetLastError();
+            return CC_ERR_CUDA;
+        }
+        const int st1 = fftconv_dispatch<IO>(dr, g, dv, B, L, D, ws, ws_bytes, s, dev, 3);
+        const int st2 = fftconv_dispatch<IO>(dr, v, dg, B, L, D, ws, ws_bytes, sp->s2, dev, 3);
+        // join whatever was enqueued, also after an error
+        if (cudaEventRecord(sp->join, sp->s2) != cudaSuccess || cudaStreamWaitEvent(s, sp->join, 0) != cudaSuccess) {
+            cudaGetLastError();
+            return CC_ERR_CUDA;
+        }
+        return st1 != CC_OK ? st1 : st2;
+    }
     int st = fftconv_dispatch<IO>(dr, g, dv, B, L, D, ws, ws_bytes, s, dev, 3);
     if (st != CC_OK) return st;
     return fftconv_dispatch<IO>(dr, v, dg, B, L, D, ws, ws_bytes, s, dev, 3);
