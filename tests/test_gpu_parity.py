@@ -381,6 +381,38 @@ def test_cuda_graph_capture_and_replay(shape):
     assert torch.equal(out, ref)
 
 
+def test_bwd_fork_join_capture_and_side_stream():
+    """The backward of fused-kernel rows forks its dg launch onto a library
+    stream and joins it back: on a caller's side stream and inside a CUDA
+    graph capture the results equal the eager default-stream call bit for
+    bit, and the caller's stream sees both outputs complete."""
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    rng = np.random.Generator(np.random.PCG64(21))
+    dr, v, g = (to_dev(rng.standard_normal((3, 777, 24)).astype(np.float32), "f32") for _ in range(3))
+    ref_dv, ref_dg = ssm.causal_conv_bwd(dr, v, g)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    dv, dg = torch.empty_like(dr), torch.empty_like(dr)
+    with torch.cuda.stream(s):
+        ssm.causal_conv_bwd(dr, v, g, dv=dv, dg=dg, stream=s)
+        # consumers on the caller's stream: both halves are complete here
+        cv, cg = dv.clone(), dg.clone()
+    s.synchronize()
+    assert torch.equal(dv, ref_dv) and torch.equal(dg, ref_dg)
+    assert torch.equal(cv, ref_dv) and torch.equal(cg, ref_dg)
+    graph = torch.cuda.CUDAGraph()
+    dv.zero_()
+    dg.zero_()
+    with torch.cuda.graph(graph):
+        ssm.causal_conv_bwd(dr, v, g, dv=dv, dg=dg, stream=torch.cuda.current_stream())
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(dv, ref_dv) and torch.equal(dg, ref_dg)
+
+
 def test_rejects_host_pointer_on_device_entry():
     import torch
     from spectral_sequence_mixing_b200 import _lib
