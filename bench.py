@@ -42,7 +42,8 @@ _FUSED_SOURCES = ["fftconv_fused.cuh", "fft_reg.cuh", "tma.cuh", "configs_fused.
 KERNEL_SOURCES = {
     "fftconv_fused_kernel": _FUSED_SOURCES,
     "bigrow_group_kernel": ["bigconv.cuh", "configs_rows.cuh"] + _FUSED_SOURCES,
-    "bigconv_kernel": ["bigconv.cuh", "configs_rows.cuh", "transpose.cuh"] + _FUSED_SOURCES,
+    "bigconv_kernel": ["bigconv.cuh", "configs_rows.cuh"] + _FUSED_SOURCES,
+    "hr_mid_kernel": ["hbmrows.cuh"] + _FUSED_SOURCES,
     "ntt_conv_kernel": ["ntt.cuh"],
     "tcconv_kernel": ["tcconv.cuh", "tcgen05.cuh", "tma.cuh"],
     "mhf_gate_kernel": ["mhf_gate.cuh", "tcgen05.cuh", "tma.cuh"],
@@ -146,7 +147,7 @@ def recorded_counters(workload: str, kernel: str):
     p = os.path.join(ROOT, "profiles", "kernel_counters.txt")
     if not os.path.exists(p):
         return None, None, None
-    kernel = kernel.split(" (")[0]  # "bigconv_kernel (two-pass step: ...)" -> the row kernel
+    kernel = kernel.split(" (")[0]  # "hr_mid_kernel (four-step: ...)" -> the kernel name
     for line in open(p):
         f = line.split()
         if len(f) == 6 and not line.startswith("#") and f[0] == workload and f[1] == kernel:
@@ -315,7 +316,7 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def dominant_kernel(w: workloads.Workload, two_pass: bool) -> str:
+def dominant_kernel(w: workloads.Workload, four_step: bool) -> str:
     """The kernel that does a forward call's transform on workload `w`."""
     if w.dtype == "i32":
         return "ntt_conv_kernel"
@@ -325,7 +326,8 @@ def dominant_kernel(w: workloads.Workload, two_pass: bool) -> str:
         return "bigrow_group_kernel"
     if w.L <= 4096:
         return "tcconv_kernel" if w.dtype == "bf16" else "bigrow_group_kernel"
-    return "bigconv_kernel (two-pass step: 2 transposes in, 1 out)" if two_pass else "bigconv_kernel"
+    return ("hr_mid_kernel (four-step path: the norm, alpha, fwd, mid and inv launches of a step; traffic and "
+            "ALU counts are the whole step's)") if four_step else "bigconv_kernel"
 
 
 def probe_rates():
@@ -431,7 +433,7 @@ def time_config(w: workloads.Workload, rank, world, dev, pg, steps: int, warmup:
         "transform_len": 2 ** math.ceil(math.log2(2 * w.L)),
         "ms_per_step": ms, "steps": reps * G, "value": achieved * world, "unit": "GB/s",
         "outputs_per_s": w.units * world / (ms * 1e-3),
-        "launch": f"CUDA graph replay of {G} steps ({4 if n_ws else 1} launches per step)",
+        "launch": f"CUDA graph replay of {G} steps ({5 if n_ws else 1} launches per step)",
         "l2": f"cold: {n_sets} rotating (v,g,r) sets of {set_bytes / 2 ** 20:.1f} MiB",
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)", "kernel": kernel,
@@ -484,11 +486,11 @@ def run_ours(args, rank, world, local):
     sets = [(v0, g0, torch.empty_like(v0))] + [(v0.clone(), g0.clone(), torch.empty_like(v0)) for _ in
                                                 range(n_sets - 1)]
     stream = torch.cuda.current_stream(dev)
-    # optional workspace of the two-pass long-row path (rows transposed to be
-    # contiguous): 2 transposes in, the row kernel, 1 transpose out per conv
+    # optional workspace of the four-step long-row path: norm partials, row
+    # scales, the forward pass, the middle pass and the inverse pass per conv
     n_ws = ssm.fast_workspace_bytes(tdt, w.B, w.L, w.D)
     ws = torch.empty(n_ws, dtype=torch.uint8, device=dev)
-    conv_launches = 4 if n_ws else 1
+    conv_launches = 5 if n_ws else 1
     if args.path == "fwd":
         def fn(a, b, out, stream):
             ssm.causal_conv(a, b, out=out, workspace=ws, stream=stream)

@@ -71,8 +71,8 @@ typedef enum {
  *   workspace / workspace_bytes: device scratch of at least
  *   causal_conv_workspace_bytes(CC_DTYPE_F32, B, L, D) bytes (0 for every
  *   supported L: NULL, 0 is valid).  A workspace of at least
- *   causal_conv_fast_workspace_bytes(...) bytes (nonzero for 4096 < L) makes
- *   long rows take the two-pass path (rows transposed to be contiguous); it
+ *   causal_conv_fast_workspace_bytes(...) bytes (nonzero for 4096 < L),
+ *   16-byte aligned, makes long rows take the four-step path through it; it
  *   must then not overlap v, g or r (CC_ERR_ALIAS).  Caller-owned; its
  *   contents are scratch, undefined after the call.
  *
@@ -230,18 +230,23 @@ CC_API int causal_conv_from_host(int dtype, const void *v_host, const void *g_ho
 
 /*
  * causal_conv_fast_workspace_bytes -- optional workspace for rows longer than
- * one CTA holds (4096 < L <= 65536, float paths).  Such a row is transformed
- * by a cluster of 8 CTAs; read straight from a channel-last [B, L, D] tensor
- * its time steps are D elements apart.  When causal_fftconv_f32/bf16 and the
- * backward entry points receive a workspace of at least this many bytes they
- * take a two-pass path instead: v and g are transposed to [B, D, L] in the
- * workspace (rows contiguous), the rows are transformed from there, and r is
- * transposed back (three [B, L, D] arrays, each 256-byte aligned).  The result
- * is the same convolution computed in the same order; the workspace must not
- * overlap any tensor of the call (CC_ERR_ALIAS).  A smaller workspace (or
- * none) selects the single-pass path.  Returns 0 when no such path applies
- * (L <= 4096, the NTT path, B > 65535) and for invalid arguments.  The pages
- * have no counterpart; it is a layout choice of this library.
+ * one CTA holds (4096 < L <= 65536, float paths; transform length N = 131072).
+ * Without it such a row is transformed by a cluster of 8 CTAs reading the
+ * channel-last tensors straight (time steps D elements apart; 8-CTA clusters
+ * fit 120 of B200's 148 SMs).  When causal_fftconv_f32/bf16 and the backward
+ * entry points receive a 16-byte-aligned workspace of at least this many
+ * bytes they take the four-step path instead (Caracal, limitations: 100k+
+ * contexts): per row the sums of squares of v and g, the 256-point DFTs over
+ * n2 of t = n1 + 512 n2, the 512-point DFTs over n1 with the spectral product
+ * and the first half of the real-output inverse, then the last inverse step
+ * with the stores -- each pass on every SM, exchanging the partial transforms
+ * through the workspace (N x B x D float2, rows innermost, then 64 float2 of
+ * norm partials and one float2 of scales per row).  Same convolution, same
+ * accuracy bound, a different summation order from the single-pass path.
+ * The workspace must not overlap any tensor of the call (CC_ERR_ALIAS); its
+ * contents are scratch.  A smaller or misaligned workspace (or none) selects
+ * the single-pass path.  Returns 0 when no such path applies (L <= 4096, the
+ * NTT path, B x D beyond INT32_MAX) and for invalid arguments.
  */
 CC_API size_t causal_conv_fast_workspace_bytes(int dtype, int64_t B, int64_t L, int64_t D);
 

@@ -54,7 +54,7 @@ def _stream_ptr(stream) -> int:
 
 def fast_workspace_bytes(dtype: torch.dtype, B: int, L: int, D: int) -> int:
     """Bytes of the optional workspace that lets long rows (4096 < L <= 65536)
-    take the two-pass path with contiguous rows; 0 where it does not apply."""
+    take the four-step path through device memory; 0 where it does not apply."""
     return int(load().causal_conv_fast_workspace_bytes(_DT[dtype], B, L, D))
 
 
@@ -63,7 +63,7 @@ _ONE_CTA_ROW = 4096  # rows up to this length never use the optional workspace
 
 def _workspace(workspace, dtype_code: int, B: int, L: int, D: int, device):
     """(pointer, bytes) of the caller's workspace; with none given, one of the
-    optional two-pass size is taken from the torch allocator when that path
+    optional four-step size is taken from the torch allocator when that path
     applies.  A tensor of 0 bytes selects the single-pass path."""
     if workspace is None:
         if L <= _ONE_CTA_ROW or dtype_code == CC_DTYPE_I32:

@@ -22,7 +22,7 @@
 #include "bigconv.cuh"
 #include "ntt.cuh"
 #include "decode.cuh"
-#include "transpose.cuh"
+#include "hbmrows.cuh"
 #include "mhf_gate.cuh"
 #include "dwconv.cuh"
 #include "tcconv.cuh"
@@ -38,6 +38,7 @@ __device__ float2 g_tw_m[CfgM<float>::TW_SIZE];
 __device__ float2 g_tw_bm[BigM<float>::TW_SIZE];
 __device__ float2 g_tw_bl[BigL<float>::TW_SIZE];
 __device__ float2 g_tw_bx[BigX<float>::TW_SIZE];
+__device__ __align__(16) float2 g_tw_hr[kHrTwSize];
 
 static double kTwoPi = 6.283185307179586476925286766559;
 
@@ -96,6 +97,34 @@ static std::vector<float2> big_twiddles() {
                 t[Cfg::TAHB + k * (STAH / QA) + lh] = omega((int64_t)QA * lh * k, SL / 2);
         }
     }
+    return t;
+}
+
+// Four-step long-row tables (hbmrows.cuh); theta = omega_2N, phi = theta^2.
+static std::vector<float2> hr_twiddles() {
+    std::vector<float2> t(kHrTwSize);
+    const int64_t N2 = 2 * (int64_t)kHrN;
+    for (int n2 = 0; n2 < 128; ++n2) t[kHrTW1 + n2] = omega(n2, 512);
+    for (int a = 0; a < 16; ++a)
+        for (int c = 0; c < 16; ++c) t[kHrTA + a * 16 + c] = omega(a * c, 256);
+    for (int n1 = 0; n1 < kHrA; ++n1)
+        for (int c = 0; c < 16; ++c) {
+            t[kHrTO1 + n1 * 16 + c] = omega((int64_t)n1 * (2 * c + 1), N2);
+            t[kHrTO2 + n1 * 16 + c] = omega((int64_t)32 * n1 * c, N2);
+        }
+    for (int p = 0; p < 16; ++p)
+        for (int u = 0; u < 32; ++u) t[kHrT512 + p * 32 + u] = omega(p * u, 512);
+    for (int k2 = 0; k2 < kHrB; ++k2) t[kHrPK1 + k2] = omega(-(2 * (int64_t)k2 + 1), N2);
+    for (int u = 0; u < 32; ++u)
+        for (int q = 0; q < 8; ++q) {
+            t[kHrPK2 + u * 8 + q] = omega(-(512 * (int64_t)u + 16384 * (int64_t)q), N2);
+            t[kHrTI + u * 8 + q] = omega(-(int64_t)u * q, 256);
+        }
+    for (int k2 = 0; k2 < kHrB; ++k2) {
+        for (int al = 0; al < 8; ++al) t[kHrTWa + k2 * 8 + al] = omega(-2 * (int64_t)al * (2 * k2 + 1), N2);
+        for (int be = 0; be < 32; ++be) t[kHrTWb + k2 * 32 + be] = omega(-16 * (int64_t)be * (2 * k2 + 1), N2);
+    }
+    for (int m2 = 0; m2 < 128; ++m2) t[kHrTU + m2] = omega(-m2, 512);
     return t;
 }
 
@@ -206,8 +235,8 @@ static unsigned long long current_ctx_id() {
 // Per device: SM count and, per kernel instantiation, resident CTAs per SM.
 static int g_num_sms[128];
 // Per device: device addresses of the twiddle tables (fused N = 512, 2048; one-CTA
-// rows N = 8192; cluster rows; one-CTA rows N = 4096).
-static void *g_tw_addr[128][5];
+// rows N = 8192; cluster rows; one-CTA rows N = 4096; four-step long rows).
+static void *g_tw_addr[128][6];
 
 template <class Cfg, typename IO, int MINB>
 static cudaError_t set_smem_attr() {
@@ -256,6 +285,21 @@ static cudaError_t ensure_init(int dev) {
         auto t = big_twiddles<BigX<float>>();
         if ((e = cudaMemcpyToSymbol(g_tw_bx, t.data(), t.size() * sizeof(float2))) != cudaSuccess) return e;
     }
+    {
+        auto t = hr_twiddles();
+        if ((e = cudaMemcpyToSymbol(g_tw_hr, t.data(), t.size() * sizeof(float2))) != cudaSuccess) return e;
+        if ((e = cudaFuncSetAttribute(hr_fwd_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kHrFwdSmem)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(hr_fwd_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kHrFwdSmem)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(hr_inv_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kHrFwdSmem)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(hr_inv_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kHrFwdSmem)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(hr_mid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kHrMidSmem)) != cudaSuccess)
+            return e;
+    }
     if ((e = set_big_attr<BigM<float>, float, kMinbBigM>()) != cudaSuccess) return e;
     if ((e = set_big_attr<BigM<__nv_bfloat16>, __nv_bfloat16, kMinbBigM>()) != cudaSuccess) return e;
     if ((e = set_big_attr<BigL<float>, float, kMinbBigL>()) != cudaSuccess) return e;
@@ -280,6 +324,7 @@ static cudaError_t ensure_init(int dev) {
     if ((e = cudaGetSymbolAddress(&g_tw_addr[dev][2], g_tw_bl)) != cudaSuccess) return e;
     if ((e = cudaGetSymbolAddress(&g_tw_addr[dev][3], g_tw_bx)) != cudaSuccess) return e;
     if ((e = cudaGetSymbolAddress(&g_tw_addr[dev][4], g_tw_bm)) != cudaSuccess) return e;
+    if ((e = cudaGetSymbolAddress(&g_tw_addr[dev][5], g_tw_hr)) != cudaSuccess) return e;
     g_init_ctx[dev] = current_ctx_id();
     g_init_done[dev] = true;
     return cudaSuccess;
@@ -468,20 +513,17 @@ static int launch_big(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int
     return CC_OK;
 }
 
-// Workspace that enables the two-pass path of rows longer than one CTA holds
-// (three [B, L, D] arrays: v and g with rows made contiguous, and r before
-// its transpose back); 0 when that path does not apply.
+// Workspace that enables the four-step path of rows longer than one CTA
+// holds (hbmrows.cuh: the partial transforms of every row, norm partials and
+// per-row scales); 0 when that path does not apply.
 static size_t fast_ws_bytes(int dtype, int64_t B, int64_t L, int64_t D) {
     if (dtype != CC_DTYPE_F32 && dtype != CC_DTYPE_BF16) return 0;
     if (B < 1 || D < 1 || L <= BigL<float>::LMAX || L > BigX<float>::LMAX) return 0;
-    if (B > 65535 || (L + kTrTile - 1) / kTrTile > 65535 || (D + kTrTile - 1) / kTrTile > 65535) return 0;
-    const int64_t es = dtype == CC_DTYPE_F32 ? 4 : 2;
-    if (D > INT64_MAX / (16 * L * es) / B) return 0;
-    const size_t one = ((size_t)(B * L * D * es) + 255) / 256 * 256;
-    return 3 * one;
+    if (D > INT32_MAX / B) return 0;  // rows and channel tiles are int
+    return hr_ws_bytes(B * D);
 }
 
-// A workspace large enough for the two-pass path is used by it: it must be
+// A workspace large enough for the four-step path is used by it: it must be
 // device memory of the current device and overlap none of the tensors.
 static int check_fast_ws(int dtype, int64_t B, int64_t L, int64_t D, const void *ws, size_t ws_bytes,
                          std::initializer_list<const void *> tensors) {
@@ -560,6 +602,35 @@ static int launch_tcconv(const __nv_bfloat16 *v, const __nv_bfloat16 *g, __nv_bf
     return cudaGetLastError() == cudaSuccess ? CC_OK : CC_ERR_CUDA;
 }
 
+// Four-step long rows through the workspace (hbmrows.cuh): norms, alpha,
+// forward over n2, the middle pass (forward over n1, product, packing, inner
+// inverse) in place, inverse over k2 with the stores.
+template <typename IO>
+static int launch_hbm_rows(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, void *ws,
+                           const float2 *tw, cudaStream_t s, int rev) {
+    const int64_t rows = B * D, tpb = (D + kHrCG - 1) / kHrCG, tiles = B * tpb;
+    float2 *Y = reinterpret_cast<float2 *>(ws);
+    float2 *part = reinterpret_cast<float2 *>(reinterpret_cast<char *>(ws) + hr_ws_part_off(rows));
+    float2 *as = reinterpret_cast<float2 *>(reinterpret_cast<char *>(ws) + hr_ws_as_off(rows));
+    constexpr uintptr_t vb = 4 * sizeof(IO);  // bytes of four channels
+    if (D % 4 == 0 && (reinterpret_cast<uintptr_t>(v) % vb) == 0 && (reinterpret_cast<uintptr_t>(g) % vb) == 0) {
+        const int64_t tpb4 = (D + 127) / 128;
+        hr_norms4_kernel<IO><<<dim3((unsigned)(B * tpb4), kHrSlices), 256, 0, s>>>(v, g, part, (int)L, (int)D,
+                                                                                  (int)rows, (int)tpb4);
+    } else {
+        hr_norms_kernel<IO><<<dim3((unsigned)tiles, kHrSlices), kHrNormThreads, 0, s>>>(v, g, part, (int)L, (int)D,
+                                                                                         (int)rows, (int)tpb);
+    }
+    hr_alpha_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(part, as, (int)rows);
+    hr_fwd_kernel<IO><<<dim3((unsigned)tiles, kHrA), kHrFwdThreads, kHrFwdSmem, s>>>(v, g, Y, as, tw, (int)L, (int)D,
+                                                                                      (int)rows, (int)tpb, rev);
+    hr_mid_kernel<<<dim3((unsigned)((rows + kHrRows2 - 1) / kHrRows2), kHrB / 2), kHrMidThreads, kHrMidSmem, s>>>(
+        Y, tw, (int)rows);
+    hr_inv_kernel<IO><<<dim3((unsigned)tiles, kHrB), kHrInvThreads, kHrFwdSmem, s>>>(Y, r, as, v, g, tw, (int)L,
+                                                                                      (int)D, (int)rows, (int)tpb, rev);
+    return cudaGetLastError() == cudaSuccess ? CC_OK : CC_ERR_CUDA;
+}
+
 template <typename IO>
 static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, void *ws,
                             size_t ws_bytes, cudaStream_t s, int dev, int rev = 0) {
@@ -577,22 +648,12 @@ static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t 
         return launch_group<BigL<IO>, kMinbBigL>(v, g, r, B, L, D, (const float2 *)tws[2], s, rev);
     }
     if (L <= BigX<IO>::LMAX) {
-        const void *tw = tws[3];
+        // rows of 8-CTA clusters read straight from the tensors, or the
+        // four-step path through a workspace that holds it
         const size_t fast = fast_ws_bytes(sizeof(IO) == 4 ? CC_DTYPE_F32 : CC_DTYPE_BF16, B, L, D);
-        if (ws == nullptr || fast == 0 || ws_bytes < fast)
-            return launch_big<BigX<IO>, kMinbBigX>(v, g, r, B, L, D, (const float2 *)tw, s, rev, 0);
-        // two-pass path: rows made contiguous in the workspace, transformed, transposed back
-        typedef typename std::conditional<sizeof(IO) == 4, uint32_t, uint16_t>::type W;
-        const size_t one = fast / 3;
-        IO *vt = reinterpret_cast<IO *>(ws);
-        IO *gt = reinterpret_cast<IO *>(reinterpret_cast<char *>(ws) + one);
-        IO *rt = reinterpret_cast<IO *>(reinterpret_cast<char *>(ws) + 2 * one);
-        int st;
-        if ((st = transpose_last2<W>((const W *)v, (W *)vt, B, L, D, s)) != CC_OK) return st;
-        if ((st = transpose_last2<W>((const W *)g, (W *)gt, B, L, D, s)) != CC_OK) return st;
-        if ((st = launch_big<BigX<IO>, kMinbBigX>(vt, gt, rt, B, L, D, (const float2 *)tw, s, rev, 1)) != CC_OK)
-            return st;
-        return transpose_last2<W>((const W *)rt, (W *)r, B, D, L, s);
+        if (ws == nullptr || fast == 0 || ws_bytes < fast || (reinterpret_cast<uintptr_t>(ws) & 15) != 0)
+            return launch_big<BigX<IO>, kMinbBigX>(v, g, r, B, L, D, (const float2 *)tws[3], s, rev, 0);
+        return launch_hbm_rows<IO>(v, g, r, B, L, D, ws, (const float2 *)tws[5], s, rev);
     }
     return CC_ERR_UNSUPPORTED;
 }

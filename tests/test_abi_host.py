@@ -165,13 +165,16 @@ def test_fault_flags_host_checks(lib):
 
 def test_fast_workspace_bytes(lib):
     f = lib.causal_conv_fast_workspace_bytes
-    assert f(0, 1, 4096, 8) == 0                       # rows of one CTA: no two-pass path
-    one = (4097 * 8 * 4 + 255) // 256 * 256
-    assert f(0, 1, 4097, 8) == 3 * one                  # fp32: three [B, L, D] arrays, 256-byte aligned
-    assert f(1, 2, 65536, 16) == 3 * (2 * 65536 * 16 * 2)
+
+    def four_step(rows):  # partial transforms [131072][rows] float2, 64 norm partials and a scale pair per row
+        return 131072 * rows * 8 + 64 * rows * 8 + rows * 8
+    assert f(0, 1, 4096, 8) == 0                       # rows of one CTA: no workspace path
+    assert f(0, 1, 4097, 8) == four_step(8)
+    assert f(1, 2, 65536, 16) == four_step(32)          # bf16 keeps fp32 partial transforms
     assert f(2, 1, 5000, 8) == 0                       # NTT path
     assert f(0, 1, 65537, 8) == 0                      # beyond the longest row
-    assert f(0, 70000, 5000, 8) == 0                   # B beyond the transpose grid
+    assert f(0, 70000, 5000, 8) == four_step(560000)
+    assert f(0, 2 ** 20, 5000, 2 ** 12) == 0           # B * D rows beyond int
     assert f(0, 1, 5000, 0) == 0 and f(7, 1, 5000, 8) == 0
 
 

@@ -46,7 +46,7 @@ def test_header_is_c99_and_host_queries_answer_from_c():
     assert (P * pinv) % 2 ** 32 == 1 and r2 == pow(2, 64, P)
     assert got["max_len"] == ["65536", "65536", "8192"]
     assert got["workspace"] == ["0"]
-    assert got["fast_workspace"] == ["0", str(3 * ((4097 * 8 * 4 + 255) // 256 * 256))]
+    assert got["fast_workspace"] == ["0", str(8 * (131072 * 8 + 64 * 8 + 8))]  # 8 rows of the four-step path
     assert got["strerror"] and got["null_args"] == ["1"]
 
 

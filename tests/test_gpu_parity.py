@@ -177,8 +177,9 @@ CLUSTER_SHAPES = [(1, 4097, 3), (2, 20000, 2), (1, 65536, 2), (2, 5000, 33)]
 @pytest.mark.parametrize("two_pass", [True, False], ids=["two_pass", "single_pass"])
 @pytest.mark.parametrize("shape", CLUSTER_SHAPES, ids=lambda s: "x".join(map(str, s)))
 def test_cluster_rows_sampled_oracle(shape, two_pass):
-    """Rows beyond one CTA: with the optional workspace (transposed rows) and
-    without it (rows read straight from the channel-last tensors)."""
+    """Rows beyond one CTA: with the optional workspace (the four-step path)
+    and without it (8-CTA cluster rows read straight from the channel-last
+    tensors)."""
     import torch
     import spectral_sequence_mixing_b200 as ssm
     B, L, D = shape
@@ -195,6 +196,79 @@ def test_cluster_rows_sampled_oracle(shape, two_pass):
     r_ref, den = oracle.causal_conv_points(v, g, pts)
     n_bad, worst = float_violations(r[pts[:, 0], pts[:, 1], pts[:, 2]], r_ref, den, F32_TOL)
     assert n_bad == 0, f"{n_bad} violations, worst ratio {worst:.3g}"
+
+
+# Four-step shapes: ragged channel tiles of 32 ((3, 5000, 50), (5, 4097, 27)),
+# a partial mid-pass group of 8 rows ((1, 8192, 130), (16, 4100, 9) with 144
+# rows), L past several 512-step columns and ragged in them.
+FOUR_STEP_SHAPES = [(3, 5000, 50), (1, 8192, 130), (5, 4097, 27), (16, 4100, 9)]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", FOUR_STEP_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_cluster_rows_four_step_and_single_pass(shape, dtype):
+    """The four-step path (workspace) and the single-pass cluster rows (no
+    workspace) against the oracle on sampled outputs, fp32 and bf16."""
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    B, L, D = shape
+    rng = np.random.Generator(np.random.PCG64(11 + sum(shape)))
+    v = rng.standard_normal(shape).astype(np.float32)
+    g = (rng.standard_normal(shape) * (1.0 + np.arange(L).reshape(1, L, 1)) ** -0.75).astype(np.float32)
+    if dtype == "bf16":
+        v, g = workloads.bf16_round(v), workloads.bf16_round(g)
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    ws = torch.empty(ssm.fast_workspace_bytes(tdt, B, L, D), dtype=torch.uint8, device="cuda")
+    vd, gd = to_dev(v, dtype), to_dev(g, dtype)
+    r4 = ssm.causal_conv(vd, gd, workspace=ws)
+    r1 = ssm.causal_conv(vd, gd, workspace=torch.empty(0, dtype=torch.uint8, device="cuda"))
+    torch.cuda.synchronize()
+    pts = workloads.sample_points(B, L, D, 1024, seed=17)
+    r_ref, den = oracle.causal_conv_points(as_f32(v, dtype), as_f32(g, dtype), pts)
+    tol = F32_TOL if dtype == "f32" else BF16_TOL
+    for r in (r4, r1):
+        got = as_f32(from_dev(r, dtype), dtype) if dtype == "bf16" else from_dev(r, dtype)
+        n_bad, worst = float_violations(got[pts[:, 0], pts[:, 1], pts[:, 2]], r_ref, den, tol)
+        assert n_bad == 0, f"{n_bad} violations, worst ratio {worst:.3g}"
+
+
+def test_four_step_capture_side_stream_and_zero_rows():
+    """The four-step path on a caller's side stream and replayed from a CUDA
+    graph equals the eager default-stream call bit for bit (forward and the
+    backward's time-reversed reads and writes); rows whose v or g is all zero
+    come out exactly zero."""
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    B, L, D = 2, 6000, 72
+    rng = np.random.Generator(np.random.PCG64(31))
+    dr, v, g = (to_dev(rng.standard_normal((B, L, D)).astype(np.float32), "f32") for _ in range(3))
+    v[0, :, 5] = 0.0
+    g[1, :, 70] = 0.0
+    ws = torch.empty(ssm.fast_workspace_bytes(torch.float32, B, L, D), dtype=torch.uint8, device="cuda")
+    ref_dv, ref_dg = ssm.causal_conv_bwd(dr, v, g, workspace=ws)
+    ref_r = ssm.causal_conv(v, g, workspace=ws)
+    torch.cuda.synchronize()
+    assert not ref_r[0, :, 5].any() and not ref_r[1, :, 70].any()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    dv, dg, r = torch.empty_like(dr), torch.empty_like(dr), torch.empty_like(dr)
+    with torch.cuda.stream(s):
+        ssm.causal_conv_bwd(dr, v, g, dv=dv, dg=dg, workspace=ws, stream=s)
+        ssm.causal_conv(v, g, out=r, workspace=ws, stream=s)
+        cv, cg, cr = dv.clone(), dg.clone(), r.clone()  # consumers on the caller's stream
+    s.synchronize()
+    assert torch.equal(cv, ref_dv) and torch.equal(cg, ref_dg) and torch.equal(cr, ref_r)
+    graph = torch.cuda.CUDAGraph()
+    dv.zero_()
+    dg.zero_()
+    r.zero_()
+    with torch.cuda.graph(graph):
+        ssm.causal_conv_bwd(dr, v, g, dv=dv, dg=dg, workspace=ws, stream=torch.cuda.current_stream())
+        ssm.causal_conv(v, g, out=r, workspace=ws, stream=torch.cuda.current_stream())
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(dv, ref_dv) and torch.equal(dg, ref_dg) and torch.equal(r, ref_r)
 
 
 @pytest.mark.parametrize("name", ["large_bf16", "long_f32"])
