@@ -296,6 +296,10 @@ static cudaError_t ensure_init(int dev) {
                                       (int)kHrFwdSmem)) != cudaSuccess ||
             (e = cudaFuncSetAttribute(hr_inv_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kHrFwdSmem)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(hr_fwd_tma_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)hr_fwd_tma_smem<float>())) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(hr_fwd_tma_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)hr_fwd_tma_smem<__nv_bfloat16>())) != cudaSuccess ||
             (e = cudaFuncSetAttribute(hr_mid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kHrMidSmem)) != cudaSuccess)
             return e;
@@ -446,6 +450,26 @@ static bool encode_btd_map(CUtensorMap *m, const IO *base, int64_t B, int64_t L,
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUtensorMapDataType dt = sizeof(IO) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     return enc(m, dt, 3, const_cast<IO *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 4-D map {d, n1, n2, b} of a [B, L, D] tensor for the four-step forward
+// pass: time t = n1 + 512 n2 for the whole 512-step rows n2 < L / 512; box
+// [128 n2][1 n1][32 d].  False when the layout allows no map.
+template <typename IO>
+static bool encode_hr_map(CUtensorMap *m, const IO *base, int64_t B, int64_t L, int64_t D) {
+    const int64_t es = sizeof(IO), nb2 = L / kHrA;
+    if (((uintptr_t)base & 15) != 0 || (D * es) % 16 != 0 || nb2 < 1) return false;
+    if (D > (int64_t)UINT32_MAX || B > (int64_t)UINT32_MAX || es * D * L >= ((int64_t)1 << 40)) return false;
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)kHrA, (cuuint64_t)nb2, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)(D * es), (cuuint64_t)(kHrA * D * es), (cuuint64_t)(L * D * es)};
+    const cuuint32_t box[4] = {(cuuint32_t)kHrCG, 1, 128, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUtensorMapDataType dt = sizeof(IO) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    return enc(m, dt, 4, const_cast<IO *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -607,7 +631,7 @@ static int launch_tcconv(const __nv_bfloat16 *v, const __nv_bfloat16 *g, __nv_bf
 // inverse) in place, inverse over k2 with the stores.
 template <typename IO>
 static int launch_hbm_rows(const IO *v, const IO *g, IO *r, int64_t B, int64_t L, int64_t D, void *ws,
-                           const float2 *tw, cudaStream_t s, int rev) {
+                           const float2 *tw, cudaStream_t s, int dev, int rev) {
     const int64_t rows = B * D, tpb = (D + kHrCG - 1) / kHrCG, tiles = B * tpb;
     float2 *Y = reinterpret_cast<float2 *>(ws);
     float2 *part = reinterpret_cast<float2 *>(reinterpret_cast<char *>(ws) + hr_ws_part_off(rows));
@@ -622,8 +646,21 @@ static int launch_hbm_rows(const IO *v, const IO *g, IO *r, int64_t B, int64_t L
                                                                                          (int)rows, (int)tpb);
     }
     hr_alpha_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(part, as, (int)rows);
-    hr_fwd_kernel<IO><<<dim3((unsigned)tiles, kHrA), kHrFwdThreads, kHrFwdSmem, s>>>(v, g, Y, as, tw, (int)L, (int)D,
-                                                                                      (int)rows, (int)tpb, rev);
+    // forward reads staged by TMA where a map describes the tensors (not for
+    // the time-reversed reads of the backward pass)
+    CUtensorMap tmv, tmg;
+    memset(&tmv, 0, sizeof(tmv));
+    memset(&tmg, 0, sizeof(tmg));
+    const int64_t items = tiles * kHrA;
+    if (!(rev & 1) && items <= INT32_MAX && encode_hr_map<IO>(&tmv, v, B, L, D) && encode_hr_map<IO>(&tmg, g, B, L, D)) {
+        const int64_t grid = std::min<int64_t>(items, g_num_sms[dev]);
+        hr_fwd_tma_kernel<IO><<<(unsigned)grid, kHrFwdThreads, hr_fwd_tma_smem<IO>(), s>>>(
+            v, g, Y, as, tw, (int)L, (int)D, (int)rows, (int)tpb, (int)tiles, (int)items, tmv, tmg);
+    } else {
+        hr_fwd_kernel<IO><<<dim3((unsigned)tiles, kHrA), kHrFwdThreads, kHrFwdSmem, s>>>(v, g, Y, as, tw, (int)L,
+                                                                                          (int)D, (int)rows,
+                                                                                          (int)tpb, rev);
+    }
     hr_mid_kernel<<<dim3((unsigned)((rows + kHrRows2 - 1) / kHrRows2), kHrB / 2), kHrMidThreads, kHrMidSmem, s>>>(
         Y, tw, (int)rows);
     hr_inv_kernel<IO><<<dim3((unsigned)tiles, kHrB), kHrInvThreads, kHrFwdSmem, s>>>(Y, r, as, v, g, tw, (int)L,
@@ -653,7 +690,7 @@ static int fftconv_dispatch(const IO *v, const IO *g, IO *r, int64_t B, int64_t 
         const size_t fast = fast_ws_bytes(sizeof(IO) == 4 ? CC_DTYPE_F32 : CC_DTYPE_BF16, B, L, D);
         if (ws == nullptr || fast == 0 || ws_bytes < fast || (reinterpret_cast<uintptr_t>(ws) & 15) != 0)
             return launch_big<BigX<IO>, kMinbBigX>(v, g, r, B, L, D, (const float2 *)tws[3], s, rev, 0);
-        return launch_hbm_rows<IO>(v, g, r, B, L, D, ws, (const float2 *)tws[5], s, rev);
+        return launch_hbm_rows<IO>(v, g, r, B, L, D, ws, (const float2 *)tws[5], s, dev, rev);
     }
     return CC_ERR_UNSUPPORTED;
 }

@@ -43,6 +43,7 @@
 
 #include "fft_reg.cuh"
 #include "fftconv_fused.cuh"  // IO_t, spectral_product, kHeadT0
+#include "tma.cuh"
 
 namespace ccv {
 
@@ -244,6 +245,110 @@ __global__ void __launch_bounds__(kHrFwdThreads, 2)
             const int k2 = c + 16 * dd;
             Y[((int64_t)k2 * kHrA + n1) * rows + row] = cmul(cmul(y[dd], o1), __ldg(tw + kHrTO2 + n1 * 16 + dd));
         }
+    }
+}
+
+// The forward pass with its inputs staged by TMA (forward calls, D * element
+// size a multiple of 16 bytes, aligned tensors): persistent CTAs, one per SM,
+// walk the (n1, channel tile) items (consecutive CTAs share n1, so together
+// they read whole runs of adjacent time steps); one thread keeps the inputs
+// of the next kHrFwdStages - 1 items in flight as TMA boxes
+// [128 n2][1 n1][32 d] of the 4-D maps {d, n1, n2, b} of v and g (zero fill
+// past D and past the last whole 512-step row; the ragged row of a length
+// that is not a multiple of 512 is read directly), so the loads of later
+// items overlap the transforms of the current one.
+constexpr int kHrFwdStages = 3;
+constexpr size_t kHrFwdXBytes = (size_t)kHrCG * kHrSP * 8;  // exchange buffer, a multiple of 128 bytes
+template <typename IO>
+constexpr size_t hr_fwd_stage_elems() { return (size_t)2 * 128 * kHrCG; }
+template <typename IO>
+constexpr size_t hr_fwd_tma_smem() {
+    return kHrFwdXBytes + kHrFwdStages * hr_fwd_stage_elems<IO>() * sizeof(IO) + 8 * kHrFwdStages;
+}
+
+template <typename IO>
+__global__ void __launch_bounds__(kHrFwdThreads, 1)
+    hr_fwd_tma_kernel(const IO *__restrict__ v, const IO *__restrict__ g, float2 *__restrict__ Y,
+                      const float2 *__restrict__ as, const float2 *__restrict__ tw, int L, int D, int rows,
+                      int tiles_per_batch, int ntiles, int items, const __grid_constant__ CUtensorMap tmv,
+                      const __grid_constant__ CUtensorMap tmg) {
+    extern __shared__ __align__(128) unsigned char hr_raw[];
+    constexpr int S = kHrFwdStages;
+    constexpr int SE = (int)hr_fwd_stage_elems<IO>();  // IO elements per stage: v then g, [n2][d]
+    float2 *xs = reinterpret_cast<float2 *>(hr_raw);
+    IO *stg = reinterpret_cast<IO *>(hr_raw + kHrFwdXBytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(hr_raw + kHrFwdXBytes + (size_t)S * SE * sizeof(IO));
+    const int tid = threadIdx.x, lane = tid & 31, a = tid >> 5;
+    const int nb2 = L / kHrA;  // whole 512-step rows the maps cover
+    if (tid == 0)
+        for (int q = 0; q < S; ++q) mbar_init(full + q, 1);
+    __syncthreads();
+    auto item_at = [&](int j) { return (int)blockIdx.x + j * (int)gridDim.x; };
+    auto issue = [&](int item, int q) {
+        const int n1 = item / ntiles, tile = item - n1 * ntiles;
+        const int b = tile / tiles_per_batch, d0 = (tile - b * tiles_per_batch) * kHrCG;
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(full + q, (unsigned)(SE * sizeof(IO)));
+        tma_load_4d(stg + q * SE, &tmv, d0, n1, 0, b, full + q);
+        tma_load_4d(stg + q * SE + SE / 2, &tmg, d0, n1, 0, b, full + q);
+    };
+    if (tid == 0)
+        for (int j = 0; j < S - 1; ++j)
+            if (item_at(j) < items) issue(item_at(j), j);
+    float2 *col = xs + lane * kHrSP;
+    for (int j = 0; item_at(j) < items; ++j) {
+        const int item = item_at(j), q = j % S;
+        // the stage of item j + S - 1 was last read in iteration j - 1, before its barriers
+        if (tid == 0 && item_at(j + S - 1) < items) issue(item_at(j + S - 1), (j + S - 1) % S);
+        const bool got = mbar_wait_bounded(full + q, (unsigned)((j / S) & 1));
+        if (!__syncthreads_and(got)) {
+            // a copy did not arrive in time: flag it, give the copies in flight
+            // one more bounded wait each, and stop
+            if (tid == 0) {
+                atomicOr(&g_cc_fault, kFaultTmaWait);
+                for (int k = j; k < j + S && item_at(k) < items; ++k) mbar_wait_bounded(full + k % S, (unsigned)((k / S) & 1));
+            }
+            return;
+        }
+        const int n1 = item / ntiles, tile = item - n1 * ntiles;
+        const int b = tile / tiles_per_batch, d = (tile - b * tiles_per_batch) * kHrCG + lane;
+        const bool ok = d < D;
+        const int64_t row = (int64_t)b * D + d;
+        const int64_t base = (int64_t)b * L * D + d;
+        const float alpha = ok ? as[row].x : 1.f;
+        const IO *sv = stg + q * SE, *sg = sv + SE / 2;
+        float2 x[16];
+#pragma unroll
+        for (int bb = 0; bb < 8; ++bb) {
+            const int n2 = a + 16 * bb;
+            const int t = n1 + kHrA * n2;
+            float2 z = make_float2(0.f, 0.f);
+            if (n2 < nb2) {
+                z = make_float2(IO_t<IO>::cvt(sv[n2 * kHrCG + lane]), alpha * IO_t<IO>::cvt(sg[n2 * kHrCG + lane]));
+            } else if (ok && t < L) {
+                z = make_float2(IO_t<IO>::cvt(IO_t<IO>::ld(v + base + (int64_t)t * D)),
+                                alpha * IO_t<IO>::cvt(IO_t<IO>::ld(g + base + (int64_t)t * D)));
+            }
+            x[bitrev(bb, 4)] = cmul(z, __ldg(tw + kHrTW1 + n2));
+        }
+        fft_dit<16, false, true>(x);  // x[c]
+#pragma unroll
+        for (int c = 0; c < 16; ++c) col[c * 16 + a] = cmul(x[c], __ldg(tw + kHrTA + a * 16 + c));
+        __syncthreads();  // exchange written; stage q free
+        const int c = a;
+        float2 y[16];
+#pragma unroll
+        for (int aa = 0; aa < 16; ++aa) y[bitrev(aa, 4)] = col[c * 16 + aa];
+        fft_dit<16, false>(y);  // y[dd]: k2 = c + 16 dd
+        if (ok) {
+            const float2 o1 = __ldg(tw + kHrTO1 + n1 * 16 + c);
+#pragma unroll
+            for (int dd = 0; dd < 16; ++dd) {
+                const int k2 = c + 16 * dd;
+                Y[((int64_t)k2 * kHrA + n1) * rows + row] = cmul(cmul(y[dd], o1), __ldg(tw + kHrTO2 + n1 * 16 + dd));
+            }
+        }
+        __syncthreads();  // exchange read before the next item writes it
     }
 }
 
