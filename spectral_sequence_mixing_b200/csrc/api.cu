@@ -456,7 +456,7 @@ static bool encode_btd_map(CUtensorMap *m, const IO *base, int64_t B, int64_t L,
 
 // 4-D map {d, n1, n2, b} of a [B, L, D] tensor for the four-step forward
 // pass: time t = n1 + 512 n2 for the whole 512-step rows n2 < L / 512; box
-// [128 n2][1 n1][32 d].  False when the layout allows no map.
+// [128 n2][1 n1][16 d].  False when the layout allows no map.
 template <typename IO>
 static bool encode_hr_map(CUtensorMap *m, const IO *base, int64_t B, int64_t L, int64_t D) {
     const int64_t es = sizeof(IO), nb2 = L / kHrA;
@@ -466,7 +466,7 @@ static bool encode_hr_map(CUtensorMap *m, const IO *base, int64_t B, int64_t L, 
     if (!enc) return false;
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)kHrA, (cuuint64_t)nb2, (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)(D * es), (cuuint64_t)(kHrA * D * es), (cuuint64_t)(L * D * es)};
-    const cuuint32_t box[4] = {(cuuint32_t)kHrCG, 1, 128, 1};
+    const cuuint32_t box[4] = {(cuuint32_t)kHrFwdCG, 1, 128, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUtensorMapDataType dt = sizeof(IO) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     return enc(m, dt, 4, const_cast<IO *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -651,11 +651,11 @@ static int launch_hbm_rows(const IO *v, const IO *g, IO *r, int64_t B, int64_t L
     CUtensorMap tmv, tmg;
     memset(&tmv, 0, sizeof(tmv));
     memset(&tmg, 0, sizeof(tmg));
-    const int64_t items = tiles * kHrA;
+    const int64_t tpb16 = (D + kHrFwdCG - 1) / kHrFwdCG, tiles16 = B * tpb16, items = tiles16 * kHrA;
     if (!(rev & 1) && items <= INT32_MAX && encode_hr_map<IO>(&tmv, v, B, L, D) && encode_hr_map<IO>(&tmg, g, B, L, D)) {
-        const int64_t grid = std::min<int64_t>(items, g_num_sms[dev]);
-        hr_fwd_tma_kernel<IO><<<(unsigned)grid, kHrFwdThreads, hr_fwd_tma_smem<IO>(), s>>>(
-            v, g, Y, as, tw, (int)L, (int)D, (int)rows, (int)tpb, (int)tiles, (int)items, tmv, tmg);
+        const int64_t grid = std::min<int64_t>(items, 2 * (int64_t)g_num_sms[dev]);
+        hr_fwd_tma_kernel<IO><<<(unsigned)grid, kHrFwdTmaThreads, hr_fwd_tma_smem<IO>(), s>>>(
+            v, g, Y, as, tw, (int)L, (int)D, (int)rows, (int)tpb16, (int)tiles16, (int)items, tmv, tmg);
     } else {
         hr_fwd_kernel<IO><<<dim3((unsigned)tiles, kHrA), kHrFwdThreads, kHrFwdSmem, s>>>(v, g, Y, as, tw, (int)L,
                                                                                           (int)D, (int)rows,

@@ -249,36 +249,39 @@ __global__ void __launch_bounds__(kHrFwdThreads, 2)
 }
 
 // The forward pass with its inputs staged by TMA (forward calls, D * element
-// size a multiple of 16 bytes, aligned tensors): persistent CTAs, one per SM,
-// walk the (n1, channel tile) items (consecutive CTAs share n1, so together
-// they read whole runs of adjacent time steps); one thread keeps the inputs
-// of the next kHrFwdStages - 1 items in flight as TMA boxes
-// [128 n2][1 n1][32 d] of the 4-D maps {d, n1, n2, b} of v and g (zero fill
+// size a multiple of 16 bytes, aligned tensors): persistent CTAs, two per SM,
+// walk the (n1, 16-channel tile) items (consecutive CTAs share n1, so
+// together they read whole runs of adjacent time steps); one thread keeps the
+// inputs of the next kHrFwdStages - 1 items in flight as TMA boxes
+// [128 n2][1 n1][16 d] of the 4-D maps {d, n1, n2, b} of v and g (zero fill
 // past D and past the last whole 512-step row; the ragged row of a length
 // that is not a multiple of 512 is read directly), so the loads of later
 // items overlap the transforms of the current one.
 constexpr int kHrFwdStages = 3;
-constexpr size_t kHrFwdXBytes = (size_t)kHrCG * kHrSP * 8;  // exchange buffer, a multiple of 128 bytes
+constexpr int kHrFwdCG = 16;        // channels per CTA of the TMA forward pass (half a warp)
+constexpr int kHrFwdTmaThreads = 256;
+constexpr size_t kHrFwdXBytes = (size_t)kHrFwdCG * kHrSP * 8;  // exchange buffer, a multiple of 128 bytes
 template <typename IO>
-constexpr size_t hr_fwd_stage_elems() { return (size_t)2 * 128 * kHrCG; }
+constexpr size_t hr_fwd_stage_elems() { return (size_t)2 * 128 * kHrFwdCG; }
 template <typename IO>
 constexpr size_t hr_fwd_tma_smem() {
     return kHrFwdXBytes + kHrFwdStages * hr_fwd_stage_elems<IO>() * sizeof(IO) + 8 * kHrFwdStages;
 }
 
 template <typename IO>
-__global__ void __launch_bounds__(kHrFwdThreads, 1)
+__global__ void __launch_bounds__(kHrFwdTmaThreads, 2)
     hr_fwd_tma_kernel(const IO *__restrict__ v, const IO *__restrict__ g, float2 *__restrict__ Y,
                       const float2 *__restrict__ as, const float2 *__restrict__ tw, int L, int D, int rows,
                       int tiles_per_batch, int ntiles, int items, const __grid_constant__ CUtensorMap tmv,
                       const __grid_constant__ CUtensorMap tmg) {
     extern __shared__ __align__(128) unsigned char hr_raw[];
-    constexpr int S = kHrFwdStages;
+    constexpr int S = kHrFwdStages, CG = kHrFwdCG;
     constexpr int SE = (int)hr_fwd_stage_elems<IO>();  // IO elements per stage: v then g, [n2][d]
     float2 *xs = reinterpret_cast<float2 *>(hr_raw);
     IO *stg = reinterpret_cast<IO *>(hr_raw + kHrFwdXBytes);
     uint64_t *full = reinterpret_cast<uint64_t *>(hr_raw + kHrFwdXBytes + (size_t)S * SE * sizeof(IO));
-    const int tid = threadIdx.x, lane = tid & 31, a = tid >> 5;
+    // thread (a, channel): half-warp a = tid / 16 (step A: digit a; step B: digit c), channel tid % 16
+    const int tid = threadIdx.x, ch = tid & (CG - 1), a = tid / CG;
     const int nb2 = L / kHrA;  // whole 512-step rows the maps cover
     if (tid == 0)
         for (int q = 0; q < S; ++q) mbar_init(full + q, 1);
@@ -286,7 +289,7 @@ __global__ void __launch_bounds__(kHrFwdThreads, 1)
     auto item_at = [&](int j) { return (int)blockIdx.x + j * (int)gridDim.x; };
     auto issue = [&](int item, int q) {
         const int n1 = item / ntiles, tile = item - n1 * ntiles;
-        const int b = tile / tiles_per_batch, d0 = (tile - b * tiles_per_batch) * kHrCG;
+        const int b = tile / tiles_per_batch, d0 = (tile - b * tiles_per_batch) * CG;
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(full + q, (unsigned)(SE * sizeof(IO)));
         tma_load_4d(stg + q * SE, &tmv, d0, n1, 0, b, full + q);
@@ -295,7 +298,7 @@ __global__ void __launch_bounds__(kHrFwdThreads, 1)
     if (tid == 0)
         for (int j = 0; j < S - 1; ++j)
             if (item_at(j) < items) issue(item_at(j), j);
-    float2 *col = xs + lane * kHrSP;
+    float2 *col = xs + ch * kHrSP;
     for (int j = 0; item_at(j) < items; ++j) {
         const int item = item_at(j), q = j % S;
         // the stage of item j + S - 1 was last read in iteration j - 1, before its barriers
@@ -306,12 +309,13 @@ __global__ void __launch_bounds__(kHrFwdThreads, 1)
             // one more bounded wait each, and stop
             if (tid == 0) {
                 atomicOr(&g_cc_fault, kFaultTmaWait);
-                for (int k = j; k < j + S && item_at(k) < items; ++k) mbar_wait_bounded(full + k % S, (unsigned)((k / S) & 1));
+                for (int k = j; k < j + S && item_at(k) < items; ++k)
+                    mbar_wait_bounded(full + k % S, (unsigned)((k / S) & 1));
             }
             return;
         }
         const int n1 = item / ntiles, tile = item - n1 * ntiles;
-        const int b = tile / tiles_per_batch, d = (tile - b * tiles_per_batch) * kHrCG + lane;
+        const int b = tile / tiles_per_batch, d = (tile - b * tiles_per_batch) * CG + ch;
         const bool ok = d < D;
         const int64_t row = (int64_t)b * D + d;
         const int64_t base = (int64_t)b * L * D + d;
@@ -324,7 +328,7 @@ __global__ void __launch_bounds__(kHrFwdThreads, 1)
             const int t = n1 + kHrA * n2;
             float2 z = make_float2(0.f, 0.f);
             if (n2 < nb2) {
-                z = make_float2(IO_t<IO>::cvt(sv[n2 * kHrCG + lane]), alpha * IO_t<IO>::cvt(sg[n2 * kHrCG + lane]));
+                z = make_float2(IO_t<IO>::cvt(sv[n2 * CG + ch]), alpha * IO_t<IO>::cvt(sg[n2 * CG + ch]));
             } else if (ok && t < L) {
                 z = make_float2(IO_t<IO>::cvt(IO_t<IO>::ld(v + base + (int64_t)t * D)),
                                 alpha * IO_t<IO>::cvt(IO_t<IO>::ld(g + base + (int64_t)t * D)));
