@@ -257,6 +257,17 @@ __global__ void __launch_bounds__(kHrFwdThreads, 2)
 // past D and past the last whole 512-step row; the ragged row of a length
 // that is not a multiple of 512 is read directly), so the loads of later
 // items overlap the transforms of the current one.
+// 4-D tiled TMA load of one box into shared memory, completing on `bar`.
+// x (innermost) * element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, int x, int y, int z, int w,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+        "%5}], [%6];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+        : "memory");
+}
+
 constexpr int kHrFwdStages = 3;
 constexpr int kHrFwdCG = 16;        // channels per CTA of the TMA forward pass (half a warp)
 constexpr int kHrFwdTmaThreads = 256;
