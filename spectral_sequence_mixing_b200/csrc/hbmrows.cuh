@@ -33,7 +33,7 @@
 // Rows are innermost in the workspace, so every pass reads and writes whole
 // runs of adjacent channels (a channel-last tensor's rows are its channels):
 // the fwd and inv passes take 32 channels per CTA (one per lane), the mid
-// pass 8 rows per CTA (one per warp), staged through shared memory.
+// pass kHrRows2 rows per CTA (one per warp), staged through shared memory.
 //
 // Each sub-transform is a two-level decomposition inside a CTA: register
 // DFTs of 8, 16 or 32 points (fft_reg.cuh) with one shared-memory exchange.
@@ -52,16 +52,17 @@ constexpr int kHrA = 512;             // n = n1 + A n2; k = k2 + kHrB k1
 constexpr int kHrB = 256;
 constexpr int kHrLMAX = kHrN / 2;     // longest row
 constexpr int kHrCG = 32;             // channels per fwd / inv CTA (one per lane)
-constexpr int kHrRows2 = 8;           // rows per mid CTA (one per warp)
+constexpr int kHrRows2 = 4;           // rows per mid CTA (one per warp)
 constexpr int kHrSlices = 64;         // time slices of the norm pass
 constexpr int kHrSliceT = kHrLMAX / kHrSlices;
 constexpr int kHrSP = 257;            // fwd / inv shared-memory column pitch (float2)
 constexpr int kHrColM = 576;          // mid: one 512-point column (pitch-18 groups of 16 after the first step)
-constexpr int kHrRowM = 2 * kHrColM + 2;  // mid: one row's two columns (pitch = 2 mod 16: conflict-free loads)
-constexpr int kHrFwdThreads = 512, kHrMidThreads = 256, kHrInvThreads = 512, kHrNormThreads = 128;
+constexpr int kHrRowM = 2 * kHrColM + 4;  // mid: one row's two columns (pitch = 4 mod 16: conflict-free loads)
+constexpr int kHrFwdThreads = 512, kHrMidThreads = 32 * kHrRows2, kHrInvThreads = 512, kHrNormThreads = 128;
 constexpr size_t kHrFwdSmem = (size_t)kHrCG * kHrSP * 8;
-constexpr size_t kHrMidStage = (size_t)2 * kHrB * 9;  // float2: [sel][m1] x 9 (8 rows + pad)
-constexpr size_t kHrMidSmem = ((size_t)kHrRows2 * kHrRowM + kHrMidStage) * 8;
+constexpr int kHrMidSP = kHrRows2 + 1;  // mid output staging pitch: [sel][m1][rows + pad], over the row area
+constexpr size_t kHrMidSmem = (size_t)kHrRows2 * kHrRowM * 8;
+static_assert((size_t)2 * kHrB * kHrMidSP <= (size_t)kHrRows2 * kHrRowM, "output staging fits the row area");
 
 // Twiddle table (float2, built on the host in fp64); theta = exp(-i pi / N),
 // omega_R = exp(-2 pi i / R), phi = theta^2.
@@ -368,9 +369,10 @@ __global__ void __launch_bounds__(kHrFwdTmaThreads, 2)
 }
 
 // ---------------------------------------------------------------- mid
-// grid (row groups of 8, k2 pairs kp < 128: k2a = kp, k2b = 255 - kp).
+// grid (row groups of kHrRows2, k2 pairs kp < 128: k2a = kp, k2b = 255 - kp).
 // Shared memory: per row (warp) two columns (sel = 0: k2a, 1: k2b) of
-// kHrColM float2, then the output staging [sel][m1][8 rows (+1 pad)].
+// kHrColM float2; at the end the output staging [sel][m1][rows (+1 pad)]
+// over the same space.
 // Within a warp (its row), n1 = p + 16 q and k1 = u + 32 s:
 //   step A  lane (sel, p): 32-point DFT over q -> u, times omega_512^(p u);
 //           stored at [u * 18 + p] (16-byte aligned pairs for step B);
@@ -382,10 +384,10 @@ __global__ void __launch_bounds__(kHrFwdTmaThreads, 2)
 //   step C  lane (sel, al, h): 16-point inverse over u = 2 i + h, the
 //           radix-2 combination with the partner lane (h ^ 1) -> be, times
 //           phi^-(m1 (2 k2 + 1)); staged, then stored with rows innermost.
-__global__ void __launch_bounds__(kHrMidThreads, 2) hr_mid_kernel(float2 *__restrict__ Y,
+__global__ void __launch_bounds__(kHrMidThreads, 16 / kHrRows2) hr_mid_kernel(float2 *__restrict__ Y,
                                                                   const float2 *__restrict__ tw, int rows) {
     extern __shared__ float2 hr_sm[];
-    float2 *stage = hr_sm + kHrRows2 * kHrRowM;
+    float2 *stage = hr_sm;  // output staging, written once every warp is done with its row
     const int tid = threadIdx.x, lane = tid & 31, r8 = tid >> 5;
     const int64_t row0 = (int64_t)blockIdx.x * kHrRows2;
     const int kp = blockIdx.y, k2a = kp, k2b = kHrB - 1 - kp;
@@ -393,7 +395,7 @@ __global__ void __launch_bounds__(kHrMidThreads, 2) hr_mid_kernel(float2 *__rest
     // n1 = tid / 8 + 32 j), each column's 16 loads issued before their stores
     {
         constexpr int PER = kHrA * kHrRows2 / kHrMidThreads;  // loads per thread and column
-        const int r = tid & (kHrRows2 - 1), nb = tid >> 3;
+        const int r = tid & (kHrRows2 - 1), nb = tid / kHrRows2;
         const bool rok = row0 + r < rows;
 #pragma unroll
         for (int sel = 0; sel < 2; ++sel) {
@@ -401,9 +403,10 @@ __global__ void __launch_bounds__(kHrMidThreads, 2) hr_mid_kernel(float2 *__rest
             float2 buf[PER];
 #pragma unroll
             for (int j = 0; j < PER; ++j)
-                buf[j] = rok ? src[(int64_t)(nb + 32 * j) * rows] : make_float2(0.f, 0.f);
+                buf[j] = rok ? src[(int64_t)(nb + (kHrMidThreads / kHrRows2) * j) * rows] : make_float2(0.f, 0.f);
 #pragma unroll
-            for (int j = 0; j < PER; ++j) hr_sm[r * kHrRowM + sel * kHrColM + nb + 32 * j] = buf[j];
+            for (int j = 0; j < PER; ++j)
+                hr_sm[r * kHrRowM + sel * kHrColM + nb + (kHrMidThreads / kHrRows2) * j] = buf[j];
         }
     }
     __syncthreads();
@@ -486,6 +489,8 @@ __global__ void __launch_bounds__(kHrMidThreads, 2) hr_mid_kernel(float2 *__rest
     }
     __syncwarp();
     // ---- step C: lane (sel, al, h)
+    float2 out[16];
+    const int csel = lane >> 4, cal = (lane >> 1) & 7, ch = lane & 1;
     {
         const int sel = lane >> 4, al = (lane >> 1) & 7, h = lane & 1;
         const int k2 = sel ? k2b : k2a;
@@ -496,7 +501,6 @@ __global__ void __launch_bounds__(kHrMidThreads, 2) hr_mid_kernel(float2 *__rest
         fft_dit<16, true>(x);  // E (h = 0) or O (h = 1) at be' < 16
         const float sg1 = h ? -1.f : 1.f;
         const float2 twa = __ldg(tw + kHrTWa + k2 * 8 + al);
-        float2 *st = stage + (size_t)sel * kHrB * 9 + r8;
         const float4 *tb4 = reinterpret_cast<const float4 *>(tw + kHrTWb + k2 * 32 + 16 * h);
         float2 twb[16];
 #pragma unroll
@@ -511,16 +515,22 @@ __global__ void __launch_bounds__(kHrMidThreads, 2) hr_mid_kernel(float2 *__rest
             if (h && bq > 0) mine = cmul_conj(mine, tw_const(bq, 32));  // O times omega_32^-be'
             const float2 other = shfl_xor2(mine, 1);
             const float2 o = make_float2(fmaf(sg1, mine.x, other.x), fmaf(sg1, mine.y, other.y));
-            const int be = bq + 16 * h, m1 = al + 8 * be;
-            st[m1 * 9] = cmul(cmul(o, twa), twb[bq]);
+            out[bq] = cmul(cmul(o, twa), twb[bq]);
         }
+    }
+    __syncthreads();  // every warp is done with its row: the staging may overwrite them
+    {
+        float2 *st = stage + (size_t)csel * kHrB * kHrMidSP + r8;
+#pragma unroll
+        for (int bq = 0; bq < 16; ++bq) st[(cal + 8 * (bq + 16 * ch)) * kHrMidSP] = out[bq];
     }
     __syncthreads();
     // W[k2][m1][row0 + r] over the first 256 slots of each k2 block of Y
     for (int e = tid; e < 2 * kHrB * kHrRows2; e += kHrMidThreads) {
-        const int r = e & (kHrRows2 - 1), m1 = (e >> 3) & (kHrB - 1), sel = e >> 11;
+        const int r = e & (kHrRows2 - 1), m1 = (e / kHrRows2) & (kHrB - 1), sel = e / (kHrRows2 * kHrB);
         const int k2 = sel ? k2b : k2a;
-        if (row0 + r < rows) Y[((int64_t)k2 * kHrA + m1) * rows + row0 + r] = stage[((size_t)sel * kHrB + m1) * 9 + r];
+        if (row0 + r < rows)
+            Y[((int64_t)k2 * kHrA + m1) * rows + row0 + r] = stage[((size_t)sel * kHrB + m1) * kHrMidSP + r];
     }
 }
 
