@@ -198,10 +198,15 @@ def test_cluster_rows_sampled_oracle(shape, two_pass):
     assert n_bad == 0, f"{n_bad} violations, worst ratio {worst:.3g}"
 
 
-# Four-step shapes: ragged channel tiles of 32 ((3, 5000, 50), (5, 4097, 27)),
-# a partial mid-pass group of 8 rows ((1, 8192, 130), (16, 4100, 9) with 144
-# rows), L past several 512-step columns and ragged in them.
-FOUR_STEP_SHAPES = [(3, 5000, 50), (1, 8192, 130), (5, 4097, 27), (16, 4100, 9)]
+# Four-step shapes: ragged channel tiles ((3, 5000, 50), (5, 4097, 27)), a
+# partial mid-pass group of rows ((1, 8192, 130), (16, 4100, 9) with 144
+# rows), L past several 512-step columns and ragged in them; rows whose
+# D * element size is a multiple of 16 bytes take the TMA forward pass and the
+# 16-byte norm loads: (2, 6000, 72) (two batches, a partial 16-channel tile, a
+# ragged last 512-step row read directly), (3, 4608, 20) (L a whole number of
+# 512-step rows), (1, 8192, 40).
+FOUR_STEP_SHAPES = [(3, 5000, 50), (1, 8192, 130), (5, 4097, 27), (16, 4100, 9), (2, 6000, 72), (3, 4608, 20),
+                    (1, 8192, 40)]
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
@@ -229,6 +234,38 @@ def test_cluster_rows_four_step_and_single_pass(shape, dtype):
     for r in (r4, r1):
         got = as_f32(from_dev(r, dtype), dtype) if dtype == "bf16" else from_dev(r, dtype)
         n_bad, worst = float_violations(got[pts[:, 0], pts[:, 1], pts[:, 2]], r_ref, den, tol)
+        assert n_bad == 0, f"{n_bad} violations, worst ratio {worst:.3g}"
+
+
+def test_four_step_misaligned_workspace_and_inputs():
+    """A workspace that is not 16-byte aligned selects the single-pass path;
+    inputs at a 4-byte offset (no tensor map) take the direct-load forward
+    pass and the per-channel norm loads; both agree with the oracle."""
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    B, L, D = 1, 5000, 64
+    rng = np.random.Generator(np.random.PCG64(77))
+    v = rng.standard_normal((B, L, D)).astype(np.float32)
+    g = (rng.standard_normal((B, L, D)) * (1.0 + np.arange(L).reshape(1, L, 1)) ** -0.75).astype(np.float32)
+    n_ws = ssm.fast_workspace_bytes(torch.float32, B, L, D)
+    big = torch.empty(n_ws + 64, dtype=torch.uint8, device="cuda")
+    pts = workloads.sample_points(B, L, D, 1024, seed=19)
+    r_ref, den = oracle.causal_conv_points(v, g, pts)
+    vd, gd = to_dev(v, "f32"), to_dev(g, "f32")
+    # unaligned inputs: the same values one float past a 16-byte boundary
+    vbuf = torch.empty(v.size + 1, dtype=torch.float32, device="cuda")
+    gbuf = torch.empty(v.size + 1, dtype=torch.float32, device="cuda")
+    vu = vbuf[1:].view(B, L, D)
+    gu = gbuf[1:].view(B, L, D)
+    vu.copy_(vd)
+    gu.copy_(gd)
+    outs = [ssm.causal_conv(vd, gd, workspace=big[8:8 + n_ws]),      # misaligned workspace: single pass
+            ssm.causal_conv(vu, gu, workspace=big[:n_ws]),          # four-step, direct loads
+            ssm.causal_conv(vd, gd, workspace=big[:n_ws])]          # four-step, TMA forward pass
+    torch.cuda.synchronize()
+    for r in outs:
+        got = from_dev(r, "f32")
+        n_bad, worst = float_violations(got[pts[:, 0], pts[:, 1], pts[:, 2]], r_ref, den, F32_TOL)
         assert n_bad == 0, f"{n_bad} violations, worst ratio {worst:.3g}"
 
 
