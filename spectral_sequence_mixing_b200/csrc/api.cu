@@ -652,7 +652,9 @@ static int launch_hbm_rows(const IO *v, const IO *g, IO *r, int64_t B, int64_t L
     memset(&tmv, 0, sizeof(tmv));
     memset(&tmg, 0, sizeof(tmg));
     const int64_t tpb16 = (D + kHrFwdCG - 1) / kHrFwdCG, tiles16 = B * tpb16, items = tiles16 * kHrA;
-    if (!(rev & 1) && items <= INT32_MAX && encode_hr_map<IO>(&tmv, v, B, L, D) && encode_hr_map<IO>(&tmg, g, B, L, D)) {
+    // (item indices of the persistent loop stay below INT32_MAX, lookahead included)
+    if (!(rev & 1) && items <= INT32_MAX - 8 * (int64_t)g_num_sms[dev] && encode_hr_map<IO>(&tmv, v, B, L, D) &&
+        encode_hr_map<IO>(&tmg, g, B, L, D)) {
         const int64_t grid = std::min<int64_t>(items, 2 * (int64_t)g_num_sms[dev]);
         hr_fwd_tma_kernel<IO><<<(unsigned)grid, kHrFwdTmaThreads, hr_fwd_tma_smem<IO>(), s>>>(
             v, g, Y, as, tw, (int)L, (int)D, (int)rows, (int)tpb16, (int)tiles16, (int)items, tmv, tmg);
