@@ -204,9 +204,9 @@ def test_cluster_rows_sampled_oracle(shape, two_pass):
 # D * element size is a multiple of 16 bytes take the TMA forward pass and the
 # 16-byte norm loads: (2, 6000, 72) (two batches, a partial 16-channel tile, a
 # ragged last 512-step row read directly), (3, 4608, 20) (L a whole number of
-# 512-step rows), (1, 8192, 40).
+# 512-step rows), (1, 8192, 40), (2, 65536, 16) (the longest rows, two batches).
 FOUR_STEP_SHAPES = [(3, 5000, 50), (1, 8192, 130), (5, 4097, 27), (16, 4100, 9), (2, 6000, 72), (3, 4608, 20),
-                    (1, 8192, 40)]
+                    (1, 8192, 40), (2, 65536, 16)]
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
@@ -432,6 +432,7 @@ def test_from_host_matches_device_path():
     for dtype, (v, g) in (("f32", _rand_float((2, 1000, 12), 1)),
                           ("f32", _rand_float((5, 300, 8), 3)),
                           ("f32", _rand_float((1, 5000, 4), 4)),
+                          ("f32", _rand_float((3, 4500, 8), 6)),  # long rows in batch pieces: four-step per piece
                           ("i32", tuple(rng.integers(-128, 128, (2, 700, 8)).astype(np.int32) for _ in range(2))),
                           ("i32", tuple(rng.integers(-128, 128, (7, 100, 4)).astype(np.int32) for _ in range(2)))):
         tv, tg = to_dev(v, dtype), to_dev(g, dtype)
