@@ -32,8 +32,9 @@
 //           scaled; r_t for t < kHeadT0 replaced by the direct sum.
 // Rows are innermost in the workspace, so every pass reads and writes whole
 // runs of adjacent channels (a channel-last tensor's rows are its channels):
-// the fwd and inv passes take 32 channels per CTA (one per lane), the mid
-// pass kHrRows2 rows per CTA (one per warp), staged through shared memory.
+// the fwd pass 16 channels per CTA with TMA-staged inputs (32, one per lane,
+// in its direct-load variant), the inv pass 32, the mid pass kHrRows2 rows per
+// CTA (one per warp), staged through shared memory.
 //
 // Each sub-transform is a two-level decomposition inside a CTA: register
 // DFTs of 8, 16 or 32 points (fft_reg.cuh) with one shared-memory exchange.
