@@ -296,9 +296,15 @@ static cudaError_t ensure_init(int dev) {
                                       (int)kHrFwdSmem)) != cudaSuccess ||
             (e = cudaFuncSetAttribute(hr_inv_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kHrFwdSmem)) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(hr_fwd_tma_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            (e = cudaFuncSetAttribute(hr_fwd_tma_kernel<float, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)hr_fwd_tma_smem<float>())) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(hr_fwd_tma_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            (e = cudaFuncSetAttribute(hr_fwd_tma_kernel<float, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)hr_fwd_tma_smem<float>())) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(hr_fwd_tma_kernel<__nv_bfloat16, false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)hr_fwd_tma_smem<__nv_bfloat16>())) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(hr_fwd_tma_kernel<__nv_bfloat16, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)hr_fwd_tma_smem<__nv_bfloat16>())) != cudaSuccess ||
             (e = cudaFuncSetAttribute(hr_mid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kHrMidSmem)) != cudaSuccess)
@@ -646,17 +652,18 @@ static int launch_hbm_rows(const IO *v, const IO *g, IO *r, int64_t B, int64_t L
                                                                                          (int)rows, (int)tpb);
     }
     hr_alpha_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(part, as, (int)rows);
-    // forward reads staged by TMA where a map describes the tensors (not for
-    // the time-reversed reads of the backward pass)
+    // inputs staged by TMA where a map describes the tensors (v read reversed
+    // in time for the backward pass)
     CUtensorMap tmv, tmg;
     memset(&tmv, 0, sizeof(tmv));
     memset(&tmg, 0, sizeof(tmg));
     const int64_t tpb16 = (D + kHrFwdCG - 1) / kHrFwdCG, tiles16 = B * tpb16, items = tiles16 * kHrA;
     // (item indices of the persistent loop stay below INT32_MAX, lookahead included)
-    if (!(rev & 1) && items <= INT32_MAX - 8 * (int64_t)g_num_sms[dev] && encode_hr_map<IO>(&tmv, v, B, L, D) &&
+    if (items <= INT32_MAX - 8 * (int64_t)g_num_sms[dev] && encode_hr_map<IO>(&tmv, v, B, L, D) &&
         encode_hr_map<IO>(&tmg, g, B, L, D)) {
         const int64_t grid = std::min<int64_t>(items, 2 * (int64_t)g_num_sms[dev]);
-        hr_fwd_tma_kernel<IO><<<(unsigned)grid, kHrFwdTmaThreads, hr_fwd_tma_smem<IO>(), s>>>(
+        auto kern = (rev & 1) ? hr_fwd_tma_kernel<IO, true> : hr_fwd_tma_kernel<IO, false>;
+        kern<<<(unsigned)grid, kHrFwdTmaThreads, hr_fwd_tma_smem<IO>(), s>>>(
             v, g, Y, as, tw, (int)L, (int)D, (int)rows, (int)tpb16, (int)tiles16, (int)items, tmv, tmg);
     } else {
         hr_fwd_kernel<IO><<<dim3((unsigned)tiles, kHrA), kHrFwdThreads, kHrFwdSmem, s>>>(v, g, Y, as, tw, (int)L,

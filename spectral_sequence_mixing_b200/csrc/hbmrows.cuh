@@ -250,8 +250,8 @@ __global__ void __launch_bounds__(kHrFwdThreads, 2)
     }
 }
 
-// The forward pass with its inputs staged by TMA (forward calls, D * element
-// size a multiple of 16 bytes, aligned tensors): persistent CTAs, two per SM,
+// The forward pass with its inputs staged by TMA (D * element size a multiple
+// of 16 bytes, aligned tensors; REVA: v read reversed in time, the backward): persistent CTAs, two per SM,
 // walk the (n1, 16-channel tile) items (consecutive CTAs share n1, so
 // together they read whole runs of adjacent time steps); one thread keeps the
 // inputs of the next kHrFwdStages - 1 items in flight as TMA boxes
@@ -281,7 +281,7 @@ constexpr size_t hr_fwd_tma_smem() {
     return kHrFwdXBytes + kHrFwdStages * hr_fwd_stage_elems<IO>() * sizeof(IO) + 8 * kHrFwdStages;
 }
 
-template <typename IO>
+template <typename IO, bool REVA>
 __global__ void __launch_bounds__(kHrFwdTmaThreads, 2)
     hr_fwd_tma_kernel(const IO *__restrict__ v, const IO *__restrict__ g, float2 *__restrict__ Y,
                       const float2 *__restrict__ as, const float2 *__restrict__ tw, int L, int D, int rows,
@@ -305,7 +305,15 @@ __global__ void __launch_bounds__(kHrFwdTmaThreads, 2)
         const int b = tile / tiles_per_batch, d0 = (tile - b * tiles_per_batch) * CG;
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(full + q, (unsigned)(SE * sizeof(IO)));
-        tma_load_4d(stg + q * SE, &tmv, d0, n1, 0, b, full + q);
+        if constexpr (REVA) {
+            // v_(L-1-t) for t = n1 + 512 n2, n2 < 128: with L - 1 - n1 = c1 + 512 c2
+            // these are rows c2 - n2 of column c1, a box of rows c2 - 127 .. c2
+            // (row 127 - n2 of the box; rows below 0 arrive as zeros)
+            const int c = L - 1 - n1;
+            tma_load_4d(stg + q * SE, &tmv, d0, c & (kHrA - 1), (c >> 9) - 127, b, full + q);
+        } else {
+            tma_load_4d(stg + q * SE, &tmv, d0, n1, 0, b, full + q);
+        }
         tma_load_4d(stg + q * SE + SE / 2, &tmg, d0, n1, 0, b, full + q);
     };
     if (tid == 0)
@@ -334,19 +342,30 @@ __global__ void __launch_bounds__(kHrFwdTmaThreads, 2)
         const int64_t base = (int64_t)b * L * D + d;
         const float alpha = ok ? as[row].x : 1.f;
         const IO *sv = stg + q * SE, *sg = sv + SE / 2;
+        const int c2 = (L - 1 - n1) >> 9;  // reversed reads: v_(L-1-t) sits in row c2 - n2
         float2 x[16];
 #pragma unroll
         for (int bb = 0; bb < 8; ++bb) {
             const int n2 = a + 16 * bb;
             const int t = n1 + kHrA * n2;
-            float2 z = make_float2(0.f, 0.f);
-            if (n2 < nb2) {
-                z = make_float2(IO_t<IO>::cvt(sv[n2 * CG + ch]), alpha * IO_t<IO>::cvt(sg[n2 * CG + ch]));
-            } else if (ok && t < L) {
-                z = make_float2(IO_t<IO>::cvt(IO_t<IO>::ld(v + base + (int64_t)t * D)),
-                                alpha * IO_t<IO>::cvt(IO_t<IO>::ld(g + base + (int64_t)t * D)));
+            float vv = 0.f, gg = 0.f;
+            if constexpr (REVA) {
+                const int n2v = c2 - n2;
+                if (n2v >= 0 && n2v < nb2)
+                    vv = IO_t<IO>::cvt(sv[(127 - n2) * CG + ch]);
+                else if (n2v == nb2 && ok && t < L)  // the ragged last row, read directly
+                    vv = IO_t<IO>::cvt(IO_t<IO>::ld(v + base + (int64_t)(L - 1 - t) * D));
+            } else {
+                if (n2 < nb2)
+                    vv = IO_t<IO>::cvt(sv[n2 * CG + ch]);
+                else if (ok && t < L)
+                    vv = IO_t<IO>::cvt(IO_t<IO>::ld(v + base + (int64_t)t * D));
             }
-            x[bitrev(bb, 4)] = cmul(z, __ldg(tw + kHrTW1 + n2));
+            if (n2 < nb2)
+                gg = IO_t<IO>::cvt(sg[n2 * CG + ch]);
+            else if (ok && t < L)
+                gg = IO_t<IO>::cvt(IO_t<IO>::ld(g + base + (int64_t)t * D));
+            x[bitrev(bb, 4)] = cmul(make_float2(vv, alpha * gg), __ldg(tw + kHrTW1 + n2));
         }
         fft_dit<16, false, true>(x);  // x[c]
 #pragma unroll

@@ -574,12 +574,16 @@ def test_bwd_sampled_oracle(shape):
         assert n_bad == 0, f"{name}: {n_bad} violations, worst ratio {worst:.3g}"
 
 
-@pytest.mark.parametrize("two_pass", [True, False], ids=["two_pass", "single_pass"])
-@pytest.mark.parametrize("shape", [(1, 4099, 3), (2, 9001, 2)], ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("two_pass", [True, False], ids=["four_step", "single_pass"])
+@pytest.mark.parametrize("shape", [(1, 4099, 3), (2, 9001, 2), (2, 5001, 8), (1, 4608, 16)],
+                         ids=lambda s: "x".join(map(str, s)))
 def test_bwd_cluster_rows_odd_length(shape, two_pass):
-    """Backward on cluster rows (v read and r written reversed in time) with an
-    odd length, so the last output pair of the real-output inverse is cut in
-    half; with and without the transposing workspace."""
+    """Backward on long rows (v read and r written reversed in time), with
+    and without the workspace (four-step path / cluster rows): odd lengths cut
+    the last output pair of the real-output inverse in half; D = 8 and 16
+    take the TMA forward pass with reversed reads, at a ragged length (the
+    row of the last 512 time steps read directly) and at a whole number of
+    512-step rows."""
     import torch
     import spectral_sequence_mixing_b200 as ssm
     B, L, D = shape
