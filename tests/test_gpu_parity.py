@@ -269,6 +269,27 @@ def test_four_step_misaligned_workspace_and_inputs():
         assert n_bad == 0, f"{n_bad} violations, worst ratio {worst:.3g}"
 
 
+@pytest.mark.parametrize("scale", [1e-4, 1e4])
+def test_four_step_imbalanced_streams(scale):
+    """Streams whose norms differ by ~1e8 share one complex transform only
+    after the per-row power-of-two balance (norm pass and alpha): the
+    four-step path still meets the per-element bound on sampled outputs."""
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    B, L, D = 2, 5000, 16
+    rng = np.random.Generator(np.random.PCG64(int(1 / scale) % 1000 + 3))
+    v = (rng.standard_normal((B, L, D)) / scale).astype(np.float32)
+    g = (rng.standard_normal((B, L, D)) * scale * (1.0 + np.arange(L).reshape(1, L, 1)) ** -0.75).astype(np.float32)
+    ws = torch.empty(ssm.fast_workspace_bytes(torch.float32, B, L, D), dtype=torch.uint8, device="cuda")
+    r = ssm.causal_conv(to_dev(v, "f32"), to_dev(g, "f32"), workspace=ws)
+    torch.cuda.synchronize()
+    r = from_dev(r, "f32")
+    pts = workloads.sample_points(B, L, D, 1024, seed=23)
+    r_ref, den = oracle.causal_conv_points(v, g, pts)
+    n_bad, worst = float_violations(r[pts[:, 0], pts[:, 1], pts[:, 2]], r_ref, den, F32_TOL)
+    assert n_bad == 0, f"{n_bad} violations, worst ratio {worst:.3g}"
+
+
 def test_four_step_capture_side_stream_and_zero_rows():
     """The four-step path on a caller's side stream and replayed from a CUDA
     graph equals the eager default-stream call bit for bit (forward and the
@@ -362,10 +383,11 @@ def _leak(dtype, v, g, t_c, scale, seed):
     return float(np.abs(r1[:, : t_c + 1, :].astype(np.float64) - r0[:, : t_c + 1, :]).max())
 
 
-# one representative shape per kernel: fused, channel groups, cluster rows (the
-# binding takes the two-pass path), and the NTT
+# one representative shape per kernel: fused, channel groups, long rows (the
+# binding takes the four-step path; D = 8 and 16 with TMA-staged inputs), and
+# the NTT
 DEGENERATE_CASES = [("f32", (2, 1000, 5)), ("bf16", (1, 700, 8)), ("f32", (1, 3000, 9)), ("bf16", (2, 4096, 8)),
-                    ("f32", (1, 5000, 3)), ("i32", (2, 3000, 5))]
+                    ("f32", (1, 5000, 3)), ("f32", (1, 5000, 8)), ("bf16", (1, 6000, 16)), ("i32", (2, 3000, 5))]
 
 
 @pytest.mark.parametrize("dtype,shape", DEGENERATE_CASES, ids=lambda c: str(c))
