@@ -411,8 +411,9 @@ __global__ void __launch_bounds__(kHrMidThreads, 16 / kHrRows2) hr_mid_kernel(fl
     const int tid = threadIdx.x, lane = tid & 31, r8 = tid >> 5;
     const int64_t row0 = (int64_t)blockIdx.x * kHrRows2;
     const int kp = blockIdx.y, k2a = kp, k2b = kHrB - 1 - kp;
-    // load Y[k2][n1][row0 + r] (r fastest; thread tid takes r = tid % 8 and
-    // n1 = tid / 8 + 32 j), each column's 16 loads issued before their stores
+    // load Y[k2][n1][row0 + r] (r fastest; thread tid takes r = tid % kHrRows2
+    // and n1 = tid / kHrRows2 + 32 j), each column's 16 loads issued before
+    // their stores
     {
         constexpr int PER = kHrA * kHrRows2 / kHrMidThreads;  // loads per thread and column
         const int r = tid & (kHrRows2 - 1), nb = tid / kHrRows2;
