@@ -62,18 +62,35 @@ _ONE_CTA_ROW = 4096  # rows up to this length never use the optional workspace
 
 
 def _workspace(workspace, dtype_code: int, B: int, L: int, D: int, device):
-    """(pointer, bytes) of the caller's workspace; with none given, one of the
-    optional four-step size is taken from the torch allocator when that path
-    applies.  A tensor of 0 bytes selects the single-pass path."""
+    """(pointer, bytes, tensor allocated here or None) of the workspace: the
+    caller's; with none given, one of the optional four-step size taken from
+    the torch allocator when that path applies (the single-pass path when the
+    allocator has no room for it).  A tensor of 0 bytes selects the
+    single-pass path."""
+    own = None
     if workspace is None:
         if L <= _ONE_CTA_ROW or dtype_code == CC_DTYPE_I32:
-            return None, 0
+            return None, 0, None
         n = int(load().causal_conv_fast_workspace_bytes(dtype_code, B, L, D))
         if n == 0:
-            return None, 0
-        workspace = torch.empty(n, dtype=torch.uint8, device=device)
+            return None, 0, None
+        try:
+            workspace = own = torch.empty(n, dtype=torch.uint8, device=device)
+        except torch.cuda.OutOfMemoryError:
+            return None, 0, None
     nbytes = workspace.numel() * workspace.element_size()
-    return (workspace.data_ptr() if nbytes else None), nbytes
+    return (workspace.data_ptr() if nbytes else None), nbytes, own
+
+
+def _record(stream, *tensors):
+    """Tensors allocated here (on the current stream) and handed to the
+    library's work on `stream`: tell the caching allocator, so their memory is
+    not given out again before that stream has finished with it."""
+    if stream is None:
+        return
+    for t in tensors:
+        if t is not None and stream != torch.cuda.current_stream(t.device):
+            t.record_stream(stream)
 
 
 def _run(dtype_code: int, v: torch.Tensor, g: torch.Tensor, out, workspace, stream):
@@ -83,16 +100,18 @@ def _run(dtype_code: int, v: torch.Tensor, g: torch.Tensor, out, workspace, stre
     if not v.is_cuda or not g.is_cuda or v.device != g.device:
         raise ValueError("v and g must be CUDA tensors on the same device")
     B, L, D = v.shape
-    if out is None:
+    own_out = out is None
+    if own_out:
         out = torch.empty_like(v)
     _check(out, "out", dtype, v.shape)
-    ws_ptr, ws_bytes = _workspace(workspace, dtype_code, B, L, D, v.device)
+    ws_ptr, ws_bytes, own_ws = _workspace(workspace, dtype_code, B, L, D, v.device)
     fn = getattr(load(), _FN[dtype_code])
     if v.device.index == torch.cuda.current_device():
         st = fn(v.data_ptr(), g.data_ptr(), out.data_ptr(), B, L, D, ws_ptr, ws_bytes, _stream_ptr(stream))
     else:  # the library works on the current device: switch to the tensors' one (and its stream)
         with torch.cuda.device(v.device):
             st = fn(v.data_ptr(), g.data_ptr(), out.data_ptr(), B, L, D, ws_ptr, ws_bytes, _stream_ptr(stream))
+    _record(stream, own_ws, out if own_out else None)
     if st != 0:
         raise CausalConvError(st, _FN[dtype_code])
     return out
@@ -135,16 +154,18 @@ def causal_conv_bwd(dr: torch.Tensor, v: torch.Tensor, g: torch.Tensor, dv=None,
         _check(t, name, dtype, v.shape)
         if not t.is_cuda or t.device != v.device:
             raise ValueError("dr, v, g must be CUDA tensors on the same device")
+    own = [dv is None, dg is None]
     dv = torch.empty_like(v) if dv is None else dv
     dg = torch.empty_like(v) if dg is None else dg
     _check(dv, "dv", dtype, v.shape)
     _check(dg, "dg", dtype, v.shape)
     B, L, D = v.shape
-    ws_ptr, ws_bytes = _workspace(workspace, _DT[dtype], B, L, D, v.device)
+    ws_ptr, ws_bytes, own_ws = _workspace(workspace, _DT[dtype], B, L, D, v.device)
     fn = "causal_fftconv_bwd_f32" if dtype == torch.float32 else "causal_fftconv_bwd_bf16"
     with torch.cuda.device(v.device):
         st = getattr(load(), fn)(dr.data_ptr(), v.data_ptr(), g.data_ptr(), dv.data_ptr(), dg.data_ptr(), B, L, D,
                                  ws_ptr, ws_bytes, _stream_ptr(stream))
+    _record(stream, own_ws, dv if own[0] else None, dg if own[1] else None)
     if st != 0:
         raise CausalConvError(st, fn)
     return dv, dg
@@ -165,16 +186,18 @@ def causal_conv_decode(v_cache: torch.Tensor, g_cache: torch.Tensor, t: int, out
     _check(v_cache, "v_cache", dtype)
     _check(g_cache, "g_cache", dtype, v_cache.shape)
     B, Lcap, D = v_cache.shape
-    if out is None:
+    own_out, own_ws = out is None, workspace is None
+    if own_out:
         out = torch.empty((B, D), dtype=dtype, device=v_cache.device)
     nbytes = decode_workspace_bytes(dtype, B, D, t)
-    if workspace is None:
+    if own_ws:
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=v_cache.device)
     fn = "causal_conv_decode_f32" if dtype == torch.float32 else "causal_conv_decode_bf16"
     with torch.cuda.device(v_cache.device):
         st = getattr(load(), fn)(v_cache.data_ptr(), g_cache.data_ptr(), out.data_ptr(), B, Lcap, D, int(t),
                                  workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                  _stream_ptr(stream))
+    _record(stream, workspace if own_ws else None, out if own_out else None)
     if st != 0:
         raise CausalConvError(st, fn)
     return out
@@ -194,11 +217,12 @@ def causal_conv_from_host(v_host: torch.Tensor, g_host: torch.Tensor, r_host: to
     if v_host.is_cuda or g_host.is_cuda or r_host.is_cuda:
         raise ValueError("*_host tensors must live in host memory")
     B, L, D = v_host.shape
-    ws_ptr, ws_bytes = _workspace(workspace, _DT[dtype], B, L, D, v_dev.device)
+    ws_ptr, ws_bytes, own_ws = _workspace(workspace, _DT[dtype], B, L, D, v_dev.device)
     with torch.cuda.device(v_dev.device):
         st = load().causal_conv_from_host(_DT[dtype], v_host.data_ptr(), g_host.data_ptr(), r_host.data_ptr(),
                                           v_dev.data_ptr(), g_dev.data_ptr(), r_dev.data_ptr(), B, L, D, ws_ptr,
                                           ws_bytes, _stream_ptr(stream))
+    _record(stream, own_ws)
     if st != 0:
         raise CausalConvError(st, "causal_conv_from_host")
 
@@ -262,13 +286,15 @@ def mhf_gate(a: torch.Tensor, w: torch.Tensor, bias: torch.Tensor | None, n_head
         raise ValueError("a must be a CUDA tensor")
     B, L, D = a.shape
     K = _check_gate_params(w, bias, D, n_head, a.device)
-    if out is None:
+    own_out = out is None
+    if own_out:
         out = torch.empty_like(a)
     _check(out, "out", a.dtype, a.shape)
     fn = getattr(load(), _GATE_FN[a.dtype])
     with torch.cuda.device(a.device):
         st = fn(a.data_ptr(), w.data_ptr(), bias.data_ptr() if bias is not None else None, out.data_ptr(), B, L, D,
                 n_head, K, _stream_ptr(stream))
+    _record(stream, out if own_out else None)
     if st != 0:
         raise CausalConvError(st, _GATE_FN[a.dtype])
     return out
@@ -291,10 +317,11 @@ def mhf_gated_conv(v: torch.Tensor, a: torch.Tensor, w: torch.Tensor, bias: torc
         raise ValueError("v and a must be CUDA tensors on the same device")
     B, L, D = v.shape
     K = _check_gate_params(w, bias, D, n_head, v.device)
-    if out is None:
+    own_out, own_ws = out is None, workspace is None
+    if own_out:
         out = torch.empty_like(v)
     _check(out, "out", v.dtype, v.shape)
-    if workspace is None:
+    if own_ws:
         workspace = torch.empty(mhf_gated_conv_workspace_bytes(v.dtype, B, L, D), dtype=torch.uint8,
                                 device=v.device)
     nbytes = workspace.numel() * workspace.element_size()
@@ -303,6 +330,7 @@ def mhf_gated_conv(v: torch.Tensor, a: torch.Tensor, w: torch.Tensor, bias: torc
         st = fn(v.data_ptr(), a.data_ptr(), w.data_ptr(), bias.data_ptr() if bias is not None else None,
                 out.data_ptr(), B, L, D, n_head, K, workspace.data_ptr() if nbytes else None, nbytes,
                 _stream_ptr(stream))
+    _record(stream, workspace if own_ws else None, out if own_out else None)
     if st != 0:
         raise CausalConvError(st, _GATED_FN[v.dtype])
     return out
@@ -331,13 +359,15 @@ def causal_dwconv(x: torch.Tensor, w: torch.Tensor, bias: torch.Tensor | None = 
     if bias is not None and (not isinstance(bias, torch.Tensor) or bias.dtype != torch.float32
                              or tuple(bias.shape) != (D,) or not bias.is_contiguous() or bias.device != x.device):
         raise ValueError("bias must be a contiguous float32 tensor [D] on the device of x, or None")
-    if out is None:
+    own_out = out is None
+    if own_out:
         out = torch.empty_like(x)
     _check(out, "out", x.dtype, x.shape)
     fn = getattr(load(), _DW_FN[x.dtype])
     with torch.cuda.device(x.device):
         st = fn(x.data_ptr(), w.data_ptr(), bias.data_ptr() if bias is not None else None, out.data_ptr(), B, L, D,
                 int(w.shape[1]), _stream_ptr(stream))
+    _record(stream, out if own_out else None)
     if st != 0:
         raise CausalConvError(st, _DW_FN[x.dtype])
     return out

@@ -290,6 +290,45 @@ def test_four_step_imbalanced_streams(scale):
     assert n_bad == 0, f"{n_bad} violations, worst ratio {worst:.3g}"
 
 
+def test_internal_workspace_on_a_side_stream_and_when_memory_is_short(monkeypatch):
+    """Long rows with no workspace given: the binding takes one from the torch
+    allocator and, when the call runs on another stream, records that stream
+    on it (and on the output it allocates), so memory freed on return is not
+    reused by the current stream while the call's kernels still run; when the
+    allocator has no room for the four-step workspace the single-pass path
+    runs instead.  Both agree with the oracle."""
+    import torch
+    import spectral_sequence_mixing_b200 as ssm
+    B, L, D = 1, 6000, 32
+    rng = np.random.Generator(np.random.PCG64(41))
+    v = rng.standard_normal((B, L, D)).astype(np.float32)
+    g = (rng.standard_normal((B, L, D)) * (1.0 + np.arange(L).reshape(1, L, 1)) ** -0.75).astype(np.float32)
+    vd, gd = to_dev(v, "f32"), to_dev(g, "f32")
+    pts = workloads.sample_points(B, L, D, 1024, seed=29)
+    r_ref, den = oracle.causal_conv_points(v, g, pts)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    r_side = ssm.causal_conv(vd, gd, stream=s)  # workspace and output allocated here, used on s
+    # fresh allocations on the current stream meanwhile, written at once
+    junk = [torch.full((1 << 22,), 7.0, device="cuda") for _ in range(64)]
+    s.synchronize()
+    torch.cuda.synchronize()
+    del junk
+    real_empty = torch.empty
+
+    def empty_or_oom(*args, **kw):
+        if kw.get("dtype") is torch.uint8 and args and int(args[0]) > (1 << 24):
+            raise torch.cuda.OutOfMemoryError("no room for the workspace")
+        return real_empty(*args, **kw)
+    monkeypatch.setattr(ssm.torch, "empty", empty_or_oom)
+    r_short = ssm.causal_conv(vd, gd)  # single-pass path
+    torch.cuda.synchronize()
+    for r in (r_side, r_short):
+        got = from_dev(r, "f32")
+        n_bad, worst = float_violations(got[pts[:, 0], pts[:, 1], pts[:, 2]], r_ref, den, F32_TOL)
+        assert n_bad == 0, f"{n_bad} violations, worst ratio {worst:.3g}"
+
+
 def test_four_step_capture_side_stream_and_zero_rows():
     """The four-step path on a caller's side stream and replayed from a CUDA
     graph equals the eager default-stream call bit for bit (forward and the
