@@ -108,10 +108,7 @@ static std::vector<float2> hr_twiddles() {
     for (int a = 0; a < 16; ++a)
         for (int c = 0; c < 16; ++c) t[kHrTA + a * 16 + c] = omega(a * c, 256);
     for (int n1 = 0; n1 < kHrA; ++n1)
-        for (int c = 0; c < 16; ++c) {
-            t[kHrTO1 + n1 * 16 + c] = omega((int64_t)n1 * (2 * c + 1), N2);
-            t[kHrTO2 + n1 * 16 + c] = omega((int64_t)32 * n1 * c, N2);
-        }
+        for (int k2 = 0; k2 < kHrB; ++k2) t[kHrTO + n1 * kHrB + k2] = omega((int64_t)n1 * (2 * k2 + 1), N2);
     for (int p = 0; p < 16; ++p)
         for (int u = 0; u < 32; ++u) t[kHrT512 + p * 32 + u] = omega(p * u, 512);
     for (int k2 = 0; k2 < kHrB; ++k2) t[kHrPK1 + k2] = omega(-(2 * (int64_t)k2 + 1), N2);

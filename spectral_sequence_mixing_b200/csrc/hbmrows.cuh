@@ -69,9 +69,8 @@ static_assert((size_t)2 * kHrB * kHrMidSP <= (size_t)kHrRows2 * kHrRowM, "output
 // omega_R = exp(-2 pi i / R), phi = theta^2.
 constexpr int kHrTW1 = 0;                    // [n2 < 128]           omega_512^n2
 constexpr int kHrTA = kHrTW1 + 128;          // [a * 16 + c]         omega_256^(a c)
-constexpr int kHrTO1 = kHrTA + 256;          // [n1 * 16 + c]        theta^(n1 (2c + 1))
-constexpr int kHrTO2 = kHrTO1 + kHrA * 16;   // [n1 * 16 + d]        theta^(32 n1 d)
-constexpr int kHrT512 = kHrTO2 + kHrA * 16;  // [p * 32 + u]         omega_512^(p u)
+constexpr int kHrTO = kHrTA + 256;           // [n1 * 256 + k2]      theta^(n1 (2 k2 + 1))
+constexpr int kHrT512 = kHrTO + kHrA * kHrB; // [p * 32 + u]         omega_512^(p u)
 constexpr int kHrPK1 = kHrT512 + 512;        // [k2]                 theta^-(2 k2 + 1)
 constexpr int kHrPK2 = kHrPK1 + 256;         // [u * 8 + s]          theta^-(512 u + 16384 s)
 constexpr int kHrTI = kHrPK2 + 256;          // [u * 8 + al]         exp(2 pi i u al / 256)
@@ -241,11 +240,10 @@ __global__ void __launch_bounds__(kHrFwdThreads, 2)
     for (int aa = 0; aa < 16; ++aa) y[bitrev(aa, 4)] = col[c * 16 + aa];
     fft_dit<16, false>(y);  // y[dd]: k2 = c + 16 dd
     if (ok) {
-        const float2 o1 = __ldg(tw + kHrTO1 + n1 * 16 + c);
 #pragma unroll
         for (int dd = 0; dd < 16; ++dd) {
             const int k2 = c + 16 * dd;
-            Y[((int64_t)k2 * kHrA + n1) * rows + row] = cmul(cmul(y[dd], o1), __ldg(tw + kHrTO2 + n1 * 16 + dd));
+            Y[((int64_t)k2 * kHrA + n1) * rows + row] = cmul(y[dd], __ldg(tw + kHrTO + n1 * kHrB + k2));
         }
     }
 }
@@ -377,11 +375,10 @@ __global__ void __launch_bounds__(kHrFwdTmaThreads, 2)
         for (int aa = 0; aa < 16; ++aa) y[bitrev(aa, 4)] = col[c * 16 + aa];
         fft_dit<16, false>(y);  // y[dd]: k2 = c + 16 dd
         if (ok) {
-            const float2 o1 = __ldg(tw + kHrTO1 + n1 * 16 + c);
 #pragma unroll
             for (int dd = 0; dd < 16; ++dd) {
                 const int k2 = c + 16 * dd;
-                Y[((int64_t)k2 * kHrA + n1) * rows + row] = cmul(cmul(y[dd], o1), __ldg(tw + kHrTO2 + n1 * 16 + dd));
+                Y[((int64_t)k2 * kHrA + n1) * rows + row] = cmul(y[dd], __ldg(tw + kHrTO + n1 * kHrB + k2));
             }
         }
         __syncthreads();  // exchange read before the next item writes it
