@@ -62,8 +62,14 @@ constexpr int kHrRowM = 2 * kHrColM + 4;  // mid: one row's two columns (pitch =
 constexpr int kHrFwdThreads = 512, kHrMidThreads = 32 * kHrRows2, kHrInvThreads = 512, kHrNormThreads = 128;
 constexpr size_t kHrFwdSmem = (size_t)kHrCG * kHrSP * 8;
 constexpr int kHrMidSP = kHrRows2 + 1;  // mid output staging pitch: [sel][m1][rows + pad], over the row area
+// one column's staging: m1 < 128, a gap of 8 float2 (so a lane pair's two
+// halves m1 and m1 + 128 fall on different banks), then m1 >= 128
+constexpr int kHrMidStageCol = kHrB * kHrMidSP + 8;
+__device__ __forceinline__ int hr_stage_idx(int sel, int m1, int r) {
+    return sel * kHrMidStageCol + m1 * kHrMidSP + (m1 >= kHrB / 2 ? 8 : 0) + r;
+}
 constexpr size_t kHrMidSmem = (size_t)kHrRows2 * kHrRowM * 8;
-static_assert((size_t)2 * kHrB * kHrMidSP <= (size_t)kHrRows2 * kHrRowM, "output staging fits the row area");
+static_assert((size_t)2 * kHrMidStageCol <= (size_t)kHrRows2 * kHrRowM, "output staging fits the row area");
 
 // Twiddle table (float2, built on the host in fp64); theta = exp(-i pi / N),
 // omega_R = exp(-2 pi i / R), phi = theta^2.
@@ -538,9 +544,8 @@ __global__ void __launch_bounds__(kHrMidThreads, 16 / kHrRows2) hr_mid_kernel(fl
     }
     __syncthreads();  // every warp is done with its row: the staging may overwrite them
     {
-        float2 *st = stage + (size_t)csel * kHrB * kHrMidSP + r8;
 #pragma unroll
-        for (int bq = 0; bq < 16; ++bq) st[(cal + 8 * (bq + 16 * ch)) * kHrMidSP] = out[bq];
+        for (int bq = 0; bq < 16; ++bq) stage[hr_stage_idx(csel, cal + 8 * (bq + 16 * ch), r8)] = out[bq];
     }
     __syncthreads();
     // W[k2][m1][row0 + r] over the first 256 slots of each k2 block of Y
@@ -548,7 +553,7 @@ __global__ void __launch_bounds__(kHrMidThreads, 16 / kHrRows2) hr_mid_kernel(fl
         const int r = e & (kHrRows2 - 1), m1 = (e / kHrRows2) & (kHrB - 1), sel = e / (kHrRows2 * kHrB);
         const int k2 = sel ? k2b : k2a;
         if (row0 + r < rows)
-            Y[((int64_t)k2 * kHrA + m1) * rows + row0 + r] = stage[((size_t)sel * kHrB + m1) * kHrMidSP + r];
+            Y[((int64_t)k2 * kHrA + m1) * rows + row0 + r] = stage[hr_stage_idx(sel, m1, r)];
     }
 }
 
